@@ -1,0 +1,130 @@
+"""Python binding of libfa.so (argument marshalling only).
+
+The names follow the C ABI in ``include/fa.h``: ``fa_fwd``,
+``fa_get_device_status`` and ``fa_status_string``.  ``attention_forward`` is
+the convenience call on torch tensors: it checks shapes, allocates O and the
+logsumexp with torch, and calls ``fa_fwd`` on the current CUDA stream.  Every
+step of the computation runs in the CUDA kernels of libfa.so; there is no other
+implementation behind this module.  If the library is missing, importing this
+module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfa.so")
+
+FA_OK = 0
+FA_ERR_NULL = -1
+FA_ERR_SHAPE = -2
+FA_ERR_HEADDIM = -3
+FA_ERR_GQA = -4
+FA_ERR_ALIGN = -5
+FA_ERR_ARCH = -6
+FA_ERR_LAUNCH = -7
+FA_ERR_DEVICE_TIMEOUT = -8
+FA_ERR_SEQLENS = -9
+
+EXPORTED = ("fa_fwd", "fa_get_device_status", "fa_status_string")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m exact_tiled_attention_32_b200.build` "
+        "(there is no fallback implementation)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_lib.fa_fwd.restype = ctypes.c_int
+_lib.fa_fwd.argtypes = [
+    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+    ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+    ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+]
+_lib.fa_get_device_status.restype = ctypes.c_int
+_lib.fa_get_device_status.argtypes = [ctypes.c_void_p]
+_lib.fa_status_string.restype = ctypes.c_char_p
+_lib.fa_status_string.argtypes = [ctypes.c_int]
+
+
+class FAError(RuntimeError):
+    def __init__(self, code: int, where: str = "fa_fwd"):
+        self.code = code
+        super().__init__(f"{where}: {fa_status_string(code)} ({code})")
+
+
+def _addr(x) -> int | None:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s) -> int | None:
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, cu_seqlens=None, stream=None) -> int:
+    """The C entry point; tensors or raw device addresses.  Returns the status."""
+    return _lib.fa_fwd(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), int(B), int(Hq),
+                       int(Hkv), int(N), int(d), float(scale), int(bool(causal)),
+                       _addr(cu_seqlens), _stream(stream))
+
+
+def fa_get_device_status(stream=None) -> int:
+    return _lib.fa_get_device_status(_stream(stream))
+
+
+def fa_status_string(code: int) -> str:
+    return _lib.fa_status_string(int(code)).decode()
+
+
+def attention_forward(q, k, v, *, causal: bool = False, scale: float | None = None,
+                      cu_seqlens=None, out=None, lse=None):
+    """O, lse = attention_forward(q, k, v) on bf16 CUDA tensors.
+
+    Dense: q [B, Hq, N, d], k/v [B, Hkv, N, d]; returns O [B, Hq, N, d] and
+    lse [B, Hq, N] (fp32).  Packed (``cu_seqlens`` int32 [B+1] on the device):
+    q [N, Hq, d], k/v [N, Hkv, d]; returns O [N, Hq, d] and lse [Hq, N].
+    """
+    import torch
+
+    if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+        raise TypeError("q, k, v must be bfloat16")
+    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+        raise ValueError("q, k, v must be CUDA tensors")
+    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    if cu_seqlens is None:
+        if q.dim() != 4 or k.shape != v.shape or k.dim() != 4:
+            raise ValueError("dense layout: q [B,Hq,N,d], k/v [B,Hkv,N,d]")
+        B, Hq, N, d = q.shape
+        Hkv = k.shape[1]
+        if k.shape[0] != B or k.shape[2] != N or k.shape[3] != d:
+            raise ValueError("k/v shape does not match q")
+        lse_shape = (B, Hq, N)
+    else:
+        if q.dim() != 3 or k.dim() != 3 or k.shape != v.shape:
+            raise ValueError("packed layout: q [N,Hq,d], k/v [N,Hkv,d]")
+        N, Hq, d = q.shape
+        Hkv = k.shape[1]
+        B = cu_seqlens.numel() - 1
+        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda:
+            raise ValueError("cu_seqlens must be an int32 CUDA tensor")
+        lse_shape = (Hq, N)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(lse_shape, dtype=torch.float32, device=q.device)
+    rc = fa_fwd(q, k, v, out, lse, B, Hq, Hkv, N, d, scale, causal, cu_seqlens,
+                torch.cuda.current_stream(q.device))
+    if rc != FA_OK:
+        raise FAError(rc)
+    return out, lse

@@ -1,0 +1,753 @@
+// fa_fwd.cu -- exact attention forward for B200 (sm_100a) and its C ABI.
+//
+// The method (pages: "Flash Attention", 14cs17.netlify.app -- "Tiling
+// Strategy", "Online Softmax" (Theorem 2), "Flash Attention Algorithm",
+// "Flash Attention 2 Improvements"): for each block Q_i of query rows, stream
+// the key/value blocks K_j, V_j through on-chip memory, form S_ij = Q_i K_j^T,
+// fold it into a running row maximum m, a running row sum l and an
+// unnormalised output O, and write only O / l (and the logsumexp) to HBM.
+//
+// B200 mapping (one persistent CTA per SM, 384 threads, warp-specialised):
+//   warp 9      TMA producer: Q_i (two 128-row tiles per work item) and a
+//               ring of K_j / V_j tiles in 128-byte-swizzled shared memory.
+//   warp 8      MMA issuer (one thread): S_t = Q_t K_j^T and O_t += P_t V_j as
+//               tcgen05.mma kind::f16 (bf16 in, fp32 accumulate in TMEM).  P_t
+//               is read straight from TMEM, where it overwrites S_t.
+//   warps 0-3   softmax for query tile 0, warps 4-7 for query tile 1: one
+//               thread per query row; tcgen05.ld of S, masking, running max in
+//               the log2 domain, exp2 via one FFMA + ex2, lazy rescale of O in
+//               TMEM (only when the max grows by more than 2^8), bf16 P written
+//               back to TMEM, and finally the epilogue O / l -> bf16 -> HBM plus
+//               the logsumexp.
+//   warps 10-11 idle (they complete the third warpgroup, which gives its
+//               registers to the softmax warpgroups through setmaxnreg).
+// The two query tiles ping-pong: while the softmax warps work on tile 0 the
+// tensor core runs tile 1's MMAs and vice versa.
+//
+// TMEM columns (512 allocated): S0/P0 [0,128), S1/P1 [128,256),
+// O0 [256, 256+D), O1 [384, 384+D).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "sm100_ptx.cuh"
+
+namespace fa_sm100 {
+
+constexpr int kBlockM = 128;           // query rows per tile (B_r)
+constexpr int kBlockN = 128;           // keys per tile (B_c)
+constexpr int kRowsPerItem = 2 * kBlockM;
+constexpr int kNumSoftmaxWarps = 8;
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp = 9;
+constexpr int kThreads = 384;
+constexpr uint32_t kSoftmaxRegs = 216;   // setmaxnreg split: 2 x 128 x 216 + 128 x 72 = 384 x 168
+constexpr uint32_t kOtherRegs = 72;
+constexpr int kMaxSeqs = 1024;         // packed batches: sequences
+constexpr int kMaxPairs = 1024;        // packed batches: 256-row pairs per sequence
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only past 2^8
+
+// where a wait gave up (reported in status[1])
+enum WaitSite : int {
+    kSiteQEmpty = 1, kSiteKvEmpty, kSiteQFull, kSiteKvFull, kSitePFull, kSiteSFull, kSiteOFinal,
+    kSiteDrain
+};
+
+struct alignas(64) Params {
+    CUtensorMap tm_q, tm_k, tm_v;
+    void* o;
+    float* lse;
+    const int32_t* cu_seqlens;
+    int* status;
+    int B, Hq, Hkv, N;
+    int group;                 // Hq / Hkv
+    int causal, packed;
+    float scale_log2;          // scale * log2(e)
+    unsigned long long timeout_ns;
+};
+
+struct Misc {
+    uint64_t bar_q_full, bar_q_empty, bar_drain;
+    uint64_t bar_kv_full[8], bar_kv_empty[8];
+    uint64_t bar_s_full[2], bar_p_full[2], bar_o_final[2];
+    uint32_t tmem_base;
+    int abort_flag;
+    int bad;
+    int total_items;
+    int pmax;
+    int seq_off[kMaxSeqs + 1];
+    int order[kMaxSeqs];       // sequences by pair count, descending
+    int pcnt[kMaxPairs];       // number of sequences with more than p pairs
+    int pstart[kMaxPairs];     // first item index at pair level p
+};
+
+template <int D>
+struct Cfg {
+    static_assert(D == 64 || D == 128, "head dim");
+    static constexpr int kTileBytes = kBlockM * D * 2;     // one 128 x D bf16 tile
+    static constexpr int kBoxBytes = kBlockM * 64 * 2;     // one 128 x 64 TMA box
+    static constexpr int kBoxes = D / 64;
+    static constexpr int kStages = (D == 128) ? 4 : 8;
+    static constexpr int kQOff = 0;
+    static constexpr int kKVOff = 2 * kTileBytes;
+    static constexpr int kMiscOff = kKVOff + kStages * kTileBytes;
+    static constexpr int kSmemBytes = kMiscOff + (int)sizeof(Misc) + 1024;
+};
+
+// One work item: two consecutive 128-row query tiles of one (sequence, head).
+struct Item {
+    int seq;       // batch index (dense) or sequence index (packed)
+    int h;         // query head
+    int q0;        // first row of tile 0 inside the sequence
+    int len;       // sequence length
+    int tok0;      // packed: first token of the sequence
+    int n[2];      // key blocks each tile visits (0: tile beyond the sequence)
+};
+
+__device__ __forceinline__ int tile_blocks(int q0, int len, int causal) {
+    if (q0 >= len) return 0;
+    const int nkv = (len + kBlockN - 1) / kBlockN;
+    return causal ? min(nkv, q0 / kBlockN + 1) : nkv;
+}
+
+// Items run in decreasing pair index (heaviest causal tiles first), then
+// sequence, then head, so that query heads sharing a key/value head run side
+// by side.
+__device__ __forceinline__ Item decode_item(int idx, const Params& p, const Misc& ms) {
+    Item it;
+    int pair;
+    if (!p.packed) {
+        const int npairs = (p.N + kRowsPerItem - 1) / kRowsPerItem;
+        const int per = p.B * p.Hq;
+        const int lvl = idx / per;
+        const int rem = idx - lvl * per;
+        pair = npairs - 1 - lvl;
+        it.seq = rem / p.Hq;
+        it.h = rem - it.seq * p.Hq;
+        it.len = p.N;
+        it.tok0 = 0;
+    } else {
+        int lo = 0, hi = ms.pmax - 1;      // smallest level whose start <= idx
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (ms.pstart[mid] <= idx) hi = mid; else lo = mid + 1;
+        }
+        pair = lo;
+        const int rem = idx - ms.pstart[lo];
+        const int k = rem / p.Hq;
+        it.h = rem - k * p.Hq;
+        it.seq = ms.order[k];
+        it.tok0 = ms.seq_off[it.seq];
+        it.len = ms.seq_off[it.seq + 1] - it.tok0;
+    }
+    it.q0 = pair * kRowsPerItem;
+    it.n[0] = tile_blocks(it.q0, it.len, p.causal);
+    it.n[1] = tile_blocks(it.q0 + kBlockM, it.len, p.causal);
+    return it;
+}
+
+// Static "snake" schedule over persistent CTAs: round r hands item
+// r*G + c to CTA c on even rounds and r*G + (G-1-c) on odd rounds, which
+// evens out the decreasing causal work between CTAs.
+__device__ __forceinline__ int item_of_round(int r) {
+    const int G = gridDim.x;
+    return r * G + ((r & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+}
+
+// Bounded wait: gives up after timeout_ns (recording the site in the status
+// word and raising the CTA's abort flag) or as soon as another role aborted.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Params& p, Misc& ms,
+                                      int site) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*reinterpret_cast<volatile int*>(&ms.abort_flag)) return false;
+        if (globaltimer_ns() - t0 > p.timeout_ns) {
+            *reinterpret_cast<volatile int*>(&ms.abort_flag) = 1;
+            if (atomicCAS(p.status, 0, FA_ERR_DEVICE_TIMEOUT) == 0) {
+                p.status[1] = site;
+                p.status[2] = blockIdx.x;
+            }
+            return false;
+        }
+    }
+}
+// Teardown wait: ignores the abort flag, still bounded.
+__device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, const Params& p) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > p.timeout_ns) return;
+    }
+}
+
+// ---------------------------------------------------------------- producer
+template <int D>
+__device__ void load_role(const Params& p, Misc& ms, uint32_t smem_q, uint32_t smem_kv, int total) {
+    using C = Cfg<D>;
+    const uint64_t pol_kv = policy_evict_last();
+    const uint64_t pol_q = policy_evict_first();
+    uint32_t kv_it = 0, item_n = 0;
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+        const int idx = item_of_round(r);
+        if (idx >= total) break;
+        const Item it = decode_item(idx, p, ms);
+        // both query tiles of the item
+        if (!(ok = wait_bar(smem_u32(&ms.bar_q_empty), (item_n & 1) ^ 1, p, ms, kSiteQEmpty))) break;
+        const uint32_t qbar = smem_u32(&ms.bar_q_full);
+        mbar_arrive_expect_tx(qbar, 2 * C::kTileBytes);
+        for (int t = 0; t < 2; ++t) {
+            const int row = it.q0 + t * kBlockM;
+            for (int b = 0; b < C::kBoxes; ++b) {
+                const uint32_t dst = smem_q + t * C::kTileBytes + b * C::kBoxBytes;
+                if (!p.packed)
+                    tma_load_4d(dst, &p.tm_q, qbar, b * 64, row, it.h, it.seq, pol_q);
+                else
+                    tma_load_4d(dst, &p.tm_q, qbar, b * 64, it.h, it.tok0 + row, 0, pol_q);
+            }
+        }
+        ++item_n;
+        const int kvh = it.h / p.group;
+        const int nmax = max(it.n[0], it.n[1]);
+        for (int j = 0; j < nmax && ok; ++j) {
+            for (int kind = 0; kind < 2; ++kind) {       // K_j then V_j
+                const uint32_t st = kv_it % C::kStages;
+                if (!(ok = wait_bar(smem_u32(&ms.bar_kv_empty[st]), ((kv_it / C::kStages) & 1) ^ 1, p,
+                                    ms, kSiteKvEmpty)))
+                    break;
+                const uint32_t bar = smem_u32(&ms.bar_kv_full[st]);
+                mbar_arrive_expect_tx(bar, C::kTileBytes);
+                const CUtensorMap* map = kind == 0 ? &p.tm_k : &p.tm_v;
+                for (int b = 0; b < C::kBoxes; ++b) {
+                    const uint32_t dst = smem_kv + st * C::kTileBytes + b * C::kBoxBytes;
+                    if (!p.packed)
+                        tma_load_4d(dst, map, bar, b * 64, j * kBlockN, kvh, it.seq, pol_kv);
+                    else
+                        tma_load_4d(dst, map, bar, b * 64, kvh, it.tok0 + j * kBlockN, 0, pol_kv);
+                }
+                ++kv_it;
+            }
+        }
+    }
+    if (!ok) {
+        // let the copies already issued land before the CTA goes away
+        if (item_n > 0) drain_bar(smem_u32(&ms.bar_q_full), (item_n - 1) & 1, p);
+        const uint32_t first = kv_it > (uint32_t)C::kStages ? kv_it - C::kStages : 0;
+        for (uint32_t i = first; i < kv_it; ++i)
+            drain_bar(smem_u32(&ms.bar_kv_full[i % C::kStages]), (i / C::kStages) & 1, p);
+    }
+}
+
+// ------------------------------------------------------------- MMA issuer
+template <int D>
+__device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_addr, uint32_t k_addr) {
+    constexpr uint32_t idesc = idesc_bf16_f32(kBlockM, kBlockN, false);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk / 4) * Cfg<D>::kBoxBytes + (kk % 4) * 32;
+        umma_ss(tmem_s, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
+                idesc, kk > 0 ? 1u : 0u);
+    }
+}
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_addr, bool accumulate) {
+    constexpr uint32_t idesc = idesc_bf16_f32(kBlockM, D, true);
+#pragma unroll
+    for (int kk = 0; kk < kBlockN / 16; ++kk) {
+        umma_ts(tmem_o, tmem_p + kk * 8, smem_desc_sw128(v_addr + kk * 16 * 128, Cfg<D>::kBoxBytes, 1024),
+                idesc, (accumulate || kk > 0) ? 1u : 0u);
+    }
+}
+
+template <int D>
+__device__ void mma_role(const Params& p, Misc& ms, uint32_t tmem, uint32_t smem_q, uint32_t smem_kv,
+                         int total) {
+    using C = Cfg<D>;
+    uint32_t kv_it = 0, item_n = 0;
+    uint32_t pc[2] = {0, 0};
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+        const int idx = item_of_round(r);
+        if (idx >= total) break;
+        const Item it = decode_item(idx, p, ms);
+        if (!(ok = wait_bar(smem_u32(&ms.bar_q_full), item_n & 1, p, ms, kSiteQFull))) break;
+        tc_fence_after();
+        ++item_n;
+        const int nmax = max(it.n[0], it.n[1]);
+        const uint32_t base = kv_it;
+        for (int j = 0; j < nmax && ok; ++j) {
+            const uint32_t kit = base + 2 * j;
+            const uint32_t kst = kit % C::kStages;
+            if (!(ok = wait_bar(smem_u32(&ms.bar_kv_full[kst]), (kit / C::kStages) & 1, p, ms, kSiteKvFull)))
+                break;
+            const uint32_t vit = kit - 1;
+            const uint32_t vst = vit % C::kStages;
+            if (j > 0 &&
+                !(ok = wait_bar(smem_u32(&ms.bar_kv_full[vst]), (vit / C::kStages) & 1, p, ms, kSiteKvFull)))
+                break;
+            tc_fence_after();
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                if (!ok) break;
+                if (j > 0 && j - 1 < it.n[t]) {          // O_t += P_t V_{j-1}
+                    if (!(ok = wait_bar(smem_u32(&ms.bar_p_full[t]), pc[t] & 1, p, ms, kSitePFull))) break;
+                    ++pc[t];
+                    tc_fence_after();
+                    issue_pv<D>(tmem + 256 + t * 128, tmem + t * 128, smem_kv + vst * C::kTileBytes, j - 1 > 0);
+                    if (j - 1 == it.n[t] - 1) umma_commit(smem_u32(&ms.bar_o_final[t]));
+                }
+                if (j < it.n[t]) {                       // S_t = Q_t K_j^T
+                    issue_qk<D>(tmem + t * 128, smem_q + t * C::kTileBytes, smem_kv + kst * C::kTileBytes);
+                    umma_commit(smem_u32(&ms.bar_s_full[t]));
+                }
+            }
+            if (!ok) break;
+            umma_commit(smem_u32(&ms.bar_kv_empty[kst]));
+            if (j > 0) umma_commit(smem_u32(&ms.bar_kv_empty[vst]));
+            if (j == nmax - 1) umma_commit(smem_u32(&ms.bar_q_empty));
+        }
+        if (!ok) break;
+        // last value block
+        const uint32_t vit = base + 2 * nmax - 1;
+        const uint32_t vst = vit % C::kStages;
+        if (!(ok = wait_bar(smem_u32(&ms.bar_kv_full[vst]), (vit / C::kStages) & 1, p, ms, kSiteKvFull))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            if (!ok || it.n[t] != nmax) continue;
+            if (!(ok = wait_bar(smem_u32(&ms.bar_p_full[t]), pc[t] & 1, p, ms, kSitePFull))) break;
+            ++pc[t];
+            tc_fence_after();
+            issue_pv<D>(tmem + 256 + t * 128, tmem + t * 128, smem_kv + vst * C::kTileBytes, nmax - 1 > 0);
+            umma_commit(smem_u32(&ms.bar_o_final[t]));
+        }
+        if (!ok) break;
+        umma_commit(smem_u32(&ms.bar_kv_empty[vst]));
+        kv_it = base + 2 * nmax;
+    }
+    // every MMA issued so far must be finished before TMEM and smem go away
+    umma_commit(smem_u32(&ms.bar_drain));
+    drain_bar(smem_u32(&ms.bar_drain), 0, p);
+}
+
+// ---------------------------------------------------------------- softmax
+template <int D>
+__device__ void softmax_role(const Params& p, Misc& ms, uint32_t tmem, int warp, int lane, int total) {
+    const int t = warp / 4;                          // query tile of this warpgroup
+    const int wq = warp % 4;                         // TMEM lane quarter
+    const int r = wq * 32 + lane;                    // row inside the tile
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t taddr_s = tmem + lane_off + t * 128;
+    const uint32_t taddr_o = tmem + lane_off + 256 + t * 128;
+    const float sl2 = p.scale_log2;
+    uint32_t sc = 0, oc = 0;
+    bool ok = true;
+    for (int rr = 0; ok; ++rr) {
+        const int idx = item_of_round(rr);
+        if (idx >= total) break;
+        const Item it = decode_item(idx, p, ms);
+        const int n = t ? it.n[1] : it.n[0];
+        if (n == 0) continue;
+        const int row = it.q0 + t * kBlockM + r;
+        const int limit = p.causal ? min(row + 1, it.len) : it.len;   // keys [0, limit) allowed
+        float m_used = -INFINITY;    // max the exponentials are taken against (log2 units)
+        float l = 0.f;               // running sum of exp2(x - m_used)
+        for (int j = 0; j < n; ++j) {
+            ok = wait_bar(smem_u32(&ms.bar_s_full[t]), sc & 1, p, ms, kSiteSFull);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            ++sc;
+            tc_fence_after();
+            uint32_t s[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32_sync(taddr_s + c * 32, s[c]);
+            if (j * kBlockN + kBlockN > limit) {      // diagonal or tail block
+                const int lim = limit - j * kBlockN;
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (c * 32 + i >= lim) s[c][i] = __float_as_uint(-INFINITY);
+            }
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(s[c][i]));
+            const float m_new = fmaxf(m_used, mx * sl2);
+            const bool need = m_new > m_used + kRescaleThreshold;
+            if (j > 0 && __any_sync(0xffffffffu, need)) {
+                // Theorem 2: rescale the partial output when the max grows
+                const float f = need ? ex2_approx(m_used - m_new) : 1.f;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32_sync(taddr_o + c * 32, o);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+                    tmem_st32(taddr_o + c * 32, o);
+                }
+                tmem_wait_st();
+            }
+            if (need) {
+                l *= (m_used == -INFINITY) ? 0.f : ex2_approx(m_used - m_new);
+                m_used = m_new;
+            }
+            const float msub = (m_used == -INFINITY) ? 0.f : m_used;
+            float rs = 0.f;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const uint32_t* sv = s[2 * half + i / 16];
+                    const float a = ex2_approx(fmaf(__uint_as_float(sv[(2 * i) % 32]), sl2, -msub));
+                    const float b = ex2_approx(fmaf(__uint_as_float(sv[(2 * i + 1) % 32]), sl2, -msub));
+                    rs += a + b;
+                    pk[i] = pack_bf16x2(a, b);
+                }
+                tmem_st32(taddr_s + half * 32, pk);
+            }
+            l += rs;
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ms.bar_p_full[t]));
+        }
+        if (!ok) break;
+        // epilogue: O / l -> bf16 -> HBM, and the logsumexp
+        ok = wait_bar(smem_u32(&ms.bar_o_final[t]), oc & 1, p, ms, kSiteOFinal);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        ++oc;
+        tc_fence_after();
+        const bool valid = row < it.len;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        uint16_t* orow;
+        float* lrow;
+        if (!p.packed) {
+            const size_t rid = (static_cast<size_t>(it.seq) * p.Hq + it.h) * p.N + row;
+            orow = static_cast<uint16_t*>(p.o) + rid * D;
+            lrow = p.lse + rid;
+        } else {
+            const size_t tok = static_cast<size_t>(it.tok0) + row;
+            orow = static_cast<uint16_t*>(p.o) + (tok * p.Hq + it.h) * D;
+            lrow = p.lse + static_cast<size_t>(it.h) * p.N + tok;
+        }
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32_sync(taddr_o + c * 32, o);
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+            if (valid) {
+                uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
+        }
+        if (valid) {
+            float lg;
+            asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg) : "f"(l));
+            *lrow = (l > 0.f) ? (m_used + lg) * 0.69314718055994531f : -INFINITY;
+        }
+        tc_fence_before();
+    }
+}
+
+// ------------------------------------------------------------------ kernel
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_constant__ Params p) {
+    using C = Cfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Misc& ms = *reinterpret_cast<Misc*>(smem + C::kMiscOff);
+    const int tid = threadIdx.x;
+    const int warp = tid / 32, lane = tid % 32;
+    const uint32_t smem_q = smem_u32(smem + C::kQOff);
+    const uint32_t smem_kv = smem_u32(smem + C::kKVOff);
+
+    if (tid == 0) {
+        mbar_init(smem_u32(&ms.bar_q_full), 1);
+        mbar_init(smem_u32(&ms.bar_q_empty), 1);
+        mbar_init(smem_u32(&ms.bar_drain), 1);
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(smem_u32(&ms.bar_kv_full[s]), 1);
+            mbar_init(smem_u32(&ms.bar_kv_empty[s]), 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(smem_u32(&ms.bar_s_full[t]), 1);
+            mbar_init(smem_u32(&ms.bar_p_full[t]), 4);
+            mbar_init(smem_u32(&ms.bar_o_final[t]), 1);
+        }
+        ms.abort_flag = 0;
+        ms.bad = 0;
+        fence_mbar_init();
+    }
+    if (warp == kLoadWarp && lane == 0) {
+        prefetch_tensormap(&p.tm_q);
+        prefetch_tensormap(&p.tm_k);
+        prefetch_tensormap(&p.tm_v);
+    }
+
+    int total;
+    if (p.packed) {
+        // stage the offsets, check them, and build the pair-level tables
+        for (int i = tid; i <= p.B; i += kThreads) ms.seq_off[i] = p.cu_seqlens[i];
+        __syncthreads();
+        if (tid == 0) {
+            int bad = ms.seq_off[0] != 0 || ms.seq_off[p.B] != p.N;
+            for (int s = 0; s < p.B && !bad; ++s) {
+                const int L = ms.seq_off[s + 1] - ms.seq_off[s];
+                if (L < 0 || L > kMaxPairs * kRowsPerItem) bad = 1;
+            }
+            ms.bad = bad;
+        }
+        __syncthreads();
+        if (ms.bad) {
+            if (tid == 0 && blockIdx.x == 0) atomicCAS(p.status, 0, FA_ERR_SEQLENS);
+            return;
+        }
+        for (int s = tid; s < p.B; s += kThreads) {
+            const int ps = (ms.seq_off[s + 1] - ms.seq_off[s] + kRowsPerItem - 1) / kRowsPerItem;
+            int rank = 0;
+            for (int u = 0; u < p.B; ++u) {
+                const int pu = (ms.seq_off[u + 1] - ms.seq_off[u] + kRowsPerItem - 1) / kRowsPerItem;
+                rank += (pu > ps) || (pu == ps && u < s);
+            }
+            ms.order[rank] = s;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            auto pairs_of = [&](int s) {
+                return (ms.seq_off[s + 1] - ms.seq_off[s] + kRowsPerItem - 1) / kRowsPerItem;
+            };
+            const int pmax = p.B > 0 ? pairs_of(ms.order[0]) : 0;
+            int k = p.B;
+            for (int lvl = 0; lvl < pmax; ++lvl) {
+                while (k > 0 && pairs_of(ms.order[k - 1]) <= lvl) --k;
+                ms.pcnt[lvl] = k;
+            }
+            int acc = 0;
+            for (int lvl = pmax - 1; lvl >= 0; --lvl) {
+                ms.pstart[lvl] = acc;
+                acc += ms.pcnt[lvl] * p.Hq;
+            }
+            ms.pmax = pmax;
+            ms.total_items = acc;
+        }
+    }
+
+    if (warp == kMmaWarp) {
+        tmem_alloc(smem_u32(&ms.tmem_base), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ms.tmem_base;
+    if (p.packed) {
+        total = ms.total_items;
+    } else {
+        total = ((p.N + kRowsPerItem - 1) / kRowsPerItem) * p.B * p.Hq;
+    }
+
+    if (warp < kNumSoftmaxWarps) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+        softmax_role<D>(p, ms, tmem, warp, lane, total);
+    } else {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
+    }
+    if (warp < kNumSoftmaxWarps) {
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) mma_role<D>(p, ms, tmem, smem_q, smem_kv, total);
+        __syncwarp();
+    } else if (warp == kLoadWarp) {
+        if (lane == 0) load_role<D>(p, ms, smem_q, smem_kv, total);
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// =================================================================== host
+struct DeviceState {
+    bool init = false;
+    int status_code = FA_OK;
+    int num_sms = 0;
+    int* status = nullptr;        // device: [0] code, [1] wait site, [2] block
+};
+
+constexpr int kMaxDevices = 64;
+static DeviceState g_dev[kMaxDevices];
+static std::mutex g_mu;
+static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+static int init_device(int dev, DeviceState** out) {
+    if (dev < 0 || dev >= kMaxDevices) return FA_ERR_LAUNCH;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState& ds = g_dev[dev];
+    if (!ds.init) {
+        ds.init = true;
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+            ds.status_code = FA_ERR_LAUNCH;
+        } else if (prop.major != 10 || prop.minor != 0) {
+            ds.status_code = FA_ERR_ARCH;
+        } else {
+            ds.num_sms = prop.multiProcessorCount;
+            if (!g_encode) {
+                cudaDriverEntryPointQueryResult q;
+                void* fn = nullptr;
+                if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                        cudaSuccess &&
+                    q == cudaDriverEntryPointSuccess)
+                    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+            }
+            bool good = g_encode != nullptr;
+            good = good && cudaMalloc(&ds.status, 4 * sizeof(int)) == cudaSuccess;
+            good = good && cudaMemset(ds.status, 0, 4 * sizeof(int)) == cudaSuccess;
+            good = good && cudaFuncSetAttribute(fa_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                Cfg<64>::kSmemBytes) == cudaSuccess;
+            good = good && cudaFuncSetAttribute(fa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                Cfg<128>::kSmemBytes) == cudaSuccess;
+            ds.status_code = good ? FA_OK : FA_ERR_LAUNCH;
+        }
+    }
+    *out = &ds;
+    return ds.status_code;
+}
+
+// 4-D bf16 tensor map with a 64 x rows box, 128-byte swizzle.
+static bool encode_map(CUtensorMap* m, const void* base, const uint64_t dims[4], const uint64_t strides[3],
+                       const uint32_t box[4]) {
+    const cuuint32_t elem[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+                          elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+static bool make_maps(Params& P, const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int N,
+                      int d, bool packed) {
+    const uint64_t e = 2;
+    if (!packed) {
+        const uint64_t dq[4] = {(uint64_t)d, (uint64_t)N, (uint64_t)Hq, (uint64_t)B};
+        const uint64_t sq[3] = {d * e, (uint64_t)N * d * e, (uint64_t)Hq * N * d * e};
+        const uint64_t dk[4] = {(uint64_t)d, (uint64_t)N, (uint64_t)Hkv, (uint64_t)B};
+        const uint64_t sk[3] = {d * e, (uint64_t)N * d * e, (uint64_t)Hkv * N * d * e};
+        const uint32_t box[4] = {64, (uint32_t)kBlockM, 1, 1};
+        return encode_map(&P.tm_q, q, dq, sq, box) && encode_map(&P.tm_k, k, dk, sk, box) &&
+               encode_map(&P.tm_v, v, dk, sk, box);
+    }
+    const uint64_t dq[4] = {(uint64_t)d, (uint64_t)Hq, (uint64_t)N, 1};
+    const uint64_t sq[3] = {d * e, (uint64_t)Hq * d * e, (uint64_t)N * Hq * d * e};
+    const uint64_t dk[4] = {(uint64_t)d, (uint64_t)Hkv, (uint64_t)N, 1};
+    const uint64_t sk[3] = {d * e, (uint64_t)Hkv * d * e, (uint64_t)N * Hkv * d * e};
+    const uint32_t box[4] = {64, 1, (uint32_t)kBlockM, 1};
+    return encode_map(&P.tm_q, q, dq, sq, box) && encode_map(&P.tm_k, k, dk, sk, box) &&
+           encode_map(&P.tm_v, v, dk, sk, box);
+}
+
+static bool aligned(const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) == 0; }
+
+}  // namespace fa_sm100
+
+using namespace fa_sm100;
+
+extern "C" int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                      int N, int d, float scale, int causal, const int32_t* cu_seqlens, void* stream) {
+    const bool packed = cu_seqlens != nullptr;
+    if (B < 0 || N < 0 || Hq < 1) return FA_ERR_SHAPE;
+    if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+    if (Hkv < 1 || Hq % Hkv != 0) return FA_ERR_GQA;
+    if (B == 0 || N == 0) return FA_OK;
+    if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+        return FA_ERR_ALIGN;
+    if (packed && (B > kMaxSeqs || !aligned(cu_seqlens, 4))) return B > kMaxSeqs ? FA_ERR_SHAPE : FA_ERR_ALIGN;
+    // row ids and item counts must fit in int
+    const long long rows = packed ? (long long)Hq * N : (long long)B * Hq * N;
+    if (rows > (1ll << 30)) return FA_ERR_SHAPE;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_LAUNCH;
+    DeviceState* ds = nullptr;
+    const int st = init_device(dev, &ds);
+    if (st != FA_OK) return st;
+
+    Params P;
+    std::memset(&P, 0, sizeof(P));
+    if (!make_maps(P, q, k, v, B, Hq, Hkv, N, d, packed)) return FA_ERR_LAUNCH;
+    P.o = o;
+    P.lse = lse;
+    P.cu_seqlens = cu_seqlens;
+    P.status = ds->status;
+    P.B = B;
+    P.Hq = Hq;
+    P.Hkv = Hkv;
+    P.N = N;
+    P.group = Hq / Hkv;
+    P.causal = causal ? 1 : 0;
+    P.packed = packed ? 1 : 0;
+    P.scale_log2 = scale * 1.4426950408889634f;
+    P.timeout_ns = 2000000000ull;
+
+    long long items;
+    if (!packed) {
+        items = (long long)((N + kRowsPerItem - 1) / kRowsPerItem) * B * Hq;
+    } else {
+        items = (long long)ds->num_sms;    // exact count is known only on the device
+    }
+    const int grid = (int)std::min<long long>(items, ds->num_sms);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (d == 64)
+        fa_fwd_kernel<64><<<grid, kThreads, Cfg<64>::kSmemBytes, s>>>(P);
+    else
+        fa_fwd_kernel<128><<<grid, kThreads, Cfg<128>::kSmemBytes, s>>>(P);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+extern "C" int fa_get_device_status(void* stream) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_LAUNCH;
+    DeviceState* ds = nullptr;
+    const int st = init_device(dev, &ds);
+    if (st != FA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int h[4] = {0, 0, 0, 0};
+    if (cudaMemcpyAsync(h, ds->status, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess) return FA_ERR_LAUNCH;
+    if (cudaMemsetAsync(ds->status, 0, sizeof(h), s) != cudaSuccess) return FA_ERR_LAUNCH;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return FA_ERR_LAUNCH;
+    return h[0];
+}
+
+extern "C" const char* fa_status_string(int status) {
+    switch (status) {
+        case FA_OK: return "ok";
+        case FA_ERR_NULL: return "a required pointer is NULL";
+        case FA_ERR_SHAPE: return "a size is negative or out of the supported range";
+        case FA_ERR_HEADDIM: return "head dimension must be 64 or 128";
+        case FA_ERR_GQA: return "Hq must be a positive multiple of Hkv";
+        case FA_ERR_ALIGN: return "q, k, v, o must be 16-byte aligned and lse 4-byte aligned";
+        case FA_ERR_ARCH: return "current device is not compute capability 10.0 (B200)";
+        case FA_ERR_LAUNCH: return "CUDA launch or runtime error";
+        case FA_ERR_DEVICE_TIMEOUT: return "device watchdog: a pipeline wait timed out";
+        case FA_ERR_SEQLENS: return "cu_seqlens inconsistent with B and N";
+        default: return "unknown status";
+    }
+}

@@ -1,0 +1,99 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact attention forward library
+ * (libfa.so).
+ *
+ * The operation: exact attention O = softmax(scale * Q K^T) V together with
+ * the per-row logsumexp, computed tile by tile with the online-softmax running
+ * maximum and running sum so that the score and probability matrices never
+ * reach device memory.  Pages: "Flash Attention" (14cs17.netlify.app),
+ * sections "Tiling Strategy", "Online Softmax" (Theorem 2) and "Flash
+ * Attention Algorithm"; the problem statement there is Q, K, V in R^{N x d}
+ * and softmax(QK^T)V.  "Flash Attention 2 Improvements" on the same page adds
+ * the variable sequence lengths and grouped-query attention supported here.
+ *
+ * All entry points are plain C: pointers, sizes, and an opaque stream handle.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes.  Every entry point returns FA_OK (0) or a negative code. */
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_NULL = -1,            /* a required pointer is NULL                        */
+    FA_ERR_SHAPE = -2,           /* a size is negative or out of the supported range  */
+    FA_ERR_HEADDIM = -3,         /* d is not 64 or 128                                */
+    FA_ERR_GQA = -4,             /* Hkv < 1 or Hq is not a multiple of Hkv            */
+    FA_ERR_ALIGN = -5,           /* q, k, v or o not 16-byte aligned, lse not 4-byte  */
+    FA_ERR_ARCH = -6,            /* current device is not compute capability 10.0     */
+    FA_ERR_LAUNCH = -7,          /* the CUDA runtime refused the launch (or no device)*/
+    FA_ERR_DEVICE_TIMEOUT = -8,  /* device watchdog: a pipeline wait ran out          */
+    FA_ERR_SEQLENS = -9          /* cu_seqlens inconsistent (found on the device)     */
+} fa_status;
+
+/*
+ * fa_fwd -- attention forward, asynchronous on `stream`.
+ *
+ *   q, k, v     bf16 inputs (device memory, read only).
+ *   o           bf16 output (device memory), same layout as q.
+ *   lse         fp32 output (device memory): natural-log logsumexp of each
+ *               row of scale * Q K^T over its allowed keys; -inf for a row
+ *               with no allowed key (its O row is then 0).
+ *   B           dense: batch size.  Packed: number of sequences.
+ *   Hq, Hkv     query heads and key/value heads; Hq % Hkv == 0.  Query head h
+ *               reads key/value head h / (Hq / Hkv).
+ *   N           dense: sequence length.  Packed: total tokens (must equal
+ *               cu_seqlens[B]).
+ *   d           head dimension, 64 or 128.
+ *   scale       multiplies Q K^T before the softmax (1/sqrt(d) is usual).
+ *   causal      nonzero: key j is allowed for query i iff j <= i, positions
+ *               counted inside the row's own sequence.
+ *   cu_seqlens  NULL for a dense batch.  Otherwise device memory holding B+1
+ *               int32 offsets, cu_seqlens[0] = 0, non-decreasing; sequence s
+ *               owns tokens [cu_seqlens[s], cu_seqlens[s+1]).
+ *   stream      a cudaStream_t (NULL = legacy default stream).
+ *
+ * Layouts (all contiguous, row-major):
+ *   dense   q, o [B, Hq, N, d]   k, v [B, Hkv, N, d]   lse [B, Hq, N]
+ *   packed  q, o [N, Hq, d]      k, v [N, Hkv, d]      lse [Hq, N]
+ *
+ * Limits: packed batches hold at most 1024 sequences, each at most 262144
+ * tokens long (FA_ERR_SHAPE / device FA_ERR_SEQLENS otherwise).  B == 0 or
+ * N == 0 is an empty problem: FA_OK, nothing is launched and the pointers
+ * may be NULL.
+ *
+ * Ownership: the caller owns every buffer.  The library allocates only a
+ * small per-device status word, once, on the first call on that device.
+ *
+ * Errors: argument errors are found on the host before any launch and return
+ * the codes above.  Errors found on the device (a pipeline wait that ran past
+ * its time limit, inconsistent cu_seqlens) do not abort the context: the
+ * kernel records a code in the device status word and returns; read it with
+ * fa_get_device_status().
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+           int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+           const int32_t* cu_seqlens, void* stream);
+
+/*
+ * fa_get_device_status -- reads and clears the status word of the current
+ * device.  Synchronises `stream` (a cudaStream_t) first, so it reports every
+ * fa_fwd launched on that stream before the call.  Returns FA_OK, a negative
+ * device-side code (FA_ERR_DEVICE_TIMEOUT, FA_ERR_SEQLENS), or FA_ERR_LAUNCH
+ * if the runtime reports an error.
+ */
+int fa_get_device_status(void* stream);
+
+/* fa_status_string -- static, human-readable text for a status code. */
+const char* fa_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */
