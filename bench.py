@@ -1,0 +1,398 @@
+#!/usr/bin/env python
+"""Benchmark of the exact attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config c3] [--impl ours|reference]
+
+A step is one fa_fwd call over the whole workload (default: causal B=1, H=32,
+N=16384, d=128, the configuration the throughput target is quoted on).  The
+inputs are seeded synthetic bf16 N(0,1) tensors already resident in HBM; they
+are 384 MiB, larger than the 126 MiB L2, so no flush runs between steps.  With
+N > 1 GPUs (one process each, launched by torch.distributed.run) every rank
+solves its own independent problem of the same shape: there is no exchange step
+in the attention forward, so no data-path collective exists and the scaling is
+weak; the timing is the maximum over ranks.
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle
+on the host cores instead (rank 0 only), each step a bounded sample of the same
+workload's query rows.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd TFLOP/s (bf16) and % of B200 dense BF16 tensor peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAK_TFLOPS = 1590.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="c3")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU time budget of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def workload_desc(w):
+    if w.packed:
+        shape = f"packed {w.B} sequences (lengths {min(w.seqlens)}..{max(w.seqlens)}), H={w.Hq}"
+    else:
+        shape = f"B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N}"
+    return f"{w.name}: {'causal' if w.causal else 'non-causal'} {shape} d={w.d}, bf16 N(0,1), scale=1/sqrt(d)"
+
+
+def config_dict(w, extra=None):
+    c = {
+        "workload": workload_desc(w),
+        "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
+        "seed": w.seed, "flops_per_step": w.flops(),
+        "l2": "inputs larger than L2 (no flush between steps)",
+    }
+    if w.packed:
+        c["seqlens"] = list(w.seqlens)
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ----------------------------------------------------------------- peaks
+def load_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["bf16_tflops"]), float(pk.get("bf16_tflops_sustained", 0)) or None, "measured"
+    except Exception:
+        return FALLBACK_PEAK_TFLOPS, None, "fallback"
+
+
+def source_sha():
+    h = hashlib.sha256()
+    for rel in ("exact_tiled_attention_32_b200/csrc/fa_fwd.cu", "exact_tiled_attention_32_b200/csrc/sm100_ptx.cuh"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(config_name):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "fa_fwd_kernel_traffic.md")
+    if not os.path.exists(path):
+        return None
+    sha = source_sha()
+    for line in open(path):
+        m = re.match(r"\|\s*(\w+)\s*\|\s*([0-9a-f]{16})\s*\|\s*([0-9.eE+]+)\s*\|", line)
+        if m and m.group(1) == config_name and m.group(2) == sha:
+            return float(m.group(3))
+    return None
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons, tagged with host time."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.samples = []
+        self.proc = None
+        self.gpu_id = gpu_id
+        self.thread = None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.gpu_id:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 7:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        inside = [p for (t, p) in self.samples if t0 <= t <= t1]
+        if not inside:        # short timed region: nearest samples after it started
+            inside = [p for (t, p) in self.samples if t >= t0][:3]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = sorted(v for v in (num(p[0]) for p in inside) if v is not None)
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for p in inside for i in range(4) if p[3 + i].lower() == "active"})
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": num(inside[0][1]),
+                "reasons": reasons, "samples": len(inside),
+                "power_w_max": max((num(p[2]) or 0) for p in inside)}
+
+
+# ------------------------------------------------------------ CPU oracle
+def oracle_sample_rows(w, nrows, rng):
+    """Random query rows of the workload (all heads, all positions)."""
+    import numpy as np
+    rows = rng.integers(0, w.total_rows(), nrows)
+    return np.unique(rows)
+
+
+def row_flops(w, rows):
+    """4*d*(keys attended) per sampled row: the per-row share of the metric's
+    4*N^2*d (halved when causal)."""
+    import numpy as np
+    if w.packed:
+        tok = rows % w.N
+        cu = w.cu_seqlens
+        s = np.searchsorted(cu, tok, side="right") - 1
+        t = tok - cu[s]
+        L = cu[s + 1] - cu[s]
+    else:
+        t = rows % w.N
+        L = np.full_like(t, w.N)
+    keys = (t + 1) if w.causal else L
+    return float(np.sum(4.0 * w.d * keys))
+
+
+def time_oracle(w, seconds, seed=0):
+    """Times the oracle on random row samples until ``seconds`` have passed."""
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(seed)
+    flops = 0.0
+    rows_done = 0
+    t0 = time.perf_counter()
+    while True:
+        rows = oracle_sample_rows(w, 64, rng)
+        oracle.attention(w.q, w.k, w.v, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal,
+                         w.cu_seqlens, rows=rows)
+        flops += row_flops(w, rows)
+        rows_done += len(rows)
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{rows_done} random query rows of the workload (fp64, materialised score rows), "
+                      f"{dt:.1f} s on the host cores"}
+
+
+def run_reference(args, rank):
+    """--impl reference: the oracle timed on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    from exact_tiled_attention_32_b200 import synthetic as syn
+    w = syn.config(args.config).draw()
+    rng = np.random.default_rng(1)
+    nrows = 32
+    for _ in range(args.warmup):
+        oracle.attention(w.q, w.k, w.v, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal,
+                         w.cu_seqlens, rows=oracle_sample_rows(w, nrows, rng))
+    flops = 0.0
+    rows_done = 0
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        rows = oracle_sample_rows(w, nrows, rng)
+        oracle.attention(w.q, w.k, w.v, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal,
+                         w.cu_seqlens, rows=rows)
+        flops += row_flops(w, rows)
+        rows_done += len(rows)
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / max(args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": config_dict(w, {"step": f"{nrows} random query rows per step"}),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"{rows_done} random query rows over {args.steps} steps"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------- GPU path
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from exact_tiled_attention_32_b200 import binding as fa
+    from exact_tiled_attention_32_b200 import synthetic as syn
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    w = syn.config(args.config)
+    w.seed += rank              # independent problem per rank
+    w.draw()
+    q = torch.from_numpy(w.q.view(np.int16)).view(torch.bfloat16).to(dev)
+    k = torch.from_numpy(w.k.view(np.int16)).view(torch.bfloat16).to(dev)
+    v = torch.from_numpy(w.v.view(np.int16)).view(torch.bfloat16).to(dev)
+    cu = None if w.cu_seqlens is None else torch.from_numpy(w.cu_seqlens).to(dev)
+    o = torch.empty_like(q)
+    lse_shape = (w.Hq, w.N) if w.packed else (w.B, w.Hq, w.N)
+    lse = torch.empty(lse_shape, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        rc = fa.fa_fwd(q, k, v, o, lse, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal, cu, stream)
+        if rc != 0:
+            raise fa.FAError(rc)
+
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.3)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    t_host0 = time.time()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    ev1.synchronize()
+    torch.cuda.synchronize(dev)
+    t_host1 = time.time()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        dist.barrier()
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    sampler.stop()
+    status = fa.fa_get_device_status(stream)
+    if status != 0:
+        raise fa.FAError(status, "device status after the timed region")
+
+    ms_per_step = ms / max(args.steps, 1)
+    value = w.flops() * world * args.steps / (ms / 1e3) / 1e12
+    achieved = w.flops() / (ms_per_step / 1e3) / 1e12          # one launch = one step
+    peak, peak_sustained, peak_kind = load_peak()
+
+    # ---- end to end through the public call, host buffers, copies timed
+    e2e = None
+    if args.e2e_steps > 0:
+        qh = torch.from_numpy(w.q.view(np.int16)).view(torch.bfloat16).pin_memory()
+        kh = torch.from_numpy(w.k.view(np.int16)).view(torch.bfloat16).pin_memory()
+        vh = torch.from_numpy(w.v.view(np.int16)).view(torch.bfloat16).pin_memory()
+        oh = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+        lh = torch.empty(lse_shape, dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            qd = qh.to(dev, non_blocking=True)
+            kd = kh.to(dev, non_blocking=True)
+            vd = vh.to(dev, non_blocking=True)
+            od, ld = fa.attention_forward(qd, kd, vd, causal=w.causal, scale=w.scale, cu_seqlens=cu)
+            oh.copy_(od, non_blocking=True)
+            lh.copy_(ld, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        e1.synchronize()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ems], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": w.flops() * world * args.e2e_steps / (ems / 1e3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": int(qh.nbytes + kh.nbytes + vh.nbytes),
+               "d2h_bytes_per_step": int(oh.nbytes + lh.nbytes),
+               "ms_per_step": ems / args.e2e_steps, "steps": args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = time_oracle(w, args.cpu_seconds)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    clocks = sampler.summary(t_host0, t_host1)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_dict(w, {"parallelism": f"replicas x{world} (independent problems, no collective)"}),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                     "frac": achieved / peak, "traffic": profiled_traffic(args.config),
+                     "peak_source": f"MEASURED_PEAKS.json bf16_tflops (burst), of {peak_kind}",
+                     "frac_of_sustained": (achieved / peak_sustained) if peak_sustained else None},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

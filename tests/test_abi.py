@@ -1,0 +1,90 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every
+function that include/*.h declares, and rejects bad arguments before it
+touches a device (no compute call is made here)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names.update(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    from exact_tiled_attention_32_b200 import binding as fa
+    lib = ctypes.CDLL(fa.LIB_PATH)
+    declared = _declared()
+    assert {"fa_fwd", "fa_get_device_status", "fa_status_string"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+
+
+def test_status_strings():
+    from exact_tiled_attention_32_b200 import binding as fa
+    for code in range(0, -10, -1):
+        s = fa.fa_status_string(code)
+        assert s and s != "unknown status"
+    assert fa.fa_status_string(-100) == "unknown status"
+
+
+def test_argument_errors_found_on_the_host():
+    from exact_tiled_attention_32_b200 import binding as fa
+    p = 1 << 20          # an aligned address that is never dereferenced
+    ok = dict(B=1, Hq=4, Hkv=2, N=128, d=128, scale=0.1, causal=1)
+
+    def call(**kw):
+        a = dict(ok)
+        ptrs = kw.pop("ptrs", (p, p, p, p, p))
+        a.update(kw)
+        return fa.fa_fwd(*ptrs, a["B"], a["Hq"], a["Hkv"], a["N"], a["d"], a["scale"],
+                         a["causal"], kw.get("cu"), None)
+
+    assert call(d=96) == fa.FA_ERR_HEADDIM
+    assert call(d=256) == fa.FA_ERR_HEADDIM
+    assert call(Hq=4, Hkv=3) == fa.FA_ERR_GQA
+    assert call(Hkv=0) == fa.FA_ERR_GQA
+    assert call(B=-1) == fa.FA_ERR_SHAPE
+    assert call(N=-5) == fa.FA_ERR_SHAPE
+    assert call(Hq=0) == fa.FA_ERR_SHAPE
+    assert call(ptrs=(p, 0, p, p, p)) == fa.FA_ERR_NULL
+    assert call(ptrs=(p, p, p, p, 0)) == fa.FA_ERR_NULL
+    assert call(ptrs=(p + 8, p, p, p, p)) == fa.FA_ERR_ALIGN
+    assert call(ptrs=(p, p, p, p + 2, p)) == fa.FA_ERR_ALIGN
+    assert call(ptrs=(p, p, p, p, p + 1)) == fa.FA_ERR_ALIGN
+    assert call(cu=p + 2) == fa.FA_ERR_ALIGN
+    assert call(B=1025, cu=p) == fa.FA_ERR_SHAPE
+    # empty problems: nothing to do, pointers may be NULL
+    assert call(B=0, ptrs=(0, 0, 0, 0, 0)) == fa.FA_OK
+    assert call(N=0, ptrs=(0, 0, 0, 0, 0)) == fa.FA_OK
+
+
+def test_no_device_means_launch_error():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    from exact_tiled_attention_32_b200 import binding as fa
+    p = 1 << 20
+    assert fa.fa_fwd(p, p, p, p, p, 1, 1, 1, 128, 64, 0.1, 0) == fa.FA_ERR_LAUNCH
+    assert fa.fa_get_device_status() == fa.FA_ERR_LAUNCH
+
+
+def test_binding_refuses_to_run_without_the_library(tmp_path, monkeypatch):
+    """The product path has no fallback: a missing libfa.so is an ImportError."""
+    import importlib.util
+    import shutil
+    pkg = tmp_path / "pkgcopy"
+    pkg.mkdir()
+    shutil.copy(os.path.join(ROOT, "exact_tiled_attention_32_b200", "binding.py"), pkg / "binding.py")
+    spec = importlib.util.spec_from_file_location("binding_copy", pkg / "binding.py")
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError):
+        spec.loader.exec_module(mod)

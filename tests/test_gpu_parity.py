@@ -1,0 +1,223 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle on B200.
+
+Small and ragged shapes are compared on every row; the full-size workloads
+(the ones the bench times, in the same launch configuration) on sampled rows
+that the oracle computes one by one.  Tolerances: O max-abs 1e-2, O mean-abs
+1e-3, lse max-abs 1e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from exact_tiled_attention_32_b200 import synthetic as syn
+from fa_util import assert_parity, bf16_round, gather, run_gpu, sample_rows, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle(w, rows=None):
+    return oracle.attention(w.q, w.k, w.v, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal,
+                            w.cu_seqlens, rows=rows)
+
+
+def test_c1_all_rows():
+    w = syn.config("c1").draw()
+    o, lse, st = run_gpu(w)
+    assert st == 0
+    assert_parity(o, lse, *_oracle(w), "c1")
+
+
+DENSE = [
+    # B, Hq, Hkv, N, d, causal
+    (2, 4, 4, 1000, 64, False),
+    (2, 4, 4, 1000, 64, True),
+    (1, 8, 2, 777, 128, True),
+    (1, 4, 1, 513, 128, False),
+    (1, 2, 2, 1, 64, True),
+    (1, 2, 2, 1, 128, False),
+    (1, 2, 2, 127, 128, True),
+    (1, 2, 2, 129, 64, False),
+    (1, 3, 3, 200, 128, True),
+    (1, 1, 1, 255, 64, True),
+    (1, 1, 1, 257, 128, True),
+    (3, 2, 2, 384, 128, True),
+    (1, 8, 1, 640, 64, True),
+    (2, 16, 2, 300, 128, False),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,causal", DENSE)
+def test_dense_all_rows(B, Hq, Hkv, N, d, causal):
+    w = syn.Workload("dense", B, Hq, Hkv, N, d, causal, 100 + N + d + Hq).draw()
+    o, lse, st = run_gpu(w)
+    assert st == 0
+    assert_parity(o, lse, *_oracle(w), f"dense {B},{Hq},{Hkv},{N},{d},{causal}")
+
+
+PACKED = [
+    ([1, 128, 129, 5, 300, 0, 256, 257], 4, 2, 128, True),
+    ([1, 128, 129, 5, 300, 0, 256, 257], 4, 2, 128, False),
+    ([700, 3, 64], 2, 1, 64, True),
+    ([0, 0, 17], 1, 1, 64, False),
+    ([513], 8, 8, 128, True),
+]
+
+
+@pytest.mark.parametrize("lens,Hq,Hkv,d,causal", PACKED)
+def test_packed_all_rows(lens, Hq, Hkv, d, causal):
+    w = syn.packed_from_lengths("packed", lens, Hq, d, causal, 200 + len(lens), Hkv=Hkv).draw()
+    o, lse, st = run_gpu(w)
+    assert st == 0
+    assert_parity(o, lse, *_oracle(w), f"packed {lens}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_large_scores_exercise_rescale(d, causal):
+    """Scores 30x larger than 1/sqrt(d) would give: the running max grows by
+    far more than the lazy-rescale threshold from block to block.  The
+    softmax is then nearly one-hot, |O| reaches 4.5 and bf16 cannot hold O to
+    1e-2, so O is compared with the oracle's O rounded to bf16."""
+    w = syn.Workload("big", 1, 2, 2, 700, d, causal, 300 + d).draw()
+    w_scale = 30.0 / math.sqrt(d)
+    import torch
+    from exact_tiled_attention_32_b200 import binding as fa
+    o, lse = fa.attention_forward(to_device(w.q), to_device(w.k), to_device(w.v),
+                                  causal=causal, scale=w_scale)
+    torch.cuda.synchronize()
+    og, lg = gather(w, o, lse)
+    oo, lo = oracle.attention(w.q, w.k, w.v, w.B, w.Hq, w.Hkv, w.N, d, w_scale, causal)
+    assert_parity(og, lg, bf16_round(oo), lo, "large scores")
+
+
+def test_increasing_scores_force_rescale_every_block():
+    """Keys whose scores grow along the sequence: the maximum moves up by more
+    than 2^8 in every key block, so the output is rescaled on every block."""
+    N, d = 1024, 64
+    q = np.zeros((1, 1, N, d))
+    q[..., 0] = 1.0
+    k = np.zeros((1, 1, N, d))
+    k[0, 0, :, 0] = np.linspace(0, 8, N)          # score = scale * j * 8/N
+    w = syn.Workload("ramp", 1, 1, 1, N, d, False, 1)
+    w.q = syn.fp64_to_bf16_bits(q)
+    w.k = syn.fp64_to_bf16_bits(k)
+    w.v = syn.Stream(77).normal_bf16((1, 1, N, d))
+    import torch
+    from exact_tiled_attention_32_b200 import binding as fa
+    scale = 100.0
+    o, lse = fa.attention_forward(to_device(w.q), to_device(w.k), to_device(w.v), scale=scale)
+    torch.cuda.synchronize()
+    og, lg = gather(w, o, lse)
+    oo, lo = oracle.attention(w.q, w.k, w.v, 1, 1, 1, N, d, scale, False)
+    assert_parity(og, lg, bf16_round(oo), lo, "ramp")
+
+
+def test_zero_queries_give_mean_of_values():
+    N, d = 300, 128
+    w = syn.Workload("zeroq", 1, 2, 2, N, d, True, 400).draw()
+    w.q = np.zeros_like(w.q)
+    o, lse, st = run_gpu(w)
+    vf = syn.bf16_bits_to_float(w.v).astype(np.float64)
+    ref = np.cumsum(vf, axis=2) / np.arange(1, N + 1)[None, None, :, None]
+    assert np.max(np.abs(o - ref.reshape(-1, d))) <= 1e-2
+    assert np.max(np.abs(lse - np.tile(np.log(np.arange(1, N + 1)), 2))) <= 1e-3
+
+
+def test_deterministic():
+    w = syn.Workload("det", 1, 4, 2, 1000, 128, True, 500).draw()
+    import torch
+    from exact_tiled_attention_32_b200 import binding as fa
+    q, k, v = to_device(w.q), to_device(w.k), to_device(w.v)
+    o1, l1 = fa.attention_forward(q, k, v, causal=True)
+    o2, l2 = fa.attention_forward(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_outputs_stay_in_bounds():
+    """Sentinels around O and lse survive the call (stand-in for a memory checker)."""
+    import torch
+    from exact_tiled_attention_32_b200 import binding as fa
+    for (B, H, N, d, cu) in [(1, 2, 200, 128, None), (3, 2, 100, 64, [0, 1, 130, 300])]:
+        if cu is None:
+            w = syn.Workload("canary", B, H, H, N, d, True, 600).draw()
+        else:
+            w = syn.packed_from_lengths("canary", np.diff(cu), H, d, True, 601).draw()
+        pad = 1024
+        numel = w.q.size
+        obuf = torch.full((numel + 2 * pad,), -7.0, dtype=torch.bfloat16, device="cuda")
+        lbuf = torch.full((w.total_rows() + 2 * pad,), -7.0, dtype=torch.float32, device="cuda")
+        o = obuf[pad:pad + numel].view(w.q.shape)
+        lse = lbuf[pad:pad + w.total_rows()]
+        cu_t = None if w.cu_seqlens is None else torch.from_numpy(w.cu_seqlens).cuda()
+        fa.attention_forward(to_device(w.q), to_device(w.k), to_device(w.v), causal=True,
+                             cu_seqlens=cu_t, out=o, lse=lse.view(-1))
+        torch.cuda.synchronize()
+        for buf, n in ((obuf, numel), (lbuf, w.total_rows())):
+            assert torch.all(buf[:pad] == -7.0) and torch.all(buf[pad + n:] == -7.0)
+        assert fa.fa_get_device_status() == 0
+
+
+def test_bad_cu_seqlens_reported_by_device():
+    import torch
+    from exact_tiled_attention_32_b200 import binding as fa
+    H, d = 2, 64
+    q = torch.zeros((20, H, d), dtype=torch.bfloat16, device="cuda")
+    o = torch.full_like(q, 3.0)
+    lse = torch.zeros((H, 20), dtype=torch.float32, device="cuda")
+    for bad in ([0, 10, 5, 20], [1, 5, 20], [0, 5, 19]):
+        cu = torch.tensor(bad, dtype=torch.int32, device="cuda")
+        rc = fa.fa_fwd(q, q, q, o, lse, len(bad) - 1, H, H, 20, d, 0.1, 1, cu,
+                       torch.cuda.current_stream())
+        assert rc == 0
+        assert fa.fa_get_device_status(torch.cuda.current_stream()) == fa.FA_ERR_SEQLENS
+        assert torch.all(o == 3.0)
+    assert fa.fa_get_device_status() == 0
+
+
+def test_empty_problems_launch_nothing():
+    from exact_tiled_attention_32_b200 import binding as fa
+    assert fa.fa_fwd(None, None, None, None, None, 0, 4, 4, 128, 128, 0.1, 1) == 0
+    assert fa.fa_fwd(None, None, None, None, None, 2, 4, 4, 0, 64, 0.1, 0) == 0
+
+
+def test_host_errors_on_device():
+    import torch
+    from exact_tiled_attention_32_b200 import binding as fa
+    q = torch.zeros((1, 2, 64, 64), dtype=torch.bfloat16, device="cuda")
+    o = torch.empty_like(q)
+    lse = torch.zeros((1, 2, 64), dtype=torch.float32, device="cuda")
+    args = dict(B=1, Hq=2, Hkv=2, N=64, d=64, scale=0.1, causal=0)
+    assert fa.fa_fwd(q, q, q, o, lse, **args) == 0
+    assert fa.fa_fwd(q.data_ptr() + 2, q, q, o, lse, **args) == fa.FA_ERR_ALIGN
+    assert fa.fa_fwd(q, q, q, o, lse.data_ptr() + 2, **args) == fa.FA_ERR_ALIGN
+    assert fa.fa_fwd(q, None, q, o, lse, **args) == fa.FA_ERR_NULL
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status() == 0
+
+
+# ---------------------------------------------------------------- full sizes
+FULL = {
+    # config: (early rows, tile stride, random rows per (sequence, head))
+    "c2nc": None,          # every row
+    "c2c": None,
+    "c3": (8, 2, 16),
+    "c4": (8, 8, 8),
+    "c5": (8, 4, 8),
+}
+
+
+@pytest.mark.parametrize("name", list(FULL))
+def test_full_size(name):
+    w = syn.config(name).draw()
+    o, lse, st = run_gpu(w)
+    assert st == 0
+    spec = FULL[name]
+    rows = None if spec is None else sample_rows(w, *spec, seed=1)
+    oo, lo = _oracle(w, rows)
+    if rows is not None:
+        o, lse = o[rows], lse[rows]
+    mx, mean, lmx = assert_parity(o, lse, oo, lo, name)
+    print(f"{name}: rows={len(lo)} O max-abs {mx:.3e} mean-abs {mean:.3e} lse max-abs {lmx:.3e}")
