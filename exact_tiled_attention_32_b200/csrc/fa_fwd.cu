@@ -8,21 +8,22 @@
 // unnormalised output O, and write only O / l (and the logsumexp) to HBM.
 //
 // B200 mapping (one persistent CTA per SM, 384 threads, warp-specialised):
-//   warp 9      TMA producer: Q_i (two 128-row tiles per work item) and a
-//               ring of K_j / V_j tiles in 128-byte-swizzled shared memory.
-//   warp 8      MMA issuer (one thread): S_t = Q_t K_j^T and O_t += P_t V_j as
-//               tcgen05.mma kind::f16 (bf16 in, fp32 accumulate in TMEM).  P_t
-//               is read straight from TMEM, where it overwrites S_t.
-//   warps 0-3   softmax for query tile 0, warps 4-7 for query tile 1: one
-//               thread per query row; tcgen05.ld of S, masking, running max in
-//               the log2 domain, exp2 via one FFMA + ex2, lazy rescale of O in
-//               TMEM (only when the max grows by more than 2^8), bf16 P written
-//               back to TMEM, and finally the epilogue O / l -> bf16 -> HBM plus
-//               the logsumexp.
-//   warps 10-11 idle (they complete the third warpgroup, which gives its
-//               registers to the softmax warpgroups through setmaxnreg).
-// The two query tiles ping-pong: while the softmax warps work on tile 0 the
-// tensor core runs tile 1's MMAs and vice versa.
+//   warps 0-3   query tile 0, warps 4-7 query tile 1 (one warpgroup each):
+//               one thread per query row; tcgen05.ld of S, masking, running
+//               max in the log2 domain, exp2 via one FFMA + ex2, lazy rescale of
+//               O in TMEM (only when the max grows by more than 2^8), bf16 P
+//               written back to TMEM over S, and the epilogue O / l -> bf16 ->
+//               HBM plus the logsumexp.
+//   warp 10     MMA issuer (one thread): S_t = Q_t K_j^T and O_t += P_t V_j as
+//               tcgen05.mma kind::f16 (bf16 in, fp32 accumulate in TMEM); the A
+//               operand of P_t V_j is read straight from TMEM.  A single issuer
+//               keeps the two tiles' MMA batches alternating, which keeps the two
+//               softmax warpgroups out of phase (ping-pong).
+//   warp 11     TMA producer: Q (two 128-row tiles per work item) and a ring of
+//               K_j / V_j tiles in 128-byte-swizzled shared memory.
+//   warps 8-9   idle apart from TMEM allocation (warp 9); they complete the
+//               third warpgroup, which gives registers to the softmax
+//               warpgroups through setmaxnreg.
 //
 // TMEM columns (512 allocated): S0/P0 [0,128), S1/P1 [128,256),
 // O0 [256, 256+D), O1 [384, 384+D).
@@ -30,6 +31,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -44,20 +46,22 @@ constexpr int kBlockM = 128;           // query rows per tile (B_r)
 constexpr int kBlockN = 128;           // keys per tile (B_c)
 constexpr int kRowsPerItem = 2 * kBlockM;
 constexpr int kNumSoftmaxWarps = 8;
-constexpr int kMmaWarp = 8;
-constexpr int kLoadWarp = 9;
+constexpr int kAllocWarp = 9;
+constexpr int kMmaWarp = 10;
+constexpr int kLoadWarp = 11;
 constexpr int kThreads = 384;
 constexpr uint32_t kSoftmaxRegs = 216;   // setmaxnreg split: 2 x 128 x 216 + 128 x 72 = 384 x 168
 constexpr uint32_t kOtherRegs = 72;
 constexpr int kMaxSeqs = 1024;         // packed batches: sequences
 constexpr int kMaxPairs = 1024;        // packed batches: 256-row pairs per sequence
 constexpr uint32_t kTmemCols = 512;
+constexpr int kMaxStages = 10;
+constexpr int kBoxBytes = kBlockM * 64 * 2;   // one 128-row x 64-column bf16 TMA box
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only past 2^8
 
 // where a wait gave up (reported in status[1])
 enum WaitSite : int {
-    kSiteQEmpty = 1, kSiteKvEmpty, kSiteQFull, kSiteKvFull, kSitePFull, kSiteSFull, kSiteOFinal,
-    kSiteDrain
+    kSiteQEmpty = 1, kSiteKvEmpty, kSiteQFull, kSiteKvFull, kSitePFull, kSiteSFull, kSiteOFinal
 };
 
 struct alignas(64) Params {
@@ -68,37 +72,62 @@ struct alignas(64) Params {
     int* status;
     int B, Hq, Hkv, N;
     int group;                 // Hq / Hkv
+    int group_units;           // dense: (batch, head) units scheduled together
     int causal, packed;
     float scale_log2;          // scale * log2(e)
     unsigned long long timeout_ns;
+    unsigned long long* trace;     // FA_TRACE builds: per-role clock64 stamps of CTA 0
 };
 
+// Optional pipeline timeline (compile with -DFA_TRACE): CTA 0 records clock64
+// stamps per role and iteration into Params::trace, laid out as
+// [role][iteration][event], kTraceIters iterations and 8 events per role.
+[[maybe_unused]] constexpr int kTraceIters = 1024;
+#ifdef FA_TRACE
+#define FA_TRACE_EV(role, it, ev)                                                              \
+    do {                                                                                       \
+        if (blockIdx.x == 0 && p.trace && (it) < kTraceIters)                                  \
+            p.trace[((role) * kTraceIters + (it)) * 8 + (ev)] = clock64();                     \
+    } while (0)
+#else
+#define FA_TRACE_EV(role, it, ev) \
+    do {                          \
+    } while (0)
+#endif
+
 struct Misc {
-    uint64_t bar_q_full, bar_q_empty, bar_drain;
-    uint64_t bar_kv_full[8], bar_kv_empty[8];
-    uint64_t bar_s_full[2], bar_p_full[2], bar_o_final[2];
+    uint64_t bar_q_full, bar_q_empty;
+    uint64_t bar_kv_full[kMaxStages], bar_kv_empty[kMaxStages];
+    uint64_t bar_s_full[2], bar_p_full[2], bar_o_final[2], bar_drain;
     uint32_t tmem_base;
     int abort_flag;
     int bad;
     int total_items;
     int pmax;
+};
+
+// Packed batches only: the sequence offsets and the pair-level schedule.
+struct SeqTables {
     int seq_off[kMaxSeqs + 1];
     int order[kMaxSeqs];       // sequences by pair count, descending
     int pcnt[kMaxPairs];       // number of sequences with more than p pairs
     int pstart[kMaxPairs];     // first item index at pair level p
 };
 
-template <int D>
+template <int D, bool PK>
 struct Cfg {
     static_assert(D == 64 || D == 128, "head dim");
     static constexpr int kTileBytes = kBlockM * D * 2;     // one 128 x D bf16 tile
-    static constexpr int kBoxBytes = kBlockM * 64 * 2;     // one 128 x 64 TMA box
     static constexpr int kBoxes = D / 64;
-    static constexpr int kStages = (D == 128) ? 4 : 8;
+    // K/V ring depth: what fits next to the two Q tiles (and the packed tables)
+    static constexpr int kStages = (D == 128) ? (PK ? 4 : 5) : 10;
+    static_assert(kStages <= kMaxStages, "ring");
     static constexpr int kQOff = 0;
     static constexpr int kKVOff = 2 * kTileBytes;
     static constexpr int kMiscOff = kKVOff + kStages * kTileBytes;
-    static constexpr int kSmemBytes = kMiscOff + (int)sizeof(Misc) + 1024;
+    static constexpr int kTabOff = kMiscOff + (((int)sizeof(Misc) + 127) / 128) * 128;
+    static constexpr int kSmemBytes = kTabOff + (PK ? (int)sizeof(SeqTables) : 0) + 1024;
+    static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
 // One work item: two consecutive 128-row query tiles of one (sequence, head).
@@ -117,35 +146,44 @@ __device__ __forceinline__ int tile_blocks(int q0, int len, int causal) {
     return causal ? min(nkv, q0 / kBlockN + 1) : nkv;
 }
 
-// Items run in decreasing pair index (heaviest causal tiles first), then
-// sequence, then head, so that query heads sharing a key/value head run side
-// by side.
-__device__ __forceinline__ Item decode_item(int idx, const Params& p, const Misc& ms) {
+// Dense batches: the (batch, head) units are cut into groups whose K/V fit in
+// L2 together (query heads sharing a key/value head are adjacent); a group's
+// items run in decreasing pair index (heaviest causal tiles first).  Packed
+// batches: decreasing pair index over all sequences, then sequence, then head.
+template <bool PK>
+__device__ __forceinline__ Item decode_item(int idx, const Params& p, const Misc& ms, const SeqTables& tab) {
     Item it;
     int pair;
-    if (!p.packed) {
+    if constexpr (!PK) {
+        // units (b, h) in groups of group_units whose K/V fit in L2 together;
+        // inside a group, heaviest pair first
         const int npairs = (p.N + kRowsPerItem - 1) / kRowsPerItem;
         const int per = p.B * p.Hq;
-        const int lvl = idx / per;
-        const int rem = idx - lvl * per;
+        const int G = p.group_units;
+        const int g = idx / (npairs * G);
+        const int gbase = g * G;
+        const int gsz = min(G, per - gbase);
+        const int r = idx - g * npairs * G;
+        const int lvl = r / gsz;
+        const int unit = gbase + (r - lvl * gsz);
         pair = npairs - 1 - lvl;
-        it.seq = rem / p.Hq;
-        it.h = rem - it.seq * p.Hq;
+        it.seq = unit / p.Hq;
+        it.h = unit - it.seq * p.Hq;
         it.len = p.N;
         it.tok0 = 0;
     } else {
         int lo = 0, hi = ms.pmax - 1;      // smallest level whose start <= idx
         while (lo < hi) {
             const int mid = (lo + hi) >> 1;
-            if (ms.pstart[mid] <= idx) hi = mid; else lo = mid + 1;
+            if (tab.pstart[mid] <= idx) hi = mid; else lo = mid + 1;
         }
         pair = lo;
-        const int rem = idx - ms.pstart[lo];
+        const int rem = idx - tab.pstart[lo];
         const int k = rem / p.Hq;
         it.h = rem - k * p.Hq;
-        it.seq = ms.order[k];
-        it.tok0 = ms.seq_off[it.seq];
-        it.len = ms.seq_off[it.seq + 1] - it.tok0;
+        it.seq = tab.order[k];
+        it.tok0 = tab.seq_off[it.seq];
+        it.len = tab.seq_off[it.seq + 1] - it.tok0;
     }
     it.q0 = pair * kRowsPerItem;
     it.n[0] = tile_blocks(it.q0, it.len, p.causal);
@@ -161,6 +199,14 @@ __device__ __forceinline__ int item_of_round(int r) {
     return r * G + ((r & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
 }
 
+// A waiting thread sleeps in try_wait (woken when the phase completes) instead
+// of spinning, so it leaves issue slots to the softmax warps of its SM
+// sub-partition; the sleep is bounded so that the timeout is still checked.
+#ifndef FA_SUSPEND_NS
+#define FA_SUSPEND_NS 20000u
+#endif
+constexpr uint32_t kSuspendNs = FA_SUSPEND_NS;
+
 // Bounded wait: gives up after timeout_ns (recording the site in the status
 // word and raising the CTA's abort flag) or as soon as another role aborted.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Params& p, Misc& ms,
@@ -168,7 +214,7 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Pa
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
         if (*reinterpret_cast<volatile int*>(&ms.abort_flag)) return false;
         if (globaltimer_ns() - t0 > p.timeout_ns) {
             *reinterpret_cast<volatile int*>(&ms.abort_flag) = 1;
@@ -189,9 +235,10 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, const P
 }
 
 // ---------------------------------------------------------------- producer
-template <int D>
-__device__ void load_role(const Params& p, Misc& ms, uint32_t smem_q, uint32_t smem_kv, int total) {
-    using C = Cfg<D>;
+template <int D, bool PK>
+__device__ void load_role(const Params& p, Misc& ms, const SeqTables& tab, uint32_t smem_q, uint32_t smem_kv,
+                          int total) {
+    using C = Cfg<D, PK>;
     const uint64_t pol_kv = policy_evict_last();
     const uint64_t pol_q = policy_evict_first();
     uint32_t kv_it = 0, item_n = 0;
@@ -199,7 +246,7 @@ __device__ void load_role(const Params& p, Misc& ms, uint32_t smem_q, uint32_t s
     for (int r = 0; ok; ++r) {
         const int idx = item_of_round(r);
         if (idx >= total) break;
-        const Item it = decode_item(idx, p, ms);
+        const Item it = decode_item<PK>(idx, p, ms, tab);
         // both query tiles of the item
         if (!(ok = wait_bar(smem_u32(&ms.bar_q_empty), (item_n & 1) ^ 1, p, ms, kSiteQEmpty))) break;
         const uint32_t qbar = smem_u32(&ms.bar_q_full);
@@ -207,8 +254,8 @@ __device__ void load_role(const Params& p, Misc& ms, uint32_t smem_q, uint32_t s
         for (int t = 0; t < 2; ++t) {
             const int row = it.q0 + t * kBlockM;
             for (int b = 0; b < C::kBoxes; ++b) {
-                const uint32_t dst = smem_q + t * C::kTileBytes + b * C::kBoxBytes;
-                if (!p.packed)
+                const uint32_t dst = smem_q + t * C::kTileBytes + b * kBoxBytes;
+                if constexpr (!PK)
                     tma_load_4d(dst, &p.tm_q, qbar, b * 64, row, it.h, it.seq, pol_q);
                 else
                     tma_load_4d(dst, &p.tm_q, qbar, b * 64, it.h, it.tok0 + row, 0, pol_q);
@@ -227,8 +274,8 @@ __device__ void load_role(const Params& p, Misc& ms, uint32_t smem_q, uint32_t s
                 mbar_arrive_expect_tx(bar, C::kTileBytes);
                 const CUtensorMap* map = kind == 0 ? &p.tm_k : &p.tm_v;
                 for (int b = 0; b < C::kBoxes; ++b) {
-                    const uint32_t dst = smem_kv + st * C::kTileBytes + b * C::kBoxBytes;
-                    if (!p.packed)
+                    const uint32_t dst = smem_kv + st * C::kTileBytes + b * kBoxBytes;
+                    if constexpr (!PK)
                         tma_load_4d(dst, map, bar, b * 64, j * kBlockN, kvh, it.seq, pol_kv);
                     else
                         tma_load_4d(dst, map, bar, b * 64, kvh, it.tok0 + j * kBlockN, 0, pol_kv);
@@ -247,53 +294,57 @@ __device__ void load_role(const Params& p, Misc& ms, uint32_t smem_q, uint32_t s
 }
 
 // ------------------------------------------------------------- MMA issuer
+// S_t = Q_t K^T over K = d (steps of 16), both operands K-major, 128-byte
+// swizzle; O_t (+)= P_t V with P read from TMEM.  Each is one asm block.
 template <int D>
-__device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_addr, uint32_t k_addr) {
+__device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint64_t dq, uint64_t dk) {
     constexpr uint32_t idesc = idesc_bf16_f32(kBlockM, kBlockN, false);
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk / 4) * Cfg<D>::kBoxBytes + (kk % 4) * 32;
-        umma_ss(tmem_s, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
-                idesc, kk > 0 ? 1u : 0u);
-    }
+    if constexpr (D == 128)
+        umma_ss_k128_x8(tmem_s, dq, dk, idesc);
+    else
+        umma_ss_k64_x4(tmem_s, dq, dk, idesc);
 }
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_addr, bool accumulate) {
+__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint64_t dv, bool accumulate) {
     constexpr uint32_t idesc = idesc_bf16_f32(kBlockM, D, true);
-#pragma unroll
-    for (int kk = 0; kk < kBlockN / 16; ++kk) {
-        umma_ts(tmem_o, tmem_p + kk * 8, smem_desc_sw128(v_addr + kk * 16 * 128, Cfg<D>::kBoxBytes, 1024),
-                idesc, (accumulate || kk > 0) ? 1u : 0u);
-    }
+    umma_ts_kv128_x8(tmem_o, tmem_p, dv, idesc, accumulate ? 1u : 0u);
 }
 
-template <int D>
-__device__ void mma_role(const Params& p, Misc& ms, uint32_t tmem, uint32_t smem_q, uint32_t smem_kv,
-                         int total) {
-    using C = Cfg<D>;
+// The MMA issuer.  Per work item it walks j = 0 .. nmax (nmax = the larger
+// block count of the two tiles): O_t += P_t V_{j-1} for each tile that had
+// block j-1, then S_t = Q_t K_j^T for each tile that has block j, tile 0
+// before tile 1 -- the order that keeps the two softmax warpgroups out of phase.
+template <int D, bool PK>
+__device__ void mma_role(const Params& p, Misc& ms, const SeqTables& tab, uint32_t tmem, uint32_t smem_q,
+                         uint32_t smem_kv, int total) {
+    using C = Cfg<D, PK>;
+    // descriptors of Q tile 0 and of ring stage 0; other tiles/stages are offsets
+    const uint64_t dq0 = smem_desc_sw128(smem_q, 16, 1024);
+    const uint64_t dk0 = smem_desc_sw128(smem_kv, 16, 1024);              // K-major (K tiles)
+    const uint64_t dv0 = smem_desc_sw128(smem_kv, kBoxBytes, 1024);       // MN-major (V tiles)
+    constexpr uint64_t kTileStep = C::kTileBytes >> 4;
     uint32_t kv_it = 0, item_n = 0;
     uint32_t pc[2] = {0, 0};
     bool ok = true;
     for (int r = 0; ok; ++r) {
         const int idx = item_of_round(r);
         if (idx >= total) break;
-        const Item it = decode_item(idx, p, ms);
+        const Item it = decode_item<PK>(idx, p, ms, tab);
         if (!(ok = wait_bar(smem_u32(&ms.bar_q_full), item_n & 1, p, ms, kSiteQFull))) break;
         tc_fence_after();
         ++item_n;
         const int nmax = max(it.n[0], it.n[1]);
         const uint32_t base = kv_it;
-        for (int j = 0; j < nmax && ok; ++j) {
-            const uint32_t kit = base + 2 * j;
-            const uint32_t kst = kit % C::kStages;
-            if (!(ok = wait_bar(smem_u32(&ms.bar_kv_full[kst]), (kit / C::kStages) & 1, p, ms, kSiteKvFull)))
+        for (int j = 0; j <= nmax && ok; ++j) {
+            [[maybe_unused]] const uint32_t mit = base / 2 + j;   // iteration counter for the trace
+            FA_TRACE_EV(2, mit, 0);
+            const uint32_t vit = base + 2 * j - 1, vst = vit % C::kStages;
+            const uint32_t kit = base + 2 * j, kst = kit % C::kStages;
+            if (j > 0 && !(ok = wait_bar(smem_u32(&ms.bar_kv_full[vst]), (vit / C::kStages) & 1, p, ms,
+                                         kSiteKvFull)))
                 break;
-            const uint32_t vit = kit - 1;
-            const uint32_t vst = vit % C::kStages;
-            if (j > 0 &&
-                !(ok = wait_bar(smem_u32(&ms.bar_kv_full[vst]), (vit / C::kStages) & 1, p, ms, kSiteKvFull)))
-                break;
-            tc_fence_after();
+            bool k_ready = false;
+            FA_TRACE_EV(2, mit, 1);
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
                 if (!ok) break;
@@ -301,36 +352,28 @@ __device__ void mma_role(const Params& p, Misc& ms, uint32_t tmem, uint32_t smem
                     if (!(ok = wait_bar(smem_u32(&ms.bar_p_full[t]), pc[t] & 1, p, ms, kSitePFull))) break;
                     ++pc[t];
                     tc_fence_after();
-                    issue_pv<D>(tmem + 256 + t * 128, tmem + t * 128, smem_kv + vst * C::kTileBytes, j - 1 > 0);
+                    FA_TRACE_EV(2, mit, 2 + 2 * t);
+                    issue_pv<D>(tmem + 256 + t * 128, tmem + t * 128, dv0 + vst * kTileStep, j - 1 > 0);
                     if (j - 1 == it.n[t] - 1) umma_commit(smem_u32(&ms.bar_o_final[t]));
                 }
                 if (j < it.n[t]) {                       // S_t = Q_t K_j^T
-                    issue_qk<D>(tmem + t * 128, smem_q + t * C::kTileBytes, smem_kv + kst * C::kTileBytes);
+                    if (!k_ready) {
+                        if (!(ok = wait_bar(smem_u32(&ms.bar_kv_full[kst]), (kit / C::kStages) & 1, p, ms,
+                                            kSiteKvFull)))
+                            break;
+                        tc_fence_after();
+                        k_ready = true;
+                    }
+                    issue_qk<D>(tmem + t * 128, dq0 + t * kTileStep, dk0 + kst * kTileStep);
                     umma_commit(smem_u32(&ms.bar_s_full[t]));
+                    FA_TRACE_EV(2, mit, 3 + 2 * t);
                 }
             }
             if (!ok) break;
-            umma_commit(smem_u32(&ms.bar_kv_empty[kst]));
+            if (k_ready) umma_commit(smem_u32(&ms.bar_kv_empty[kst]));
             if (j > 0) umma_commit(smem_u32(&ms.bar_kv_empty[vst]));
             if (j == nmax - 1) umma_commit(smem_u32(&ms.bar_q_empty));
         }
-        if (!ok) break;
-        // last value block
-        const uint32_t vit = base + 2 * nmax - 1;
-        const uint32_t vst = vit % C::kStages;
-        if (!(ok = wait_bar(smem_u32(&ms.bar_kv_full[vst]), (vit / C::kStages) & 1, p, ms, kSiteKvFull))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            if (!ok || it.n[t] != nmax) continue;
-            if (!(ok = wait_bar(smem_u32(&ms.bar_p_full[t]), pc[t] & 1, p, ms, kSitePFull))) break;
-            ++pc[t];
-            tc_fence_after();
-            issue_pv<D>(tmem + 256 + t * 128, tmem + t * 128, smem_kv + vst * C::kTileBytes, nmax - 1 > 0);
-            umma_commit(smem_u32(&ms.bar_o_final[t]));
-        }
-        if (!ok) break;
-        umma_commit(smem_u32(&ms.bar_kv_empty[vst]));
         kv_it = base + 2 * nmax;
     }
     // every MMA issued so far must be finished before TMEM and smem go away
@@ -339,8 +382,41 @@ __device__ void mma_role(const Params& p, Misc& ms, uint32_t tmem, uint32_t smem
 }
 
 // ---------------------------------------------------------------- softmax
-template <int D>
-__device__ void softmax_role(const Params& p, Misc& ms, uint32_t tmem, int warp, int lane, int total) {
+// exp2 of a pair of floats on the FMA pipe instead of the MUFU unit:
+// 2^x = 2^j * 2^f with j = round(x), f = x - j in [-0.5, 0.5]; 2^f is a
+// degree-3 minimax polynomial (max relative error 7.5e-5; coefficients fitted
+// by fit_exp2_poly.py next to this file) and 2^j is added to the exponent
+// field.  x is clamped at -126 so that the exponent never wraps; masked
+// entries (-inf) then give 2^-126 instead of 0, which is below the fp32
+// resolution of any row sum that holds the row maximum (>= 1).
+#ifndef FA_POLY_PAIRS_PER8
+#define FA_POLY_PAIRS_PER8 0
+#endif
+constexpr int kPolyPairsPer8 = FA_POLY_PAIRS_PER8;   // column pairs (of every 8) on the polynomial
+__device__ __forceinline__ uint64_t f2_const(uint32_t bits) {
+    return (static_cast<uint64_t>(bits) << 32) | bits;
+}
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
+    float x0, x1;
+    f2_unpack(x, x0, x1);
+    x = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+    const uint64_t t = f2_add(x, f2_const(0x4B400000u));        // 1.5 * 2^23 + round(x)
+    const uint64_t r = f2_add(t, f2_const(0xCB400000u));        // round(x)
+    const uint64_t f = f2_fma(r, f2_const(0xBF800000u), x);     // x - round(x)
+    uint64_t q = f2_fma(f2_const(0x3D61FBB0u), f, f2_const(0x3E786F0Du));   // c3 f + c2
+    q = f2_fma(q, f, f2_const(0x3F31798Du));                                // .. f + c1
+    q = f2_fma(q, f, f2_const(0x3F7FFB49u));                                // .. f + c0
+    float q0, q1, t0, t1;
+    f2_unpack(q, q0, q1);
+    f2_unpack(t, t0, t1);
+    q0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+    q1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+    return f2_pack(q0, q1);
+}
+
+template <int D, bool PK>
+__device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, uint32_t tmem, int warp, int lane,
+                             int total) {
     const int t = warp / 4;                          // query tile of this warpgroup
     const int wq = warp % 4;                         // TMEM lane quarter
     const int r = wq * 32 + lane;                    // row inside the tile
@@ -348,12 +424,13 @@ __device__ void softmax_role(const Params& p, Misc& ms, uint32_t tmem, int warp,
     const uint32_t taddr_s = tmem + lane_off + t * 128;
     const uint32_t taddr_o = tmem + lane_off + 256 + t * 128;
     const float sl2 = p.scale_log2;
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
     uint32_t sc = 0, oc = 0;
     bool ok = true;
     for (int rr = 0; ok; ++rr) {
         const int idx = item_of_round(rr);
         if (idx >= total) break;
-        const Item it = decode_item(idx, p, ms);
+        const Item it = decode_item<PK>(idx, p, ms, tab);
         const int n = t ? it.n[1] : it.n[0];
         if (n == 0) continue;
         const int row = it.q0 + t * kBlockM + r;
@@ -361,37 +438,53 @@ __device__ void softmax_role(const Params& p, Misc& ms, uint32_t tmem, int warp,
         float m_used = -INFINITY;    // max the exponentials are taken against (log2 units)
         float l = 0.f;               // running sum of exp2(x - m_used)
         for (int j = 0; j < n; ++j) {
+            if (lane == 0 && wq == 0) FA_TRACE_EV(t, sc, 0);
             ok = wait_bar(smem_u32(&ms.bar_s_full[t]), sc & 1, p, ms, kSiteSFull);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             ++sc;
             tc_fence_after();
-            uint32_t s[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32_sync(taddr_s + c * 32, s[c]);
+            if (lane == 0 && wq == 0) FA_TRACE_EV(t, sc - 1, 1);
+            uint32_t s[128];
+            tmem_ld128_sync(taddr_s, s);
+            if (lane == 0 && wq == 0) FA_TRACE_EV(t, sc - 1, 2);
             if (j * kBlockN + kBlockN > limit) {      // diagonal or tail block
                 const int lim = limit - j * kBlockN;
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (c * 32 + i >= lim) s[c][i] = __float_as_uint(-INFINITY);
+                for (int c = 0; c < 128; ++c)
+                    if (c >= lim) s[c] = __float_as_uint(-INFINITY);
             }
-            float mx = -INFINITY;
+            // row max: four independent chains of 3-input max
+            float mx;
+            {
+                float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-#pragma unroll
-                for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(s[c][i]));
+                for (int c = 0; c < 128; c += 8) {
+                    m0 = fmax3(m0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+                    m1 = fmax3(m1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+                    m2 = fmax3(m2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
+                    m3 = fmax3(m3, __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
+                }
+                mx = fmax3(fmaxf(m0, m1), m2, m3);
+            }
             const float m_new = fmaxf(m_used, mx * sl2);
+            if (lane == 0 && wq == 0) FA_TRACE_EV(t, sc - 1, 3);
             const bool need = m_new > m_used + kRescaleThreshold;
             if (j > 0 && __any_sync(0xffffffffu, need)) {
-                // Theorem 2: rescale the partial output when the max grows
+                // Theorem 2: rescale the partial output when the max grows.
+                // S_t(j) was issued after O_t += P_t V_{j-1}, so O_t is final here.
                 const float f = need ? ex2_approx(m_used - m_new) : 1.f;
+                const uint64_t f2 = f2_pack(f, f);
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t o[32];
                     tmem_ld32_sync(taddr_o + c * 32, o);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+                    for (int i = 0; i < 16; ++i) {
+                        float a, b;
+                        f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), f2), a, b);
+                        o[2 * i] = __float_as_uint(a);
+                        o[2 * i + 1] = __float_as_uint(b);
+                    }
                     tmem_st32(taddr_o + c * 32, o);
                 }
                 tmem_wait_st();
@@ -401,24 +494,45 @@ __device__ void softmax_role(const Params& p, Misc& ms, uint32_t tmem, int warp,
                 m_used = m_new;
             }
             const float msub = (m_used == -INFINITY) ? 0.f : m_used;
-            float rs = 0.f;
+            const uint64_t nm2 = f2_pack(-msub, -msub);
+            uint64_t acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0;   // packed row sums (+0.0f pairs)
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const uint32_t* sv = s[2 * half + i / 16];
-                    const float a = ex2_approx(fmaf(__uint_as_float(sv[(2 * i) % 32]), sl2, -msub));
-                    const float b = ex2_approx(fmaf(__uint_as_float(sv[(2 * i + 1) % 32]), sl2, -msub));
-                    rs += a + b;
-                    pk[i] = pack_bf16x2(a, b);
+                    const int gi = 32 * half + i;       // pair of columns 2gi, 2gi+1
+                    const uint64_t x = f2_fma(f2_pack(__uint_as_float(s[2 * gi]), __uint_as_float(s[2 * gi + 1])),
+                                              sl2x2, nm2);
+                    uint64_t e;
+                    if ((gi % 8) < kPolyPairsPer8) {
+                        e = exp2_poly2(x);
+                    } else {
+                        float x0, x1;
+                        f2_unpack(x, x0, x1);
+                        e = f2_pack(ex2_approx(x0), ex2_approx(x1));
+                    }
+                    switch (i & 3) {
+                        case 0: acc0 = f2_add(acc0, e); break;
+                        case 1: acc1 = f2_add(acc1, e); break;
+                        case 2: acc2 = f2_add(acc2, e); break;
+                        default: acc3 = f2_add(acc3, e); break;
+                    }
+                    float e0, e1;
+                    f2_unpack(e, e0, e1);
+                    pk[i] = pack_bf16x2(e0, e1);
                 }
                 tmem_st32(taddr_s + half * 32, pk);
             }
-            l += rs;
+            {
+                float a, b;
+                f2_unpack(f2_add(f2_add(acc0, acc1), f2_add(acc2, acc3)), a, b);
+                l += a + b;
+            }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
+            if (lane == 0) FA_TRACE_EV(t, sc - 1, wq == 0 ? 4 : 4 + wq);
             if (lane == 0) mbar_arrive(smem_u32(&ms.bar_p_full[t]));
         }
         if (!ok) break;
@@ -431,7 +545,7 @@ __device__ void softmax_role(const Params& p, Misc& ms, uint32_t tmem, int warp,
         const float inv = l > 0.f ? 1.f / l : 0.f;
         uint16_t* orow;
         float* lrow;
-        if (!p.packed) {
+        if constexpr (!PK) {
             const size_t rid = (static_cast<size_t>(it.seq) * p.Hq + it.h) * p.N + row;
             orow = static_cast<uint16_t*>(p.o) + rid * D;
             lrow = p.lse + rid;
@@ -465,12 +579,13 @@ __device__ void softmax_role(const Params& p, Misc& ms, uint32_t tmem, int warp,
 }
 
 // ------------------------------------------------------------------ kernel
-template <int D>
+template <int D, bool PK>
 __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_constant__ Params p) {
-    using C = Cfg<D>;
+    using C = Cfg<D, PK>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Misc& ms = *reinterpret_cast<Misc*>(smem + C::kMiscOff);
+    SeqTables& tab = *reinterpret_cast<SeqTables*>(smem + C::kTabOff);   // packed batches only
     const int tid = threadIdx.x;
     const int warp = tid / 32, lane = tid % 32;
     const uint32_t smem_q = smem_u32(smem + C::kQOff);
@@ -486,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(smem_u32(&ms.bar_s_full[t]), 1);
-            mbar_init(smem_u32(&ms.bar_p_full[t]), 4);
+            mbar_init(smem_u32(&ms.bar_p_full[t]), 4);    // one arrival per warp
             mbar_init(smem_u32(&ms.bar_o_final[t]), 1);
         }
         ms.abort_flag = 0;
@@ -500,14 +615,14 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     }
 
     int total;
-    if (p.packed) {
+    if constexpr (PK) {
         // stage the offsets, check them, and build the pair-level tables
-        for (int i = tid; i <= p.B; i += kThreads) ms.seq_off[i] = p.cu_seqlens[i];
+        for (int i = tid; i <= p.B; i += kThreads) tab.seq_off[i] = p.cu_seqlens[i];
         __syncthreads();
         if (tid == 0) {
-            int bad = ms.seq_off[0] != 0 || ms.seq_off[p.B] != p.N;
+            int bad = tab.seq_off[0] != 0 || tab.seq_off[p.B] != p.N;
             for (int s = 0; s < p.B && !bad; ++s) {
-                const int L = ms.seq_off[s + 1] - ms.seq_off[s];
+                const int L = tab.seq_off[s + 1] - tab.seq_off[s];
                 if (L < 0 || L > kMaxPairs * kRowsPerItem) bad = 1;
             }
             ms.bad = bad;
@@ -518,36 +633,36 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             return;
         }
         for (int s = tid; s < p.B; s += kThreads) {
-            const int ps = (ms.seq_off[s + 1] - ms.seq_off[s] + kRowsPerItem - 1) / kRowsPerItem;
+            const int ps = (tab.seq_off[s + 1] - tab.seq_off[s] + kRowsPerItem - 1) / kRowsPerItem;
             int rank = 0;
             for (int u = 0; u < p.B; ++u) {
-                const int pu = (ms.seq_off[u + 1] - ms.seq_off[u] + kRowsPerItem - 1) / kRowsPerItem;
+                const int pu = (tab.seq_off[u + 1] - tab.seq_off[u] + kRowsPerItem - 1) / kRowsPerItem;
                 rank += (pu > ps) || (pu == ps && u < s);
             }
-            ms.order[rank] = s;
+            tab.order[rank] = s;
         }
         __syncthreads();
         if (tid == 0) {
             auto pairs_of = [&](int s) {
-                return (ms.seq_off[s + 1] - ms.seq_off[s] + kRowsPerItem - 1) / kRowsPerItem;
+                return (tab.seq_off[s + 1] - tab.seq_off[s] + kRowsPerItem - 1) / kRowsPerItem;
             };
-            const int pmax = p.B > 0 ? pairs_of(ms.order[0]) : 0;
+            const int pmax = p.B > 0 ? pairs_of(tab.order[0]) : 0;
             int k = p.B;
             for (int lvl = 0; lvl < pmax; ++lvl) {
-                while (k > 0 && pairs_of(ms.order[k - 1]) <= lvl) --k;
-                ms.pcnt[lvl] = k;
+                while (k > 0 && pairs_of(tab.order[k - 1]) <= lvl) --k;
+                tab.pcnt[lvl] = k;
             }
             int acc = 0;
             for (int lvl = pmax - 1; lvl >= 0; --lvl) {
-                ms.pstart[lvl] = acc;
-                acc += ms.pcnt[lvl] * p.Hq;
+                tab.pstart[lvl] = acc;
+                acc += tab.pcnt[lvl] * p.Hq;
             }
             ms.pmax = pmax;
             ms.total_items = acc;
         }
     }
 
-    if (warp == kMmaWarp) {
+    if (warp == kAllocWarp) {
         tmem_alloc(smem_u32(&ms.tmem_base), kTmemCols);
         tmem_relinquish();
     }
@@ -555,7 +670,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ms.tmem_base;
-    if (p.packed) {
+    if constexpr (PK) {
         total = ms.total_items;
     } else {
         total = ((p.N + kRowsPerItem - 1) / kRowsPerItem) * p.B * p.Hq;
@@ -563,22 +678,21 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
 
     if (warp < kNumSoftmaxWarps) {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
-        softmax_role<D>(p, ms, tmem, warp, lane, total);
+        softmax_role<D, PK>(p, ms, tab, tmem, warp, lane, total);
     } else {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
-    }
-    if (warp < kNumSoftmaxWarps) {
-    } else if (warp == kMmaWarp) {
-        if (lane == 0) mma_role<D>(p, ms, tmem, smem_q, smem_kv, total);
-        __syncwarp();
-    } else if (warp == kLoadWarp) {
-        if (lane == 0) load_role<D>(p, ms, smem_q, smem_kv, total);
-        __syncwarp();
+        if (warp == kMmaWarp) {
+            if (lane == 0) mma_role<D, PK>(p, ms, tab, tmem, smem_q, smem_kv, total);
+            __syncwarp();
+        } else if (warp == kLoadWarp) {
+            if (lane == 0) load_role<D, PK>(p, ms, tab, smem_q, smem_kv, total);
+            __syncwarp();
+        }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == kMmaWarp) {
+    if (warp == kAllocWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
@@ -621,10 +735,18 @@ static int init_device(int dev, DeviceState** out) {
             bool good = g_encode != nullptr;
             good = good && cudaMalloc(&ds.status, 4 * sizeof(int)) == cudaSuccess;
             good = good && cudaMemset(ds.status, 0, 4 * sizeof(int)) == cudaSuccess;
-            good = good && cudaFuncSetAttribute(fa_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                Cfg<64>::kSmemBytes) == cudaSuccess;
-            good = good && cudaFuncSetAttribute(fa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                Cfg<128>::kSmemBytes) == cudaSuccess;
+            good = good && cudaFuncSetAttribute(fa_fwd_kernel<64, false>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                Cfg<64, false>::kSmemBytes) == cudaSuccess;
+            good = good && cudaFuncSetAttribute(fa_fwd_kernel<64, true>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                Cfg<64, true>::kSmemBytes) == cudaSuccess;
+            good = good && cudaFuncSetAttribute(fa_fwd_kernel<128, false>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                Cfg<128, false>::kSmemBytes) == cudaSuccess;
+            good = good && cudaFuncSetAttribute(fa_fwd_kernel<128, true>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                Cfg<128, true>::kSmemBytes) == cudaSuccess;
             ds.status_code = good ? FA_OK : FA_ERR_LAUNCH;
         }
     }
@@ -663,11 +785,23 @@ static bool make_maps(Params& P, const void* q, const void* k, const void* v, in
            encode_map(&P.tm_v, v, dk, sk, box);
 }
 
+#ifndef FA_L2_GROUP_MIB
+#define FA_L2_GROUP_MIB 1000000ll
+#endif
+
 static bool aligned(const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) == 0; }
 
 }  // namespace fa_sm100
 
 using namespace fa_sm100;
+
+#ifdef FA_TRACE
+static unsigned long long* g_trace = nullptr;
+extern "C" int fa_trace_set_buffer(void* dev_ptr) {
+    g_trace = static_cast<unsigned long long*>(dev_ptr);
+    return FA_OK;
+}
+#endif
 
 extern "C" int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                       int N, int d, float scale, int causal, const int32_t* cu_seqlens, void* stream) {
@@ -702,10 +836,21 @@ extern "C" int fa_fwd(const void* q, const void* k, const void* v, void* o, floa
     P.Hkv = Hkv;
     P.N = N;
     P.group = Hq / Hkv;
+    {
+        // K/V of one group of units should stay resident in L2 (126 MB) while
+        // the group's items run: about 48 MiB of K/V per group.
+        const long long kv_bytes = 4ll * N * d;                    // K and V of one kv head
+        long long g_kv = std::max(1ll, (FA_L2_GROUP_MIB << 20) / std::max(1ll, kv_bytes));
+        long long G = std::min<long long>(g_kv * P.group, (long long)B * Hq);
+        P.group_units = (int)std::max(1ll, G);
+    }
     P.causal = causal ? 1 : 0;
     P.packed = packed ? 1 : 0;
     P.scale_log2 = scale * 1.4426950408889634f;
     P.timeout_ns = 2000000000ull;
+#ifdef FA_TRACE
+    P.trace = g_trace;
+#endif
 
     long long items;
     if (!packed) {
@@ -715,10 +860,14 @@ extern "C" int fa_fwd(const void* q, const void* k, const void* v, void* o, floa
     }
     const int grid = (int)std::min<long long>(items, ds->num_sms);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (d == 64)
-        fa_fwd_kernel<64><<<grid, kThreads, Cfg<64>::kSmemBytes, s>>>(P);
+    if (d == 64 && !packed)
+        fa_fwd_kernel<64, false><<<grid, kThreads, Cfg<64, false>::kSmemBytes, s>>>(P);
+    else if (d == 64)
+        fa_fwd_kernel<64, true><<<grid, kThreads, Cfg<64, true>::kSmemBytes, s>>>(P);
+    else if (!packed)
+        fa_fwd_kernel<128, false><<<grid, kThreads, Cfg<128, false>::kSmemBytes, s>>>(P);
     else
-        fa_fwd_kernel<128><<<grid, kThreads, Cfg<128>::kSmemBytes, s>>>(P);
+        fa_fwd_kernel<128, true><<<grid, kThreads, Cfg<128, true>::kSmemBytes, s>>>(P);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
