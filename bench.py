@@ -249,6 +249,25 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------- ranks
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Maximum of a per-rank number over all ranks (the job's time is the
+    slowest rank's); identity on one rank."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_step: float, world: int, steps: int, ms: float) -> float:
+    """Throughput of the whole job: every rank ran ``steps`` steps of
+    ``flops_per_step`` in ``ms`` milliseconds (the maximum over ranks)."""
+    return flops_per_step * world * steps / (ms / 1e3) / 1e12
+
+
 # ------------------------------------------------------------- GPU path
 def main():
     args = parse_args()
@@ -316,16 +335,14 @@ def main():
     ms = ev0.elapsed_time(ev1)
     if world > 1:
         dist.barrier()
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, dev)
     sampler.stop()
     status = fa.fa_get_device_status(stream)
     if status != 0:
         raise fa.FAError(status, "device status after the timed region")
 
     ms_per_step = ms / max(args.steps, 1)
-    value = w.flops() * world * args.steps / (ms / 1e3) / 1e12
+    value = whole_job_tflops(w.flops(), world, args.steps, ms)
     achieved = w.flops() / (ms_per_step / 1e3) / 1e12          # one launch = one step
     peak, peak_sustained, peak_kind = load_peak()
 
@@ -357,12 +374,8 @@ def main():
             e2e_step()
         e1.record(stream)
         e1.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ems], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": w.flops() * world * args.e2e_steps / (ems / 1e3) / 1e12, "unit": UNIT,
+        ems = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": whole_job_tflops(w.flops(), world, args.e2e_steps, ems), "unit": UNIT,
                "h2d_bytes_per_step": int(qh.nbytes + kh.nbytes + vh.nbytes),
                "d2h_bytes_per_step": int(oh.nbytes + lh.nbytes),
                "ms_per_step": ems / args.e2e_steps, "steps": args.e2e_steps}
