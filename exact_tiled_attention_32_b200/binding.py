@@ -28,7 +28,7 @@ FA_ERR_LAUNCH = -7
 FA_ERR_DEVICE_TIMEOUT = -8
 FA_ERR_SEQLENS = -9
 
-EXPORTED = ("fa_fwd", "fa_get_device_status", "fa_status_string")
+EXPORTED = ("fa_fwd", "fa_get_device_status", "fa_status_string", "fa_fwd_noalloc")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -42,6 +42,8 @@ _lib.fa_fwd.argtypes = [
     ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
     ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
 ]
+_lib.fa_fwd_noalloc.restype = ctypes.c_int
+_lib.fa_fwd_noalloc.argtypes = _lib.fa_fwd.argtypes
 _lib.fa_get_device_status.restype = ctypes.c_int
 _lib.fa_get_device_status.argtypes = [ctypes.c_void_p]
 _lib.fa_status_string.restype = ctypes.c_char_p
@@ -75,6 +77,15 @@ def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, cu_seqlens=None, st
     return _lib.fa_fwd(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), int(B), int(Hq),
                        int(Hkv), int(N), int(d), float(scale), int(bool(causal)),
                        _addr(cu_seqlens), _stream(stream))
+
+
+def fa_fwd_noalloc(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, cu_seqlens=None, stream=None) -> int:
+    """The C entry point that allocates no device memory (for callers that
+    cannot allocate: its scratch is a fixed array inside the library).  Same
+    arguments and result as fa_fwd; returns the status."""
+    return _lib.fa_fwd_noalloc(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), int(B), int(Hq),
+                               int(Hkv), int(N), int(d), float(scale), int(bool(causal)),
+                               _addr(cu_seqlens), _stream(stream))
 
 
 def fa_get_device_status(stream=None) -> int:

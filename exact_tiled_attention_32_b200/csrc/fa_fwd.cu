@@ -900,3 +900,146 @@ extern "C" const char* fa_status_string(int status) {
         default: return "unknown status";
     }
 }
+
+// ======================================================= no-allocation entry
+// fa_fwd_noalloc: the same forward for callers that must not allocate device
+// memory.  The only global memory fa_fwd uses beyond the caller's buffers is
+// its device status word, which fa_fwd allocates with cudaMalloc on its first
+// call on a device.  Here that scratch lives in a fixed array compiled into the
+// library instead; every GPU that loads the library holds one copy of it
+// until the process exits.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 256;       // the array's size: the stated maximum
+constexpr size_t kStatusBytes = 4 * sizeof(int);   // what the kernel needs (status words)
+static_assert(kStatusBytes <= kNoAllocScratchBytes, "no-alloc scratch too small");
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+struct NoAllocState {
+    bool init = false;
+    int status_code = FA_OK;
+    int num_sms = 0;
+    int* scratch = nullptr;    // device address of g_noalloc_scratch on this device
+};
+NoAllocState g_noalloc[fa_sm100::kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// One-time set-up per device, with that device current: properties, the
+// tensor-map encoder, the kernels' shared-memory limits, and the device
+// address of the scratch array (the array's name is only a host-side handle).
+// None of these allocate device memory.
+int noalloc_setup(int dev, NoAllocState** out) {
+    using namespace fa_sm100;
+    if (dev < 0 || dev >= kMaxDevices) return FA_ERR_LAUNCH;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    NoAllocState& st = g_noalloc[dev];
+    if (!st.init) {
+        st.init = true;
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+            st.status_code = FA_ERR_LAUNCH;
+        } else if (prop.major != 10 || prop.minor != 0) {
+            st.status_code = FA_ERR_ARCH;
+        } else {
+            st.num_sms = prop.multiProcessorCount;
+            bool good = true;
+            {
+                std::lock_guard<std::mutex> lock2(g_mu);
+                if (!g_encode) {
+                    cudaDriverEntryPointQueryResult q;
+                    void* fn = nullptr;
+                    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+                        q == cudaDriverEntryPointSuccess)
+                        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+                }
+                good = g_encode != nullptr;
+            }
+            void* ptr = nullptr;
+            good = good && cudaGetSymbolAddress(&ptr, g_noalloc_scratch) == cudaSuccess && ptr != nullptr;
+            good = good && cudaFuncSetAttribute(fa_fwd_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                Cfg<64, false>::kSmemBytes) == cudaSuccess;
+            good = good && cudaFuncSetAttribute(fa_fwd_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                Cfg<64, true>::kSmemBytes) == cudaSuccess;
+            good = good && cudaFuncSetAttribute(fa_fwd_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                Cfg<128, false>::kSmemBytes) == cudaSuccess;
+            good = good && cudaFuncSetAttribute(fa_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                Cfg<128, true>::kSmemBytes) == cudaSuccess;
+            st.scratch = static_cast<int*>(ptr);
+            st.status_code = good ? FA_OK : FA_ERR_LAUNCH;
+        }
+    }
+    *out = &st;
+    return st.status_code;
+}
+
+}  // namespace
+
+extern "C" int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                              int Hkv, int N, int d, float scale, int causal, const int32_t* cu_seqlens,
+                              void* stream) {
+    using namespace fa_sm100;
+    const bool packed = cu_seqlens != nullptr;
+    if (B < 0 || N < 0 || Hq < 1) return FA_ERR_SHAPE;
+    if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+    if (Hkv < 1 || Hq % Hkv != 0) return FA_ERR_GQA;
+    if (B == 0 || N == 0) return FA_OK;
+    if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+        return FA_ERR_ALIGN;
+    if (packed && (B > kMaxSeqs || !aligned(cu_seqlens, 4))) return B > kMaxSeqs ? FA_ERR_SHAPE : FA_ERR_ALIGN;
+    const long long rows = packed ? (long long)Hq * N : (long long)B * Hq * N;
+    if (rows > (1ll << 30)) return FA_ERR_SHAPE;
+    // the scratch this call needs must fit the fixed array; the status words
+    // do not grow with the problem, so only a changed build could fail here
+    if (kStatusBytes > kNoAllocScratchBytes) return FA_ERR_SHAPE;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_LAUNCH;
+    NoAllocState* st = nullptr;
+    const int rc = noalloc_setup(dev, &st);
+    if (rc != FA_OK) return rc;
+
+    Params P;
+    std::memset(&P, 0, sizeof(P));
+    if (!make_maps(P, q, k, v, B, Hq, Hkv, N, d, packed)) return FA_ERR_LAUNCH;
+    P.o = o;
+    P.lse = lse;
+    P.cu_seqlens = cu_seqlens;
+    P.status = st->scratch;
+    P.B = B;
+    P.Hq = Hq;
+    P.Hkv = Hkv;
+    P.N = N;
+    P.group = Hq / Hkv;
+    {
+        const long long kv_bytes = 4ll * N * d;
+        long long g_kv = std::max(1ll, (FA_L2_GROUP_MIB << 20) / std::max(1ll, kv_bytes));
+        long long G = std::min<long long>(g_kv * P.group, (long long)B * Hq);
+        P.group_units = (int)std::max(1ll, G);
+    }
+    P.causal = causal ? 1 : 0;
+    P.packed = packed ? 1 : 0;
+    P.scale_log2 = scale * 1.4426950408889634f;
+    P.timeout_ns = 2000000000ull;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the status words keep the previous call's contents: start this call at zero
+    if (cudaMemsetAsync(st->scratch, 0, kStatusBytes, s) != cudaSuccess) return FA_ERR_LAUNCH;
+    long long items;
+    if (!packed) {
+        items = (long long)((N + kRowsPerItem - 1) / kRowsPerItem) * B * Hq;
+    } else {
+        items = (long long)st->num_sms;
+    }
+    const int grid = (int)std::min<long long>(items, st->num_sms);
+    if (d == 64 && !packed)
+        fa_fwd_kernel<64, false><<<grid, kThreads, Cfg<64, false>::kSmemBytes, s>>>(P);
+    else if (d == 64)
+        fa_fwd_kernel<64, true><<<grid, kThreads, Cfg<64, true>::kSmemBytes, s>>>(P);
+    else if (!packed)
+        fa_fwd_kernel<128, false><<<grid, kThreads, Cfg<128, false>::kSmemBytes, s>>>(P);
+    else
+        fa_fwd_kernel<128, true><<<grid, kThreads, Cfg<128, true>::kSmemBytes, s>>>(P);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}

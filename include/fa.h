@@ -92,6 +92,40 @@ int fa_get_device_status(void* stream);
 /* fa_status_string -- static, human-readable text for a status code. */
 const char* fa_status_string(int status);
 
+/*
+ * fa_fwd_noalloc -- fa_fwd for callers that must not allocate device memory.
+ * (An addition of this library; the pages have no counterpart.)
+ *
+ * fa_fwd allocates one small device buffer, its status word, with cudaMalloc
+ * the first time it runs on a device.  Some callers cannot allow that: a
+ * process whose device memory is reserved up front by another allocator
+ * (a serving runtime that claims nearly all of HBM at start-up), so that a
+ * stray cudaMalloc fails or fragments its pool; a latency-critical loop where
+ * cudaMalloc's implicit device-wide synchronisation is not acceptable; or a
+ * code base whose policy forbids new allocations after initialisation.
+ *
+ * This entry point takes the same arguments, has the same layouts, limits and
+ * host-side error codes as fa_fwd, and computes the same result with the same
+ * kernel.  It calls no cudaMalloc, cudaFree or other allocating routine: its
+ * only scratch, the status words (16 bytes whatever the problem size), lives
+ * in a fixed 256-byte array compiled into the library, which every GPU that
+ * loads the library holds until the process exits.  Since the need does not
+ * grow with B, N, Hq or d, no problem is too large for the array.
+ *
+ * The first call on each device sets that device up (device properties, the
+ * kernels' shared-memory limits and the array's device address); make that
+ * first call before any stream capture.
+ *
+ * All calls share the array, which keeps the last call's contents; each call
+ * clears the status words on its stream before its kernel starts.  Calls that
+ * overlap on the GPU (different streams, or several host threads) race on the
+ * status words.  Device-side errors of this entry point are written to that
+ * array only; fa_get_device_status reports the word of fa_fwd, not this one.
+ */
+int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                   int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                   const int32_t* cu_seqlens, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
