@@ -98,7 +98,8 @@ struct alignas(64) Params {
 struct Misc {
     uint64_t bar_q_full, bar_q_empty;
     uint64_t bar_kv_full[kMaxStages], bar_kv_empty[kMaxStages];
-    uint64_t bar_s_full[2], bar_p_full[2], bar_o_final[2], bar_drain;
+    uint64_t bar_s_full[2], bar_o_final[2], bar_drain;
+    uint64_t bar_p_half[2][2];     // P_t keys 0-63 / 64-127 are in TMEM
     uint32_t tmem_base;
     int abort_flag;
     int bad;
@@ -242,6 +243,7 @@ __device__ void load_role(const Params& p, Misc& ms, const SeqTables& tab, uint3
     const uint64_t pol_kv = policy_evict_last();
     const uint64_t pol_q = policy_evict_first();
     uint32_t kv_it = 0, item_n = 0;
+    uint32_t st = 0, ph = 0;      // ring position of tile kv_it: stage and phase parity
     bool ok = true;
     for (int r = 0; ok; ++r) {
         const int idx = item_of_round(r);
@@ -266,10 +268,7 @@ __device__ void load_role(const Params& p, Misc& ms, const SeqTables& tab, uint3
         const int nmax = max(it.n[0], it.n[1]);
         for (int j = 0; j < nmax && ok; ++j) {
             for (int kind = 0; kind < 2; ++kind) {       // K_j then V_j
-                const uint32_t st = kv_it % C::kStages;
-                if (!(ok = wait_bar(smem_u32(&ms.bar_kv_empty[st]), ((kv_it / C::kStages) & 1) ^ 1, p,
-                                    ms, kSiteKvEmpty)))
-                    break;
+                if (!(ok = wait_bar(smem_u32(&ms.bar_kv_empty[st]), ph ^ 1u, p, ms, kSiteKvEmpty))) break;
                 const uint32_t bar = smem_u32(&ms.bar_kv_full[st]);
                 mbar_arrive_expect_tx(bar, C::kTileBytes);
                 const CUtensorMap* map = kind == 0 ? &p.tm_k : &p.tm_v;
@@ -281,6 +280,10 @@ __device__ void load_role(const Params& p, Misc& ms, const SeqTables& tab, uint3
                         tma_load_4d(dst, map, bar, b * 64, kvh, it.tok0 + j * kBlockN, 0, pol_kv);
                 }
                 ++kv_it;
+                if (++st == (uint32_t)C::kStages) {
+                    st = 0;
+                    ph ^= 1u;
+                }
             }
         }
     }
@@ -304,10 +307,12 @@ __device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint64_t dq, uint64_t 
     else
         umma_ss_k64_x4(tmem_s, dq, dk, idesc);
 }
+// Half h of O_t (+)= P_t V: keys 64h .. 64h+63 (P columns 32h.., V rows 64h..)
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint64_t dv, bool accumulate) {
+__device__ __forceinline__ void issue_pv_half(uint32_t tmem_o, uint32_t tmem_p, uint64_t dv, int h, bool accumulate) {
     constexpr uint32_t idesc = idesc_bf16_f32(kBlockM, D, true);
-    umma_ts_kv128_x8(tmem_o, tmem_p, dv, idesc, accumulate ? 1u : 0u);
+    umma_ts_kv64_x4(tmem_o, tmem_p + 32 * h, dv + static_cast<uint64_t>(h * ((64 * 128) >> 4)), idesc,
+                    accumulate ? 1u : 0u);
 }
 
 // The MMA issuer.  Per work item it walks j = 0 .. nmax (nmax = the larger
@@ -323,7 +328,9 @@ __device__ void mma_role(const Params& p, Misc& ms, const SeqTables& tab, uint32
     const uint64_t dk0 = smem_desc_sw128(smem_kv, 16, 1024);              // K-major (K tiles)
     const uint64_t dv0 = smem_desc_sw128(smem_kv, kBoxBytes, 1024);       // MN-major (V tiles)
     constexpr uint64_t kTileStep = C::kTileBytes >> 4;
-    uint32_t kv_it = 0, item_n = 0;
+    // ring position (stage, phase parity) of the next K tile to consume; tiles
+    // arrive in the order K_0, V_0, K_1, V_1, ... of each item
+    uint32_t kst = 0, kph = 0, item_n = 0;
     uint32_t pc[2] = {0, 0};
     bool ok = true;
     for (int r = 0; ok; ++r) {
@@ -334,47 +341,52 @@ __device__ void mma_role(const Params& p, Misc& ms, const SeqTables& tab, uint32
         tc_fence_after();
         ++item_n;
         const int nmax = max(it.n[0], it.n[1]);
-        const uint32_t base = kv_it;
         for (int j = 0; j <= nmax && ok; ++j) {
-            [[maybe_unused]] const uint32_t mit = base / 2 + j;   // iteration counter for the trace
-            FA_TRACE_EV(2, mit, 0);
-            const uint32_t vit = base + 2 * j - 1, vst = vit % C::kStages;
-            const uint32_t kit = base + 2 * j, kst = kit % C::kStages;
-            if (j > 0 && !(ok = wait_bar(smem_u32(&ms.bar_kv_full[vst]), (vit / C::kStages) & 1, p, ms,
-                                         kSiteKvFull)))
-                break;
+            FA_TRACE_EV(2, (item_n == 1 ? j : kTraceIters), 0);
+            // V_{j-1} sits one ring position before K_j
+            const uint32_t vst = kst == 0 ? C::kStages - 1 : kst - 1;
+            const uint32_t vph = kst == 0 ? kph ^ 1u : kph;
+            if (j > 0 && !(ok = wait_bar(smem_u32(&ms.bar_kv_full[vst]), vph, p, ms, kSiteKvFull))) break;
             bool k_ready = false;
-            FA_TRACE_EV(2, mit, 1);
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
                 if (!ok) break;
-                if (j > 0 && j - 1 < it.n[t]) {          // O_t += P_t V_{j-1}
-                    if (!(ok = wait_bar(smem_u32(&ms.bar_p_full[t]), pc[t] & 1, p, ms, kSitePFull))) break;
+                if (j > 0 && j - 1 < it.n[t]) {          // O_t += P_t V_{j-1}, in two key halves
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        if (!(ok = wait_bar(smem_u32(&ms.bar_p_half[t][h]), pc[t] & 1, p, ms, kSitePFull))) break;
+                        tc_fence_after();
+                        if (h == 0) FA_TRACE_EV(2, (item_n == 1 ? j : kTraceIters), 2 + 2 * t);
+                        issue_pv_half<D>(tmem + 256 + t * 128, tmem + t * 128, dv0 + vst * kTileStep, h,
+                                         h > 0 || j - 1 > 0);
+                    }
+                    if (!ok) break;
                     ++pc[t];
-                    tc_fence_after();
-                    FA_TRACE_EV(2, mit, 2 + 2 * t);
-                    issue_pv<D>(tmem + 256 + t * 128, tmem + t * 128, dv0 + vst * kTileStep, j - 1 > 0);
                     if (j - 1 == it.n[t] - 1) umma_commit(smem_u32(&ms.bar_o_final[t]));
                 }
                 if (j < it.n[t]) {                       // S_t = Q_t K_j^T
                     if (!k_ready) {
-                        if (!(ok = wait_bar(smem_u32(&ms.bar_kv_full[kst]), (kit / C::kStages) & 1, p, ms,
-                                            kSiteKvFull)))
-                            break;
+                        if (!(ok = wait_bar(smem_u32(&ms.bar_kv_full[kst]), kph, p, ms, kSiteKvFull))) break;
                         tc_fence_after();
                         k_ready = true;
                     }
                     issue_qk<D>(tmem + t * 128, dq0 + t * kTileStep, dk0 + kst * kTileStep);
                     umma_commit(smem_u32(&ms.bar_s_full[t]));
-                    FA_TRACE_EV(2, mit, 3 + 2 * t);
+                    FA_TRACE_EV(2, (item_n == 1 ? j : kTraceIters), 3 + 2 * t);
                 }
             }
             if (!ok) break;
             if (k_ready) umma_commit(smem_u32(&ms.bar_kv_empty[kst]));
             if (j > 0) umma_commit(smem_u32(&ms.bar_kv_empty[vst]));
             if (j == nmax - 1) umma_commit(smem_u32(&ms.bar_q_empty));
+            if (j < nmax) {                               // next K tile: two positions on
+                kst += 2;
+                if (kst >= (uint32_t)C::kStages) {
+                    kst -= C::kStages;
+                    kph ^= 1u;
+                }
+            }
         }
-        kv_it = base + 2 * nmax;
     }
     // every MMA issued so far must be finished before TMEM and smem go away
     umma_commit(smem_u32(&ms.bar_drain));
@@ -523,6 +535,13 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
                     pk[i] = pack_bf16x2(e0, e1);
                 }
                 tmem_st32(taddr_s + half * 32, pk);
+                if (half == 0) {
+                    // keys 0-63 of P are ready: the tensor core can start on them
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&ms.bar_p_half[t][0]));
+                }
             }
             {
                 float a, b;
@@ -533,7 +552,7 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
             tc_fence_before();
             __syncwarp();
             if (lane == 0) FA_TRACE_EV(t, sc - 1, wq == 0 ? 4 : 4 + wq);
-            if (lane == 0) mbar_arrive(smem_u32(&ms.bar_p_full[t]));
+            if (lane == 0) mbar_arrive(smem_u32(&ms.bar_p_half[t][1]));
         }
         if (!ok) break;
         // epilogue: O / l -> bf16 -> HBM, and the logsumexp
@@ -601,7 +620,8 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(smem_u32(&ms.bar_s_full[t]), 1);
-            mbar_init(smem_u32(&ms.bar_p_full[t]), 4);    // one arrival per warp
+            mbar_init(smem_u32(&ms.bar_p_half[t][0]), 4); // one arrival per warp
+            mbar_init(smem_u32(&ms.bar_p_half[t][1]), 4);
             mbar_init(smem_u32(&ms.bar_o_final[t]), 1);
         }
         ms.abort_flag = 0;

@@ -193,6 +193,23 @@ __device__ __forceinline__ void umma_ts_kv128_x8(uint32_t d_tmem, uint32_t a_tme
         : "memory");
 }
 
+// Half of the P V product: four MMAs over 64 keys.  A = P columns from
+// a_tmem (8 per 16 keys), B = V MN-major from b_desc (+128 per 16 key rows).
+__device__ __forceinline__ void umma_ts_kv64_x4(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p0, pt;\n\t.reg .b32 t1, t2, t3;\n\t.reg .b64 b1, b2, b3;\n\t"
+        "setp.ne.b32 p0, %4, 0;\n\tsetp.eq.b32 pt, %3, %3;\n\t"
+        "add.s32 t1, %1, 8;\n\tadd.s64 b1, %2, 128;\n\tadd.s32 t2, %1, 16;\n\tadd.s64 b2, %2, 256;\n\t"
+        "add.s32 t3, %1, 24;\n\tadd.s64 b3, %2, 384;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [t1], b1, %3, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [t2], b2, %3, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [t3], b3, %3, pt;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // arrive once on `bar` when every tcgen05 op issued so far by this thread is done
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
