@@ -52,6 +52,10 @@ def parse_args():
 
 
 def workload_desc(w):
+    if w.chunk:
+        return (f"{w.name}: {'causal' if w.causal else 'non-causal'} query chunk of {w.N} rows (the last "
+                f"positions) against {w.Nk} keys, B={w.B} Hq={w.Hq} Hkv={w.Hkv} d={w.d}, bf16 N(0,1), "
+                "scale=1/sqrt(d)")
     if w.packed:
         shape = f"packed {w.B} sequences (lengths {min(w.seqlens)}..{max(w.seqlens)}), H={w.Hq}"
     else:
@@ -68,6 +72,8 @@ def config_dict(w, extra=None):
     }
     if w.packed:
         c["seqlens"] = list(w.seqlens)
+    if w.chunk:
+        c["Nk"] = w.Nk
     if extra:
         c.update(extra)
     return c
@@ -183,11 +189,25 @@ def row_flops(w, rows):
         s = np.searchsorted(cu, tok, side="right") - 1
         t = tok - cu[s]
         L = cu[s + 1] - cu[s]
+    elif w.chunk:
+        t = rows % w.N
+        keys = (w.Nk - w.N + t + 1) if w.causal else np.full_like(t, w.Nk)
+        return float(np.sum(4.0 * w.d * keys))
     else:
         t = rows % w.N
         L = np.full_like(t, w.N)
     keys = (t + 1) if w.causal else L
     return float(np.sum(4.0 * w.d * keys))
+
+
+def oracle_rows(w, rows):
+    """The oracle on the given query rows of workload ``w``."""
+    import oracle
+    if w.chunk:
+        return oracle.attention_kv(w.q, w.k, w.v, w.B, w.Hq, w.Hkv, w.N, w.Nk, w.d, w.scale, w.causal,
+                                   rows=rows)
+    return oracle.attention(w.q, w.k, w.v, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal,
+                            w.cu_seqlens, rows=rows)
 
 
 def time_oracle(w, seconds, seed=0):
@@ -200,8 +220,7 @@ def time_oracle(w, seconds, seed=0):
     t0 = time.perf_counter()
     while True:
         rows = oracle_sample_rows(w, 64, rng)
-        oracle.attention(w.q, w.k, w.v, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal,
-                         w.cu_seqlens, rows=rows)
+        oracle_rows(w, rows)
         flops += row_flops(w, rows)
         rows_done += len(rows)
         if time.perf_counter() - t0 >= seconds:
@@ -223,15 +242,13 @@ def run_reference(args, rank):
     rng = np.random.default_rng(1)
     nrows = 32
     for _ in range(args.warmup):
-        oracle.attention(w.q, w.k, w.v, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal,
-                         w.cu_seqlens, rows=oracle_sample_rows(w, nrows, rng))
+        oracle_rows(w, oracle_sample_rows(w, nrows, rng))
     flops = 0.0
     rows_done = 0
     t0 = time.perf_counter()
     for _ in range(args.steps):
         rows = oracle_sample_rows(w, nrows, rng)
-        oracle.attention(w.q, w.k, w.v, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal,
-                         w.cu_seqlens, rows=rows)
+        oracle_rows(w, rows)
         flops += row_flops(w, rows)
         rows_done += len(rows)
     dt = time.perf_counter() - t0
@@ -303,7 +320,11 @@ def main():
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        rc = fa.fa_fwd(q, k, v, o, lse, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal, cu, stream)
+        if w.chunk:
+            rc = fa.fa_fwd_kvcache(q, k, v, o, lse, w.B, w.Hq, w.Hkv, w.N, w.Nk, w.d, w.scale, w.causal,
+                                   stream)
+        else:
+            rc = fa.fa_fwd(q, k, v, o, lse, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal, cu, stream)
         if rc != 0:
             raise fa.FAError(rc)
 
@@ -359,7 +380,10 @@ def main():
             qd = qh.to(dev, non_blocking=True)
             kd = kh.to(dev, non_blocking=True)
             vd = vh.to(dev, non_blocking=True)
-            od, ld = fa.attention_forward(qd, kd, vd, causal=w.causal, scale=w.scale, cu_seqlens=cu)
+            if w.chunk:
+                od, ld = fa.attention_forward_kvcache(qd, kd, vd, causal=w.causal, scale=w.scale)
+            else:
+                od, ld = fa.attention_forward(qd, kd, vd, causal=w.causal, scale=w.scale, cu_seqlens=cu)
             oh.copy_(od, non_blocking=True)
             lh.copy_(ld, non_blocking=True)
 

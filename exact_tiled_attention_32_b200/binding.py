@@ -28,7 +28,8 @@ FA_ERR_LAUNCH = -7
 FA_ERR_DEVICE_TIMEOUT = -8
 FA_ERR_SEQLENS = -9
 
-EXPORTED = ("fa_fwd", "fa_get_device_status", "fa_status_string", "fa_fwd_noalloc")
+EXPORTED = ("fa_fwd", "fa_get_device_status", "fa_status_string", "fa_fwd_noalloc", "fa_fwd_kvcache",
+            "fa_selftest_watchdog")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -44,6 +45,14 @@ _lib.fa_fwd.argtypes = [
 ]
 _lib.fa_fwd_noalloc.restype = ctypes.c_int
 _lib.fa_fwd_noalloc.argtypes = _lib.fa_fwd.argtypes
+_lib.fa_fwd_kvcache.restype = ctypes.c_int
+_lib.fa_fwd_kvcache.argtypes = [
+    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+    ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+    ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
+]
+_lib.fa_selftest_watchdog.restype = ctypes.c_int
+_lib.fa_selftest_watchdog.argtypes = [ctypes.c_int, ctypes.c_void_p]
 _lib.fa_get_device_status.restype = ctypes.c_int
 _lib.fa_get_device_status.argtypes = [ctypes.c_void_p]
 _lib.fa_status_string.restype = ctypes.c_char_p
@@ -86,6 +95,44 @@ def fa_fwd_noalloc(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, cu_seqlens=
     return _lib.fa_fwd_noalloc(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), int(B), int(Hq),
                                int(Hkv), int(N), int(d), float(scale), int(bool(causal)),
                                _addr(cu_seqlens), _stream(stream))
+
+
+def fa_fwd_kvcache(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream=None) -> int:
+    """The C entry point for a chunk of Nq queries (the last Nq positions)
+    against Nk keys; returns the status."""
+    return _lib.fa_fwd_kvcache(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), int(B), int(Hq),
+                               int(Hkv), int(Nq), int(Nk), int(d), float(scale), int(bool(causal)),
+                               _stream(stream))
+
+
+def attention_forward_kvcache(q, k, v, *, causal: bool = False, scale: float | None = None):
+    """O, lse for q [B, Hq, Nq, d] against k/v [B, Hkv, Nk, d] (bf16 CUDA
+    tensors); query row i sits at key position Nk - Nq + i."""
+    import torch
+
+    if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+        raise TypeError("q, k, v must be bfloat16")
+    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    if q.dim() != 4 or k.dim() != 4 or k.shape != v.shape:
+        raise ValueError("q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d]")
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if k.shape[0] != B or k.shape[3] != d:
+        raise ValueError("k/v shape does not match q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    rc = fa_fwd_kvcache(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                        torch.cuda.current_stream(q.device))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_fwd_kvcache")
+    return out, lse
+
+
+def fa_selftest_watchdog(timeout_ms: int, stream=None) -> int:
+    """Launches the watchdog self-test (a bounded wait that runs out)."""
+    return _lib.fa_selftest_watchdog(int(timeout_ms), _stream(stream))
 
 
 def fa_get_device_status(stream=None) -> int:

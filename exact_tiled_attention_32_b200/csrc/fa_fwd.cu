@@ -70,7 +70,9 @@ struct alignas(64) Params {
     float* lse;
     const int32_t* cu_seqlens;
     int* status;
-    int B, Hq, Hkv, N;
+    int B, Hq, Hkv, N;         // N: query rows per sequence (dense) or total tokens (packed)
+    int Nk;                    // dense: keys per sequence (== N except for a query chunk)
+    int q_off;                 // dense: position of query row 0 among the keys (Nk - N for a chunk)
     int group;                 // Hq / Hkv
     int group_units;           // dense: (batch, head) units scheduled together
     int causal, packed;
@@ -136,15 +138,21 @@ struct Item {
     int seq;       // batch index (dense) or sequence index (packed)
     int h;         // query head
     int q0;        // first row of tile 0 inside the sequence
-    int len;       // sequence length
+    int len;       // query rows of the sequence
+    int klen;      // keys of the sequence
+    int qoff;      // position of query row 0 among the keys
     int tok0;      // packed: first token of the sequence
     int n[2];      // key blocks each tile visits (0: tile beyond the sequence)
 };
 
-__device__ __forceinline__ int tile_blocks(int q0, int len, int causal) {
+// Key blocks a 128-row query tile starting at row q0 visits: all of them, or
+// under the causal mask those up to the last valid row's position.
+__device__ __forceinline__ int tile_blocks(int q0, int len, int klen, int qoff, int causal) {
     if (q0 >= len) return 0;
-    const int nkv = (len + kBlockN - 1) / kBlockN;
-    return causal ? min(nkv, q0 / kBlockN + 1) : nkv;
+    const int nkv = (klen + kBlockN - 1) / kBlockN;
+    if (!causal) return nkv;
+    const int last_pos = min(q0 + kBlockM - 1, len - 1) + qoff;
+    return min(nkv, last_pos / kBlockN + 1);
 }
 
 // Dense batches: the (batch, head) units are cut into groups whose K/V fit in
@@ -171,6 +179,8 @@ __device__ __forceinline__ Item decode_item(int idx, const Params& p, const Misc
         it.seq = unit / p.Hq;
         it.h = unit - it.seq * p.Hq;
         it.len = p.N;
+        it.klen = p.Nk;
+        it.qoff = p.q_off;
         it.tok0 = 0;
     } else {
         int lo = 0, hi = ms.pmax - 1;      // smallest level whose start <= idx
@@ -185,10 +195,12 @@ __device__ __forceinline__ Item decode_item(int idx, const Params& p, const Misc
         it.seq = tab.order[k];
         it.tok0 = tab.seq_off[it.seq];
         it.len = tab.seq_off[it.seq + 1] - it.tok0;
+        it.klen = it.len;
+        it.qoff = 0;
     }
     it.q0 = pair * kRowsPerItem;
-    it.n[0] = tile_blocks(it.q0, it.len, p.causal);
-    it.n[1] = tile_blocks(it.q0 + kBlockM, it.len, p.causal);
+    it.n[0] = tile_blocks(it.q0, it.len, it.klen, it.qoff, p.causal);
+    it.n[1] = tile_blocks(it.q0 + kBlockM, it.len, it.klen, it.qoff, p.causal);
     return it;
 }
 
@@ -446,7 +458,8 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
         const int n = t ? it.n[1] : it.n[0];
         if (n == 0) continue;
         const int row = it.q0 + t * kBlockM + r;
-        const int limit = p.causal ? min(row + 1, it.len) : it.len;   // keys [0, limit) allowed
+        // keys [0, limit) are allowed for this row (causal: up to its own position)
+        const int limit = p.causal ? min(row + it.qoff + 1, it.klen) : it.klen;
         float m_used = -INFINITY;    // max the exponentials are taken against (log2 units)
         float l = 0.f;               // running sum of exp2(x - m_used)
         for (int j = 0; j < n; ++j) {
@@ -718,6 +731,21 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     }
 }
 
+// Watchdog self-test: one thread waits, through the same bounded wait the
+// kernel's roles use, on an mbarrier that nothing ever arrives at.  The wait
+// gives up after p.timeout_ns and records FA_ERR_DEVICE_TIMEOUT in the status
+// word; the kernel then returns normally.
+__global__ void fa_watchdog_probe_kernel(const __grid_constant__ Params p) {
+    __shared__ Misc ms;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&ms.bar_q_full), 1);
+        ms.abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)wait_bar(smem_u32(&ms.bar_q_full), 0, p, ms, kSiteQFull);
+}
+
 // =================================================================== host
 struct DeviceState {
     bool init = false;
@@ -785,13 +813,13 @@ static bool encode_map(CUtensorMap* m, const void* base, const uint64_t dims[4],
 }
 
 static bool make_maps(Params& P, const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int N,
-                      int d, bool packed) {
+                      int Nk, int d, bool packed) {
     const uint64_t e = 2;
     if (!packed) {
         const uint64_t dq[4] = {(uint64_t)d, (uint64_t)N, (uint64_t)Hq, (uint64_t)B};
         const uint64_t sq[3] = {d * e, (uint64_t)N * d * e, (uint64_t)Hq * N * d * e};
-        const uint64_t dk[4] = {(uint64_t)d, (uint64_t)N, (uint64_t)Hkv, (uint64_t)B};
-        const uint64_t sk[3] = {d * e, (uint64_t)N * d * e, (uint64_t)Hkv * N * d * e};
+        const uint64_t dk[4] = {(uint64_t)d, (uint64_t)Nk, (uint64_t)Hkv, (uint64_t)B};
+        const uint64_t sk[3] = {d * e, (uint64_t)Nk * d * e, (uint64_t)Hkv * Nk * d * e};
         const uint32_t box[4] = {64, (uint32_t)kBlockM, 1, 1};
         return encode_map(&P.tm_q, q, dq, sq, box) && encode_map(&P.tm_k, k, dk, sk, box) &&
                encode_map(&P.tm_v, v, dk, sk, box);
@@ -809,16 +837,74 @@ static bool make_maps(Params& P, const void* q, const void* k, const void* v, in
 #define FA_L2_GROUP_MIB 1000000ll
 #endif
 
+#ifdef FA_TRACE
+static unsigned long long* g_trace = nullptr;
+#endif
+
 static bool aligned(const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) == 0; }
+
+
+// Fills the launch parameters and launches the kernel variant for (d, packed)
+// on `stream`.  Nk / q_off describe a dense query chunk (Nk keys per sequence,
+// query row 0 at key position q_off); a plain forward has Nk = N, q_off = 0.
+static int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                      int N, int Nk, int q_off, int d, float scale, int causal, const int32_t* cu_seqlens,
+                      cudaStream_t s, int* status, int num_sms) {
+    const bool packed = cu_seqlens != nullptr;
+    Params P;
+    std::memset(&P, 0, sizeof(P));
+    if (!make_maps(P, q, k, v, B, Hq, Hkv, N, Nk, d, packed)) return FA_ERR_LAUNCH;
+    P.o = o;
+    P.lse = lse;
+    P.cu_seqlens = cu_seqlens;
+    P.status = status;
+    P.B = B;
+    P.Hq = Hq;
+    P.Hkv = Hkv;
+    P.N = N;
+    P.Nk = Nk;
+    P.q_off = q_off;
+    P.group = Hq / Hkv;
+    {
+        // K/V of one group of units should stay resident in L2 (126 MB) while
+        // the group's items run
+        const long long kv_bytes = 4ll * Nk * d;                   // K and V of one kv head
+        long long g_kv = std::max(1ll, (FA_L2_GROUP_MIB << 20) / std::max(1ll, kv_bytes));
+        long long G = std::min<long long>(g_kv * P.group, (long long)B * Hq);
+        P.group_units = (int)std::max(1ll, G);
+    }
+    P.causal = causal ? 1 : 0;
+    P.packed = packed ? 1 : 0;
+    P.scale_log2 = scale * 1.4426950408889634f;
+    P.timeout_ns = 2000000000ull;
+#ifdef FA_TRACE
+    P.trace = g_trace;
+#endif
+    long long items;
+    if (!packed) {
+        items = (long long)((N + kRowsPerItem - 1) / kRowsPerItem) * B * Hq;
+    } else {
+        items = (long long)num_sms;    // exact count is known only on the device
+    }
+    const int grid = (int)std::min<long long>(items, num_sms);
+    if (d == 64 && !packed)
+        fa_fwd_kernel<64, false><<<grid, kThreads, Cfg<64, false>::kSmemBytes, s>>>(P);
+    else if (d == 64)
+        fa_fwd_kernel<64, true><<<grid, kThreads, Cfg<64, true>::kSmemBytes, s>>>(P);
+    else if (!packed)
+        fa_fwd_kernel<128, false><<<grid, kThreads, Cfg<128, false>::kSmemBytes, s>>>(P);
+    else
+        fa_fwd_kernel<128, true><<<grid, kThreads, Cfg<128, true>::kSmemBytes, s>>>(P);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
 
 }  // namespace fa_sm100
 
 using namespace fa_sm100;
 
 #ifdef FA_TRACE
-static unsigned long long* g_trace = nullptr;
 extern "C" int fa_trace_set_buffer(void* dev_ptr) {
-    g_trace = static_cast<unsigned long long*>(dev_ptr);
+    fa_sm100::g_trace = static_cast<unsigned long long*>(dev_ptr);
     return FA_OK;
 }
 #endif
@@ -844,50 +930,44 @@ extern "C" int fa_fwd(const void* q, const void* k, const void* v, void* o, floa
     const int st = init_device(dev, &ds);
     if (st != FA_OK) return st;
 
+    return launch_fwd(q, k, v, o, lse, B, Hq, Hkv, N, N, 0, d, scale, causal, cu_seqlens,
+                      static_cast<cudaStream_t>(stream), ds->status, ds->num_sms);
+}
+
+extern "C" int fa_fwd_kvcache(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                              int Hkv, int Nq, int Nk, int d, float scale, int causal, void* stream) {
+    if (B < 0 || Nq < 0 || Nk < 0 || Hq < 1) return FA_ERR_SHAPE;
+    if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+    if (Hkv < 1 || Hq % Hkv != 0) return FA_ERR_GQA;
+    if (B == 0 || Nq == 0) return FA_OK;
+    if (Nk == 0 || (causal && Nk < Nq)) return FA_ERR_SHAPE;
+    if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+        return FA_ERR_ALIGN;
+    if ((long long)B * Hq * Nq > (1ll << 30) || (long long)B * Hkv * Nk > (1ll << 31)) return FA_ERR_SHAPE;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_LAUNCH;
+    DeviceState* ds = nullptr;
+    const int st = init_device(dev, &ds);
+    if (st != FA_OK) return st;
+    // the chunk's rows are the last Nq positions of the key sequence
+    return launch_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, causal ? Nk - Nq : 0, d, scale, causal, nullptr,
+                      static_cast<cudaStream_t>(stream), ds->status, ds->num_sms);
+}
+
+extern "C" int fa_selftest_watchdog(int timeout_ms, void* stream) {
+    if (timeout_ms < 1 || timeout_ms > 2000) return FA_ERR_SHAPE;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_LAUNCH;
+    DeviceState* ds = nullptr;
+    const int st = init_device(dev, &ds);
+    if (st != FA_OK) return st;
     Params P;
     std::memset(&P, 0, sizeof(P));
-    if (!make_maps(P, q, k, v, B, Hq, Hkv, N, d, packed)) return FA_ERR_LAUNCH;
-    P.o = o;
-    P.lse = lse;
-    P.cu_seqlens = cu_seqlens;
     P.status = ds->status;
-    P.B = B;
-    P.Hq = Hq;
-    P.Hkv = Hkv;
-    P.N = N;
-    P.group = Hq / Hkv;
-    {
-        // K/V of one group of units should stay resident in L2 (126 MB) while
-        // the group's items run: about 48 MiB of K/V per group.
-        const long long kv_bytes = 4ll * N * d;                    // K and V of one kv head
-        long long g_kv = std::max(1ll, (FA_L2_GROUP_MIB << 20) / std::max(1ll, kv_bytes));
-        long long G = std::min<long long>(g_kv * P.group, (long long)B * Hq);
-        P.group_units = (int)std::max(1ll, G);
-    }
-    P.causal = causal ? 1 : 0;
-    P.packed = packed ? 1 : 0;
-    P.scale_log2 = scale * 1.4426950408889634f;
-    P.timeout_ns = 2000000000ull;
-#ifdef FA_TRACE
-    P.trace = g_trace;
-#endif
-
-    long long items;
-    if (!packed) {
-        items = (long long)((N + kRowsPerItem - 1) / kRowsPerItem) * B * Hq;
-    } else {
-        items = (long long)ds->num_sms;    // exact count is known only on the device
-    }
-    const int grid = (int)std::min<long long>(items, ds->num_sms);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (d == 64 && !packed)
-        fa_fwd_kernel<64, false><<<grid, kThreads, Cfg<64, false>::kSmemBytes, s>>>(P);
-    else if (d == 64)
-        fa_fwd_kernel<64, true><<<grid, kThreads, Cfg<64, true>::kSmemBytes, s>>>(P);
-    else if (!packed)
-        fa_fwd_kernel<128, false><<<grid, kThreads, Cfg<128, false>::kSmemBytes, s>>>(P);
-    else
-        fa_fwd_kernel<128, true><<<grid, kThreads, Cfg<128, true>::kSmemBytes, s>>>(P);
+    P.timeout_ns = static_cast<unsigned long long>(timeout_ms) * 1000000ull;
+    fa_watchdog_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(P);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
@@ -1020,46 +1100,9 @@ extern "C" int fa_fwd_noalloc(const void* q, const void* k, const void* v, void*
     const int rc = noalloc_setup(dev, &st);
     if (rc != FA_OK) return rc;
 
-    Params P;
-    std::memset(&P, 0, sizeof(P));
-    if (!make_maps(P, q, k, v, B, Hq, Hkv, N, d, packed)) return FA_ERR_LAUNCH;
-    P.o = o;
-    P.lse = lse;
-    P.cu_seqlens = cu_seqlens;
-    P.status = st->scratch;
-    P.B = B;
-    P.Hq = Hq;
-    P.Hkv = Hkv;
-    P.N = N;
-    P.group = Hq / Hkv;
-    {
-        const long long kv_bytes = 4ll * N * d;
-        long long g_kv = std::max(1ll, (FA_L2_GROUP_MIB << 20) / std::max(1ll, kv_bytes));
-        long long G = std::min<long long>(g_kv * P.group, (long long)B * Hq);
-        P.group_units = (int)std::max(1ll, G);
-    }
-    P.causal = causal ? 1 : 0;
-    P.packed = packed ? 1 : 0;
-    P.scale_log2 = scale * 1.4426950408889634f;
-    P.timeout_ns = 2000000000ull;
-
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // the status words keep the previous call's contents: start this call at zero
     if (cudaMemsetAsync(st->scratch, 0, kStatusBytes, s) != cudaSuccess) return FA_ERR_LAUNCH;
-    long long items;
-    if (!packed) {
-        items = (long long)((N + kRowsPerItem - 1) / kRowsPerItem) * B * Hq;
-    } else {
-        items = (long long)st->num_sms;
-    }
-    const int grid = (int)std::min<long long>(items, st->num_sms);
-    if (d == 64 && !packed)
-        fa_fwd_kernel<64, false><<<grid, kThreads, Cfg<64, false>::kSmemBytes, s>>>(P);
-    else if (d == 64)
-        fa_fwd_kernel<64, true><<<grid, kThreads, Cfg<64, true>::kSmemBytes, s>>>(P);
-    else if (!packed)
-        fa_fwd_kernel<128, false><<<grid, kThreads, Cfg<128, false>::kSmemBytes, s>>>(P);
-    else
-        fa_fwd_kernel<128, true><<<grid, kThreads, Cfg<128, true>::kSmemBytes, s>>>(P);
-    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+    return launch_fwd(q, k, v, o, lse, B, Hq, Hkv, N, N, 0, d, scale, causal, cu_seqlens, s, st->scratch,
+                      st->num_sms);
 }

@@ -29,6 +29,8 @@ one stream; for the packed batch the sequence lengths are drawn first):
 * c3: B=1, H=32, N=16384, d=128, causal
 * c4: B=1, Hq=32, Hkv=8, N=32768, d=128, causal
 * c5: 16 sequences, lengths uniform in [512, 8192], H=16, d=128, causal
+* p3: a query chunk of 2048 rows (the last positions) against 16384 keys,
+  B=1, H=32, d=128, causal -- the chunked-prefill shape
 """
 from __future__ import annotations
 
@@ -138,6 +140,7 @@ class Workload:
     causal: bool
     seed: int
     seqlens: list[int] | None = None
+    Nk: int | None = None   # dense query chunk: keys per sequence (the chunk is the last N positions)
     q: np.ndarray | None = field(default=None, repr=False)
     k: np.ndarray | None = field(default=None, repr=False)
     v: np.ndarray | None = field(default=None, repr=False)
@@ -160,9 +163,19 @@ class Workload:
     def lengths(self) -> list[int]:
         return list(self.seqlens) if self.packed else [self.N] * self.B
 
+    @property
+    def chunk(self) -> bool:
+        return self.Nk is not None and not self.packed
+
     def flops(self) -> float:
         """4*L^2*d per (sequence, head), halved when causal (the convention of
-        the metric; the count is of the dense score matrix)."""
+        the metric; the count is of the dense score matrix).  A query chunk
+        counts 4*d per attended key per row: 4*d*Nq*Nk, or under the causal
+        mask 4*d*sum_i (Nk - Nq + i + 1)."""
+        if self.chunk:
+            Nq, Nk = self.N, self.Nk
+            keys = Nq * (Nk - Nq) + Nq * (Nq + 1) / 2 if self.causal else Nq * Nk
+            return 4.0 * self.d * keys * self.B * self.Hq
         f = sum(4.0 * L * L * self.d for L in self.lengths) * self.Hq
         return f / 2 if self.causal else f
 
@@ -170,6 +183,8 @@ class Workload:
         return (self.N, self.Hq, self.d) if self.packed else (self.B, self.Hq, self.N, self.d)
 
     def kv_shape(self):
+        if self.chunk:
+            return (self.B, self.Hkv, self.Nk, self.d)
         return (self.N, self.Hkv, self.d) if self.packed else (self.B, self.Hkv, self.N, self.d)
 
     def total_rows(self) -> int:
@@ -216,7 +231,11 @@ def config(name: str) -> Workload:
         return Workload("c4", 1, 32, 8, 32768, 128, True, 1004)
     if name == "c5":
         return packed_workload("c5", 16, 512, 8192, 16, 128, True, 1005)
+    if name == "p3":
+        # a 2048-row prefill chunk at the end of a 16384-token sequence,
+        # c3's heads and head size
+        return Workload("p3", 1, 32, 32, 2048, 128, True, 1006, Nk=16384)
     raise KeyError(name)
 
 
-CONFIGS = ("c1", "c2nc", "c2c", "c3", "c4", "c5")
+CONFIGS = ("c1", "c2nc", "c2c", "c3", "c4", "c5", "p3")

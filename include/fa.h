@@ -81,6 +81,29 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
            const int32_t* cu_seqlens, void* stream);
 
 /*
+ * fa_fwd_kvcache -- forward for a chunk of Nq queries against Nk keys (dense
+ * batches), asynchronous on `stream`.  This is the shape of chunked prefill
+ * ("FlashAttention and Chunked Prefill Mechanics", section 1: a long prompt is
+ * split into chunks, each attending to the keys and values of all earlier
+ * tokens) and of attending to a KV cache ("Flash Attention", KV Cache named as
+ * composable with the method).
+ *
+ *   q, o   [B, Hq, Nq, d] bf16      k, v  [B, Hkv, Nk, d] bf16
+ *   lse    [B, Hq, Nq] fp32         Nq >= 1, Nk >= 1
+ *
+ * The chunk's rows are the LAST Nq positions of the Nk-long sequence: query
+ * row i sits at position Nk - Nq + i.  causal != 0 allows key j for row i iff
+ * j <= Nk - Nq + i (so Nk >= Nq is required); causal == 0 allows every key.
+ * With Nq == Nk this is exactly fa_fwd.  Running a sequence through
+ * consecutive chunks [a, b) against keys [0, b) reproduces the rows of the
+ * whole causal forward.  Other arguments, ownership and errors as fa_fwd
+ * (FA_ERR_SHAPE also for Nk == 0, or causal with Nk < Nq).
+ */
+int fa_fwd_kvcache(const void* q, const void* k, const void* v, void* o, float* lse,
+                   int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                   void* stream);
+
+/*
  * fa_get_device_status -- reads and clears the status word of the current
  * device.  Synchronises `stream` (a cudaStream_t) first, so it reports every
  * fa_fwd launched on that stream before the call.  Returns FA_OK, a negative
@@ -88,6 +111,17 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
  * if the runtime reports an error.
  */
 int fa_get_device_status(void* stream);
+
+/*
+ * fa_selftest_watchdog -- checks the device-side watchdog without any fault.
+ * Launches on `stream` one thread that waits, through the same bounded wait
+ * the forward kernel uses, on a barrier nothing ever completes; after
+ * timeout_ms (1 .. 2000) the wait gives up, records FA_ERR_DEVICE_TIMEOUT in
+ * the status word (read it with fa_get_device_status) and the kernel returns.
+ * The context stays usable.  Returns FA_OK once launched, FA_ERR_SHAPE for a
+ * timeout out of range, or the device set-up error.
+ */
+int fa_selftest_watchdog(int timeout_ms, void* stream);
 
 /* fa_status_string -- static, human-readable text for a status code. */
 const char* fa_status_string(int status);

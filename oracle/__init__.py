@@ -18,6 +18,9 @@ Every function cites the passage of the pages it follows in ``oracle.c``:
                           Memory Analysis").
 * ``attention_tiled``  -- the tiled forward with the online-softmax update
                           (14cs17 page, "Flash Attention Algorithm"), in fp64.
+* ``attention_kv``     -- a chunk of queries against a longer key sequence,
+                          the chunk's rows being its last positions (xspy.com,
+                          section 1, chunked prefill).
 
 Pins (in ``tests/test_oracle.py``): the worked examples of both pages, row sums
 of one, torch's fp64 scaled-dot-product attention as an independent library
@@ -76,6 +79,11 @@ def bind(path: str):
         u16p, u16p, u16p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
         ctypes.c_int, ctypes.c_double, ctypes.c_int, i32p, ctypes.c_int, ctypes.c_int,
         i64p, dp, dp,
+    ]
+    lib.oracle_attention_kv.restype = ctypes.c_int
+    lib.oracle_attention_kv.argtypes = [
+        u16p, u16p, u16p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_int, ctypes.c_double, ctypes.c_int, i64p, ctypes.c_int64, dp, dp, ctypes.c_int,
     ]
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_num_threads.argtypes = []
@@ -172,6 +180,26 @@ def attention_tiled(q, k, v, B, Hq, Hkv, N, d, scale, causal, cu_seqlens=None,
         _ptr(lse, ctypes.c_double))
     if rc != 0:
         raise ValueError("oracle_attention_tiled: bad arguments")
+    return o, lse
+
+
+def attention_kv(q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal, rows=None, nthreads=0,
+                 lib=None) -> tuple[np.ndarray, np.ndarray]:
+    """Materialised fp64 attention of a chunk of Nq queries (the last Nq
+    positions) against Nk keys.  q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] bf16 bits;
+    row ids (b*Hq+h)*Nq+i.  Returns (o [nrows, d], lse [nrows])."""
+    q, k, v = _as_bits(q), _as_bits(k), _as_bits(v)
+    total = B * Hq * Nq
+    r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    nrows = total if r is None else r.size
+    o = np.zeros((nrows, d), dtype=np.float64)
+    lse = np.zeros(nrows, dtype=np.float64)
+    rc = _load(lib).oracle_attention_kv(
+        _ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16), _ptr(v, ctypes.c_uint16),
+        B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)), _ptr(r, ctypes.c_int64), nrows,
+        _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_attention_kv: bad arguments or row id out of range")
     return o, lse
 
 

@@ -344,6 +344,74 @@ int oracle_attention_tiled(const uint16_t* q, const uint16_t* k, const uint16_t*
     return 0;
 }
 
+/* ------------------------------------------------------------------------ */
+/* A chunk of queries against a longer key sequence (xspy.com page, section  */
+/* 1: chunked prefill splits a long prompt into chunks, each attending to    */
+/* the keys of every earlier token; 14cs17 page: KV Cache is composable).    */
+/* Query row i of the chunk sits at key position Nk - Nq + i; causal allows  */
+/* key j iff j <= that position.  Dense layout: q [B,Hq,Nq,d],              */
+/* k, v [B,Hkv,Nk,d]; row id (b*Hq + h)*Nq + i; o nrows x d, lse nrows.     */
+/* Standard attention again: each score row is materialised in full.        */
+/* ------------------------------------------------------------------------ */
+int oracle_attention_kv(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                        int B, int Hq, int Hkv, int Nq, int Nk, int d, double scale,
+                        int causal, const int64_t* rows, int64_t nrows,
+                        double* o, double* lse, int nthreads) {
+    if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || Nk < 0 || Nq < 0) return -1;
+    const int group = Hq / Hkv;
+    const int64_t total = (int64_t)B * Hq * Nq;
+    if (!rows) nrows = total;
+    int bad = 0;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel
+    {
+        double* s = (double*)malloc(sizeof(double) * (size_t)(Nk > 0 ? Nk : 1));
+        double* qv = (double*)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 8)
+        for (int64_t r = 0; r < nrows; ++r) {
+            int64_t rowid = rows ? rows[r] : r;
+            if (rowid < 0 || rowid >= total) { bad = 1; continue; }
+            const int64_t i = rowid % Nq;
+            const int64_t bh = rowid / Nq;
+            const int h = (int)(bh % Hq);
+            const int64_t b = bh / Hq;
+            const int hk = h / group;
+            const int64_t pos = (int64_t)Nk - Nq + i;          /* the row's key position */
+            const uint16_t* qrow = q + ((b * Hq + h) * Nq + i) * d;
+            const uint16_t* k0 = k + ((b * Hkv + hk) * (int64_t)Nk) * d;
+            const uint16_t* v0 = v + ((b * Hkv + hk) * (int64_t)Nk) * d;
+            for (int c = 0; c < d; ++c) qv[c] = bf16_to_double(qrow[c]);
+            double m = -INFINITY;
+            for (int64_t j = 0; j < Nk; ++j) {
+                if (causal && j > pos) { s[j] = -INFINITY; continue; }
+                double dot = 0.0;
+                for (int c = 0; c < d; ++c) dot += qv[c] * bf16_to_double(k0[j * d + c]);
+                s[j] = scale * dot;
+                if (s[j] > m) m = s[j];
+            }
+            double* orow = o + r * d;
+            for (int c = 0; c < d; ++c) orow[c] = 0.0;
+            if (m == -INFINITY) { lse[r] = -INFINITY; continue; }
+            double l = 0.0;
+            for (int64_t j = 0; j < Nk; ++j) {
+                s[j] = exp(s[j] - m);
+                l += s[j];
+            }
+            for (int64_t j = 0; j < Nk; ++j) {
+                if (s[j] == 0.0) continue;
+                double pj = s[j] / l;
+                for (int c = 0; c < d; ++c) orow[c] += pj * bf16_to_double(v0[j * d + c]);
+            }
+            lse[r] = m + log(l);
+        }
+        free(s);
+        free(qv);
+    }
+    return bad ? -1 : 0;
+}
+
 /* Number of worker threads OpenMP will use (reported by the CPU baseline). */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

@@ -385,6 +385,7 @@ MUTATIONS = {
                            "r->qrow = a->q + ((b * a->Hq + r->h) * N) * a->d + r->t;"),
     "online_no_rescale": ("double carry = (m_run == -INFINITY) ? 0.0 : exp(m_run - m_new);",
                           "double carry = (m_run == -INFINITY) ? 0.0 : 1.0;"),
+    "chunk_top_left_mask": ("const int64_t pos = (int64_t)Nk - Nq + i;", "const int64_t pos = i;"),
 }
 
 
@@ -412,6 +413,17 @@ def _pin_suite(lib):
 
     checks["torch_causal_gqa"] = lambda: torch_pin(1, 4, 2, 37, 16, True)
     checks["torch_dense"] = lambda: torch_pin(2, 2, 2, 20, 16, False)
+
+    def chunk_pin():
+        s = syn.Stream(99)
+        q = s.normal_bf16((1, 2, 5, 16))
+        k = s.normal_bf16((1, 1, 23, 16))
+        v = s.normal_bf16((1, 1, 23, 16))
+        o, lse = oracle.attention_kv(q, k, v, 1, 2, 1, 5, 23, 16, 0.3, True, lib=lib)
+        o_t, lse_t = _torch_chunk(q, k, v, 1, 2, 1, 5, 23, 16, 0.3, True)
+        return np.max(np.abs(o - o_t)) < 1e-12 and np.max(np.abs(lse - lse_t)) < 1e-12
+
+    checks["torch_chunk"] = chunk_pin
     for name, fn in checks.items():
         try:
             ok = bool(fn())
@@ -440,3 +452,90 @@ def test_planted_mistake_is_caught(name, tmp_path):
                            str(path), "-o", str(so), "-lm"])
     failed = _pin_suite(oracle.bind(str(so)))
     assert failed, f"planted mistake {name} passed every pin"
+
+
+# --------------------------------------------------------------------------
+# a chunk of queries against a longer key sequence (chunked prefill)
+# --------------------------------------------------------------------------
+
+def _torch_chunk(q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal):
+    """torch fp64 SDPA with an explicit mask: row i of the chunk may see key
+    j iff j <= Nk - Nq + i (bottom-right alignment)."""
+    qt, kt, vt = (torch.from_numpy(_f64(a)) for a in (q, k, v))
+    g = Hq // Hkv
+    kr, vr = kt.repeat_interleave(g, dim=1), vt.repeat_interleave(g, dim=1)
+    mask = None
+    if causal:
+        i = torch.arange(Nq)[:, None]
+        j = torch.arange(Nk)[None, :]
+        mask = j <= (Nk - Nq + i)
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kr, vr, attn_mask=mask, scale=scale)
+    s = scale * qt @ kr.transpose(-1, -2)
+    if causal:
+        s = s.masked_fill(~mask, -math.inf)
+    return o.reshape(-1, d).numpy(), torch.logsumexp(s, dim=-1).reshape(-1).numpy()
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Nq,Nk,d,causal", [
+    (2, 4, 2, 5, 37, 16, True),
+    (1, 4, 4, 37, 37, 32, True),
+    (1, 2, 1, 1, 130, 64, True),
+    (2, 2, 2, 20, 50, 16, False),
+    (1, 8, 2, 129, 300, 32, True),
+])
+def test_chunk_attention_matches_torch_fp64(B, Hq, Hkv, Nq, Nk, d, causal):
+    s = syn.Stream(61 + Nq + Nk)
+    q = s.normal_bf16((B, Hq, Nq, d))
+    k = s.normal_bf16((B, Hkv, Nk, d))
+    v = s.normal_bf16((B, Hkv, Nk, d))
+    o, lse = oracle.attention_kv(q, k, v, B, Hq, Hkv, Nq, Nk, d, 0.3, causal)
+    o_t, lse_t = _torch_chunk(q, k, v, B, Hq, Hkv, Nq, Nk, d, 0.3, causal)
+    assert np.max(np.abs(o - o_t)) < 1e-12
+    assert np.max(np.abs(lse - lse_t)) < 1e-12
+
+
+def test_chunk_brute_force_tiny():
+    B, Hq, Hkv, Nq, Nk, d = 1, 2, 1, 3, 7, 4
+    s = syn.Stream(71)
+    q = s.normal_bf16((B, Hq, Nq, d))
+    k = s.normal_bf16((B, Hkv, Nk, d))
+    v = s.normal_bf16((B, Hkv, Nk, d))
+    o, lse = oracle.attention_kv(q, k, v, B, Hq, Hkv, Nq, Nk, d, 0.8, True)
+    qf, kf, vf = _f64(q[0]), _f64(k[0]), _f64(v[0])
+    for h in range(Hq):
+        for i in range(Nq):
+            pos = Nk - Nq + i
+            w = [math.exp(0.8 * float(np.dot(qf[h, i], kf[0, j]))) for j in range(pos + 1)]
+            ref = sum(wj * vf[0, j] for j, wj in enumerate(w)) / sum(w)
+            r = h * Nq + i
+            assert np.max(np.abs(o[r] - ref)) < 1e-12
+            assert abs(lse[r] - math.log(sum(w))) < 1e-12
+
+
+def test_chunk_equal_lengths_is_the_plain_forward():
+    B, H, N, d = 2, 3, 70, 16
+    s = syn.Stream(72)
+    q, k, v = (s.normal_bf16((B, H, N, d)) for _ in range(3))
+    for causal in (False, True):
+        o1, l1 = oracle.attention(q, k, v, B, H, H, N, d, 0.25, causal)
+        o2, l2 = oracle.attention_kv(q, k, v, B, H, H, N, N, d, 0.25, causal)
+        assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_chunked_prefill_reproduces_the_whole_causal_forward():
+    """xspy.com page, section 1: prefill split into chunks, each chunk's
+    queries attending to the keys of all tokens up to its end, gives the rows
+    of the whole causal forward."""
+    B, H, N, d = 1, 2, 100, 16
+    s = syn.Stream(73)
+    q, k, v = (s.normal_bf16((B, H, N, d)) for _ in range(3))
+    o_full, l_full = oracle.attention(q, k, v, B, H, H, N, d, 0.25, True)
+    o_full = o_full.reshape(B, H, N, d)
+    l_full = l_full.reshape(B, H, N)
+    for a, b in ((0, 17), (17, 64), (64, 100)):
+        qc = np.ascontiguousarray(q[:, :, a:b])
+        kc = np.ascontiguousarray(k[:, :, :b])
+        vc = np.ascontiguousarray(v[:, :, :b])
+        o, l = oracle.attention_kv(qc, kc, vc, B, H, H, b - a, b, d, 0.25, True)
+        assert np.array_equal(o.reshape(B, H, b - a, d), o_full[:, :, a:b])
+        assert np.array_equal(l.reshape(B, H, b - a), l_full[:, :, a:b])
