@@ -90,6 +90,14 @@ def load_peak():
         return FALLBACK_PEAK_TFLOPS, None, "fallback"
 
 
+def load_hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
 def source_sha():
     h = hashlib.sha256()
     for rel in ("exact_tiled_attention_32_b200/csrc/fa_fwd.cu", "exact_tiled_attention_32_b200/csrc/sm100_ptx.cuh"):
@@ -318,9 +326,19 @@ def main():
     lse_shape = (w.Hq, w.N) if w.packed else (w.B, w.Hq, w.N)
     lse = torch.empty(lse_shape, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
+    splits, ws, ws_bytes = 1, None, 0
+    if w.decode:
+        splits = fa.fa_splitkv_num_splits(w.B, w.Hq, w.Hkv, w.N, w.Nk, w.d)
+        if splits < 0:
+            raise fa.FAError(splits, "fa_splitkv_num_splits")
+        ws_bytes = fa.fa_splitkv_workspace_bytes(w.B, w.Hq, w.N, w.d, splits)
+        ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
 
     def step():
-        if w.chunk:
+        if w.decode:
+            rc = fa.fa_fwd_splitkv(q, k, v, o, lse, w.B, w.Hq, w.Hkv, w.N, w.Nk, w.d, w.scale, w.causal,
+                                   splits, ws, ws_bytes, stream)
+        elif w.chunk:
             rc = fa.fa_fwd_kvcache(q, k, v, o, lse, w.B, w.Hq, w.Hkv, w.N, w.Nk, w.d, w.scale, w.causal,
                                    stream)
         else:
@@ -380,7 +398,10 @@ def main():
             qd = qh.to(dev, non_blocking=True)
             kd = kh.to(dev, non_blocking=True)
             vd = vh.to(dev, non_blocking=True)
-            if w.chunk:
+            if w.decode:
+                od, ld = fa.attention_forward_splitkv(qd, kd, vd, causal=w.causal, scale=w.scale,
+                                                      num_splits=splits, workspace=ws)
+            elif w.chunk:
                 od, ld = fa.attention_forward_kvcache(qd, kd, vd, causal=w.causal, scale=w.scale)
             else:
                 od, ld = fa.attention_forward(qd, kd, vd, causal=w.causal, scale=w.scale, cu_seqlens=cu)
@@ -414,18 +435,34 @@ def main():
     if rank != 0:
         return
     clocks = sampler.summary(t_host0, t_host1)
+    launches_per_step = 1
+    if w.decode:
+        # HBM-bound: the forward streams the K/V cache once; the roofline is
+        # bytes over the whole step (forward + the split merge), against the
+        # measured copy bandwidth
+        launches_per_step = 2 if splits > 1 else 1
+        hbm_peak, hbm_kind = load_hbm_peak()
+        gbs = w.hbm_bytes() / (ms_per_step / 1e3) / 1e9
+        roofline = {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": gbs / hbm_peak, "traffic": profiled_traffic(args.config),
+                    "peak_source": f"MEASURED_PEAKS.json hbm_gbs, of {hbm_kind}",
+                    "algorithmic_bytes": w.hbm_bytes(),
+                    "timed": f"whole step: split-key forward + merge of {splits} splits"}
+    else:
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                    "frac": achieved / peak, "traffic": profiled_traffic(args.config),
+                    "peak_source": f"MEASURED_PEAKS.json bf16_tflops (burst), of {peak_kind}",
+                    "frac_of_sustained": (achieved / peak_sustained) if peak_sustained else None}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": config_dict(w, {"parallelism": f"replicas x{world} (independent problems, no collective)"}),
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
-                     "frac": achieved / peak, "traffic": profiled_traffic(args.config),
-                     "peak_source": f"MEASURED_PEAKS.json bf16_tflops (burst), of {peak_kind}",
-                     "frac_of_sustained": (achieved / peak_sustained) if peak_sustained else None},
+        "config": config_dict(w, {"parallelism": f"replicas x{world} (independent problems, no collective)",
+                                  **({"num_splits": splits} if w.decode else {})}),
+        "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * launches_per_step,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

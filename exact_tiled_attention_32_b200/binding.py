@@ -1,7 +1,7 @@
 """Python binding of libfa.so (argument marshalling only).
 
-The names follow the C ABI in ``include/fa.h``: ``fa_fwd``,
-``fa_get_device_status`` and ``fa_status_string``.  ``attention_forward`` is
+The names follow the C ABI in ``include/fa.h`` (``fa_fwd``, ``fa_fwd_kvcache``,
+``fa_fwd_splitkv``, ``fa_get_device_status``, ``fa_status_string`` ...).  ``attention_forward`` is
 the convenience call on torch tensors: it checks shapes, allocates O and the
 logsumexp with torch, and calls ``fa_fwd`` on the current CUDA stream.  Every
 step of the computation runs in the CUDA kernels of libfa.so; there is no other
@@ -29,7 +29,7 @@ FA_ERR_DEVICE_TIMEOUT = -8
 FA_ERR_SEQLENS = -9
 
 EXPORTED = ("fa_fwd", "fa_get_device_status", "fa_status_string", "fa_fwd_noalloc", "fa_fwd_kvcache",
-            "fa_selftest_watchdog")
+            "fa_selftest_watchdog", "fa_fwd_splitkv", "fa_splitkv_num_splits", "fa_splitkv_workspace_bytes")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -51,6 +51,14 @@ _lib.fa_fwd_kvcache.argtypes = [
     ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
     ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
 ]
+_lib.fa_fwd_splitkv.restype = ctypes.c_int
+_lib.fa_fwd_splitkv.argtypes = _lib.fa_fwd_kvcache.argtypes[:-1] + [
+    ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+]
+_lib.fa_splitkv_num_splits.restype = ctypes.c_int
+_lib.fa_splitkv_num_splits.argtypes = [ctypes.c_int] * 6
+_lib.fa_splitkv_workspace_bytes.restype = ctypes.c_size_t
+_lib.fa_splitkv_workspace_bytes.argtypes = [ctypes.c_int] * 5
 _lib.fa_selftest_watchdog.restype = ctypes.c_int
 _lib.fa_selftest_watchdog.argtypes = [ctypes.c_int, ctypes.c_void_p]
 _lib.fa_get_device_status.restype = ctypes.c_int
@@ -127,6 +135,62 @@ def attention_forward_kvcache(q, k, v, *, causal: bool = False, scale: float | N
                         torch.cuda.current_stream(q.device))
     if rc != FA_OK:
         raise FAError(rc, "fa_fwd_kvcache")
+    return out, lse
+
+
+def fa_fwd_splitkv(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, num_splits, workspace,
+                   workspace_bytes, stream=None) -> int:
+    """The C entry point for decode-shaped problems (keys cut into
+    ``num_splits`` ranges merged through the logsumexp); returns the status."""
+    return _lib.fa_fwd_splitkv(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), int(B), int(Hq),
+                               int(Hkv), int(Nq), int(Nk), int(d), float(scale), int(bool(causal)),
+                               int(num_splits), _addr(workspace), int(workspace_bytes), _stream(stream))
+
+
+def fa_splitkv_num_splits(B, Hq, Hkv, Nq, Nk, d) -> int:
+    """Split count for this shape on the current device (or a negative status)."""
+    return _lib.fa_splitkv_num_splits(int(B), int(Hq), int(Hkv), int(Nq), int(Nk), int(d))
+
+
+def fa_splitkv_workspace_bytes(B, Hq, Nq, d, num_splits) -> int:
+    """Workspace bytes fa_fwd_splitkv needs (0 for one split or bad arguments)."""
+    return int(_lib.fa_splitkv_workspace_bytes(int(B), int(Hq), int(Nq), int(d), int(num_splits)))
+
+
+def attention_forward_splitkv(q, k, v, *, causal: bool = False, scale: float | None = None,
+                              num_splits: int | None = None, workspace=None):
+    """``attention_forward_kvcache`` through fa_fwd_splitkv: O, lse for
+    q [B, Hq, Nq, d] against k/v [B, Hkv, Nk, d] (bf16 CUDA tensors).
+    ``num_splits`` defaults to the library's choice for the current device;
+    the workspace is allocated with torch unless one (a CUDA tensor of at least
+    the required bytes) is passed."""
+    import torch
+
+    if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+        raise TypeError("q, k, v must be bfloat16")
+    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    if q.dim() != 4 or k.dim() != 4 or k.shape != v.shape:
+        raise ValueError("q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d]")
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if k.shape[0] != B or k.shape[3] != d:
+        raise ValueError("k/v shape does not match q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if num_splits is None:
+        num_splits = fa_splitkv_num_splits(B, Hq, Hkv, Nq, Nk, d)
+        if num_splits < 0:
+            raise FAError(num_splits, "fa_splitkv_num_splits")
+    need = fa_splitkv_workspace_bytes(B, Hq, Nq, d, num_splits)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    out = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    rc = fa_fwd_splitkv(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, num_splits, workspace,
+                        wbytes, torch.cuda.current_stream(q.device))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_fwd_splitkv")
     return out, lse
 
 

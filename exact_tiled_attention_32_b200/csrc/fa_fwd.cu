@@ -73,6 +73,11 @@ struct alignas(64) Params {
     int B, Hq, Hkv, N;         // N: query rows per sequence (dense) or total tokens (packed)
     int Nk;                    // dense: keys per sequence (== N except for a query chunk)
     int q_off;                 // dense: position of query row 0 among the keys (Nk - N for a chunk)
+    int qmod;                  // dense: row r sits at position q_off + r % qmod (rows of several
+                               // query heads packed into one sequence); 0: position q_off + r
+    int splits;                // dense: key blocks of each tile are cut into this many splits
+    float* o_part;             // splits > 1: fp32 O / l of each split, [splits][B*Hq*N][d]
+    float* lse_part;           // splits > 1: logsumexp of each split, [splits][B*Hq*N]
     int group;                 // Hq / Hkv
     int group_units;           // dense: (batch, head) units scheduled together
     int causal, packed;
@@ -142,16 +147,31 @@ struct Item {
     int klen;      // keys of the sequence
     int qoff;      // position of query row 0 among the keys
     int tok0;      // packed: first token of the sequence
-    int n[2];      // key blocks each tile visits (0: tile beyond the sequence)
+    int split;     // split of the key blocks this item covers (0 without splits)
+    int j0;        // first key block of the item
+    int n[2];      // key blocks each tile visits from j0 on (0: none)
 };
 
+// Position of query row `row` among the keys.
+__device__ __forceinline__ int row_pos(int row, int qoff, int qmod) {
+    return qoff + (qmod ? row % qmod : row);
+}
+
 // Key blocks a 128-row query tile starting at row q0 visits: all of them, or
-// under the causal mask those up to the last valid row's position.
-__device__ __forceinline__ int tile_blocks(int q0, int len, int klen, int qoff, int causal) {
+// under the causal mask those up to the largest position of its valid rows.
+__device__ __forceinline__ int tile_blocks(int q0, int len, int klen, int qoff, int qmod, int causal) {
     if (q0 >= len) return 0;
     const int nkv = (klen + kBlockN - 1) / kBlockN;
     if (!causal) return nkv;
-    const int last_pos = min(q0 + kBlockM - 1, len - 1) + qoff;
+    const int last = min(q0 + kBlockM - 1, len - 1);
+    int last_pos;
+    if (!qmod) {
+        last_pos = qoff + last;
+    } else {
+        // rows q0 .. last cover positions q0 % qmod onwards, wrapping at qmod
+        const int first = q0 % qmod;
+        last_pos = qoff + ((last - q0 >= qmod - first) ? qmod - 1 : first + (last - q0));
+    }
     return min(nkv, last_pos / kBlockN + 1);
 }
 
@@ -167,6 +187,8 @@ __device__ __forceinline__ Item decode_item(int idx, const Params& p, const Misc
         // units (b, h) in groups of group_units whose K/V fit in L2 together;
         // inside a group, heaviest pair first
         const int npairs = (p.N + kRowsPerItem - 1) / kRowsPerItem;
+        it.split = idx % p.splits;              // the splits of one tile pair are adjacent items
+        idx /= p.splits;
         const int per = p.B * p.Hq;
         const int G = p.group_units;
         const int g = idx / (npairs * G);
@@ -197,10 +219,23 @@ __device__ __forceinline__ Item decode_item(int idx, const Params& p, const Misc
         it.len = tab.seq_off[it.seq + 1] - it.tok0;
         it.klen = it.len;
         it.qoff = 0;
+        it.split = 0;
     }
     it.q0 = pair * kRowsPerItem;
-    it.n[0] = tile_blocks(it.q0, it.len, it.klen, it.qoff, p.causal);
-    it.n[1] = tile_blocks(it.q0 + kBlockM, it.len, it.klen, it.qoff, p.causal);
+    const int qmod = PK ? 0 : p.qmod;
+    it.n[0] = tile_blocks(it.q0, it.len, it.klen, it.qoff, qmod, p.causal);
+    it.n[1] = tile_blocks(it.q0 + kBlockM, it.len, it.klen, it.qoff, qmod, p.causal);
+    it.j0 = 0;
+    if (!PK && p.splits > 1) {
+        // split s covers key blocks [s * nmax / S, (s + 1) * nmax / S) of the
+        // pair, nmax the larger block count of its two tiles
+        const int nmax = max(it.n[0], it.n[1]);
+        const int j0 = static_cast<int>(static_cast<long long>(it.split) * nmax / p.splits);
+        const int j1 = static_cast<int>(static_cast<long long>(it.split + 1) * nmax / p.splits);
+        it.j0 = j0;
+        it.n[0] = max(0, min(j1, it.n[0]) - j0);
+        it.n[1] = max(0, min(j1, it.n[1]) - j0);
+    }
     return it;
 }
 
@@ -261,6 +296,7 @@ __device__ void load_role(const Params& p, Misc& ms, const SeqTables& tab, uint3
         const int idx = item_of_round(r);
         if (idx >= total) break;
         const Item it = decode_item<PK>(idx, p, ms, tab);
+        if (max(it.n[0], it.n[1]) == 0) continue;      // a split with no key block
         // both query tiles of the item
         if (!(ok = wait_bar(smem_u32(&ms.bar_q_empty), (item_n & 1) ^ 1, p, ms, kSiteQEmpty))) break;
         const uint32_t qbar = smem_u32(&ms.bar_q_full);
@@ -286,10 +322,11 @@ __device__ void load_role(const Params& p, Misc& ms, const SeqTables& tab, uint3
                 const CUtensorMap* map = kind == 0 ? &p.tm_k : &p.tm_v;
                 for (int b = 0; b < C::kBoxes; ++b) {
                     const uint32_t dst = smem_kv + st * C::kTileBytes + b * kBoxBytes;
+                    const int key0 = (it.j0 + j) * kBlockN;
                     if constexpr (!PK)
-                        tma_load_4d(dst, map, bar, b * 64, j * kBlockN, kvh, it.seq, pol_kv);
+                        tma_load_4d(dst, map, bar, b * 64, key0, kvh, it.seq, pol_kv);
                     else
-                        tma_load_4d(dst, map, bar, b * 64, kvh, it.tok0 + j * kBlockN, 0, pol_kv);
+                        tma_load_4d(dst, map, bar, b * 64, kvh, it.tok0 + key0, 0, pol_kv);
                 }
                 ++kv_it;
                 if (++st == (uint32_t)C::kStages) {
@@ -349,6 +386,7 @@ __device__ void mma_role(const Params& p, Misc& ms, const SeqTables& tab, uint32
         const int idx = item_of_round(r);
         if (idx >= total) break;
         const Item it = decode_item<PK>(idx, p, ms, tab);
+        if (max(it.n[0], it.n[1]) == 0) continue;      // a split with no key block
         if (!(ok = wait_bar(smem_u32(&ms.bar_q_full), item_n & 1, p, ms, kSiteQFull))) break;
         tc_fence_after();
         ++item_n;
@@ -456,10 +494,16 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
         if (idx >= total) break;
         const Item it = decode_item<PK>(idx, p, ms, tab);
         const int n = t ? it.n[1] : it.n[0];
-        if (n == 0) continue;
         const int row = it.q0 + t * kBlockM + r;
+        if (n == 0) {
+            // a split that holds no key block of this tile contributes nothing
+            if (!PK && p.splits > 1 && row < it.len)
+                p.lse_part[static_cast<size_t>(it.split) * p.B * p.Hq * p.N +
+                           (static_cast<size_t>(it.seq) * p.Hq + it.h) * p.N + row] = -INFINITY;
+            continue;
+        }
         // keys [0, limit) are allowed for this row (causal: up to its own position)
-        const int limit = p.causal ? min(row + it.qoff + 1, it.klen) : it.klen;
+        const int limit = p.causal ? min(row_pos(row, it.qoff, PK ? 0 : p.qmod) + 1, it.klen) : it.klen;
         float m_used = -INFINITY;    // max the exponentials are taken against (log2 units)
         float l = 0.f;               // running sum of exp2(x - m_used)
         for (int j = 0; j < n; ++j) {
@@ -472,8 +516,8 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
             uint32_t s[128];
             tmem_ld128_sync(taddr_s, s);
             if (lane == 0 && wq == 0) FA_TRACE_EV(t, sc - 1, 2);
-            if (j * kBlockN + kBlockN > limit) {      // diagonal or tail block
-                const int lim = limit - j * kBlockN;
+            if ((it.j0 + j) * kBlockN + kBlockN > limit) {      // diagonal or tail block
+                const int lim = limit - (it.j0 + j) * kBlockN;
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
                     if (c >= lim) s[c] = __float_as_uint(-INFINITY);
@@ -579,6 +623,32 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
         float* lrow;
         if constexpr (!PK) {
             const size_t rid = (static_cast<size_t>(it.seq) * p.Hq + it.h) * p.N + row;
+            if (p.splits > 1) {
+                // this split's O / l in fp32 and its logsumexp; a combine pass
+                // merges the splits
+                const size_t prid = static_cast<size_t>(it.split) * p.B * p.Hq * p.N + rid;
+                float* prow = p.o_part + prid * D;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32_sync(taddr_o + c * 32, o);
+                    if (valid) {
+                        float4* dst = reinterpret_cast<float4*>(prow + c * 32);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
+                                                 __uint_as_float(o[4 * i + 2]) * inv,
+                                                 __uint_as_float(o[4 * i + 3]) * inv);
+                    }
+                }
+                if (valid) {
+                    float lg;
+                    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg) : "f"(l));
+                    p.lse_part[prid] = (l > 0.f) ? (m_used + lg) * 0.69314718055994531f : -INFINITY;
+                }
+                tc_fence_before();
+                continue;
+            }
             orow = static_cast<uint16_t*>(p.o) + rid * D;
             lrow = p.lse + rid;
         } else {
@@ -706,7 +776,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     if constexpr (PK) {
         total = ms.total_items;
     } else {
-        total = ((p.N + kRowsPerItem - 1) / kRowsPerItem) * p.B * p.Hq;
+        total = ((p.N + kRowsPerItem - 1) / kRowsPerItem) * p.B * p.Hq * p.splits;
     }
 
     if (warp < kNumSoftmaxWarps) {
@@ -729,6 +799,58 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+}
+
+// Merge of the key splits (Theorem 2 applied to whole splits): with split s
+// holding O_s = (its P V) / l_s and lse_s = m_s + ln l_s, the row's result is
+// lse = ln sum_s exp(lse_s) and O = sum_s exp(lse_s - lse) O_s.  One warp per
+// row; each lane owns D / 32 consecutive columns.  Splits with no allowed key
+// (lse_s = -inf) carry weight 0 and their O_s is not read; a row with no
+// allowed key at all gets O = 0 and lse = -inf.
+template <int D>
+__global__ void __launch_bounds__(256) fa_combine_kernel(const float* __restrict__ o_part,
+                                                         const float* __restrict__ lse_part, uint16_t* o, float* lse,
+                                                         long long rows, int splits) {
+    constexpr int kCols = D / 32;
+    const long long row = static_cast<long long>(blockIdx.x) * 8 + threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    if (row >= rows) return;
+    float mx = -INFINITY;
+    for (int s = 0; s < splits; ++s) mx = fmaxf(mx, lse_part[s * rows + row]);
+    float acc[kCols];
+#pragma unroll
+    for (int i = 0; i < kCols; ++i) acc[i] = 0.f;
+    float wsum = 0.f;
+    if (mx != -INFINITY) {
+        for (int s = 0; s < splits; ++s) {
+            const float ls = lse_part[s * rows + row];
+            if (ls == -INFINITY) continue;
+            const float w = __expf(ls - mx);
+            wsum += w;
+            const float* src = o_part + (static_cast<size_t>(s) * rows + row) * D + lane * kCols;
+            if constexpr (kCols == 4) {
+                const float4 v = *reinterpret_cast<const float4*>(src);
+                acc[0] += w * v.x;
+                acc[1] += w * v.y;
+                acc[2] += w * v.z;
+                acc[3] += w * v.w;
+            } else {
+                const float2 v = *reinterpret_cast<const float2*>(src);
+                acc[0] += w * v.x;
+                acc[1] += w * v.y;
+            }
+        }
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    uint32_t pk[kCols / 2];
+#pragma unroll
+    for (int i = 0; i < kCols / 2; ++i) pk[i] = pack_bf16x2(acc[2 * i] * inv, acc[2 * i + 1] * inv);
+    uint16_t* dst = o + row * D + lane * kCols;
+    if constexpr (kCols == 4)
+        *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
+    else
+        *reinterpret_cast<uint32_t*>(dst) = pk[0];
+    if (lane == 0) lse[row] = wsum > 0.f ? mx + __logf(wsum) : -INFINITY;
 }
 
 // Watchdog self-test: one thread waits, through the same bounded wait the
@@ -847,9 +969,11 @@ static bool aligned(const void* ptr, uintptr_t a) { return (reinterpret_cast<uin
 // Fills the launch parameters and launches the kernel variant for (d, packed)
 // on `stream`.  Nk / q_off describe a dense query chunk (Nk keys per sequence,
 // query row 0 at key position q_off); a plain forward has Nk = N, q_off = 0.
+// qmod, splits, o_part, lse_part: see Params (a plain forward has 0, 1, NULL, NULL).
 static int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                       int N, int Nk, int q_off, int d, float scale, int causal, const int32_t* cu_seqlens,
-                      cudaStream_t s, int* status, int num_sms) {
+                      cudaStream_t s, int* status, int num_sms, int qmod = 0, int splits = 1,
+                      float* o_part = nullptr, float* lse_part = nullptr) {
     const bool packed = cu_seqlens != nullptr;
     Params P;
     std::memset(&P, 0, sizeof(P));
@@ -877,12 +1001,16 @@ static int launch_fwd(const void* q, const void* k, const void* v, void* o, floa
     P.packed = packed ? 1 : 0;
     P.scale_log2 = scale * 1.4426950408889634f;
     P.timeout_ns = 2000000000ull;
+    P.qmod = qmod;
+    P.splits = splits;
+    P.o_part = o_part;
+    P.lse_part = lse_part;
 #ifdef FA_TRACE
     P.trace = g_trace;
 #endif
     long long items;
     if (!packed) {
-        items = (long long)((N + kRowsPerItem - 1) / kRowsPerItem) * B * Hq;
+        items = (long long)((N + kRowsPerItem - 1) / kRowsPerItem) * B * Hq * splits;
     } else {
         items = (long long)num_sms;    // exact count is known only on the device
     }
@@ -954,6 +1082,120 @@ extern "C" int fa_fwd_kvcache(const void* q, const void* k, const void* v, void*
     // the chunk's rows are the last Nq positions of the key sequence
     return launch_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, causal ? Nk - Nq : 0, d, scale, causal, nullptr,
                       static_cast<cudaStream_t>(stream), ds->status, ds->num_sms);
+}
+
+// ------------------------------------------------------------ split keys
+// Decode-shaped problems (a few query rows against a long cache) have too few
+// 128-row tiles to occupy the GPU.  Two changes fix that.  The query rows of
+// the Hq / Hkv heads that share a key/value head are packed into one tile:
+// in the [B, Hq, Nq, d] layout they are adjacent, so the problem is read as
+// Hkv heads of Hq / Hkv * Nq rows, row r at position Nk - Nq + r % Nq.  And
+// the key blocks are cut into splits that run as separate work items, each
+// writing its O / l and logsumexp in fp32 to the workspace, merged by
+// fa_combine_kernel.
+namespace fa_sm100 {
+
+constexpr int kMaxSplits = 256;
+
+struct SplitShape {
+    int Hq, Hkv, N, qmod;      // the problem as the kernel sees it
+};
+
+static SplitShape split_shape(int Hq, int Hkv, int Nq) {
+    const int g = Hq / Hkv;
+    if (g > 1 && Nq < kBlockM) return {Hkv, Hkv, g * Nq, Nq};
+    return {Hq, Hkv, Nq, 0};
+}
+
+static size_t split_workspace_bytes(int B, int Hq, int Nq, int d, int splits) {
+    if (splits <= 1) return 0;
+    const size_t rows = static_cast<size_t>(B) * Hq * Nq;
+    return static_cast<size_t>(splits) * rows * (d + 1) * sizeof(float);
+}
+
+// Split count: the one minimising (waves of work items) x (key blocks per
+// item + 2 blocks of per-item overhead), smallest on ties.
+static int choose_splits(int B, int Hq, int Hkv, int Nq, int Nk, int num_sms) {
+    const SplitShape sh = split_shape(Hq, Hkv, Nq);
+    const long long units = (long long)B * sh.Hq * ((sh.N + kRowsPerItem - 1) / kRowsPerItem);
+    const int nblocks = (Nk + kBlockN - 1) / kBlockN;
+    const int smax = std::max(1, std::min(nblocks, kMaxSplits));
+    int best = 1;
+    double best_cost = 1e300;
+    for (int sp = 1; sp <= smax; ++sp) {
+        const long long waves = (units * sp + num_sms - 1) / num_sms;
+        const double cost = (double)waves * ((nblocks + sp - 1) / sp + 2);
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = sp;
+        }
+    }
+    return best;
+}
+
+}  // namespace fa_sm100
+
+extern "C" int fa_splitkv_num_splits(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
+    if (B < 1 || Hq < 1 || Nq < 1 || Nk < 1) return FA_ERR_SHAPE;
+    if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+    if (Hkv < 1 || Hq % Hkv != 0) return FA_ERR_GQA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_LAUNCH;
+    DeviceState* ds = nullptr;
+    const int st = init_device(dev, &ds);
+    if (st != FA_OK) return st;
+    return choose_splits(B, Hq, Hkv, Nq, Nk, ds->num_sms);
+}
+
+extern "C" size_t fa_splitkv_workspace_bytes(int B, int Hq, int Nq, int d, int num_splits) {
+    if (B < 0 || Hq < 1 || Nq < 0 || (d != 64 && d != 128) || num_splits < 1 || num_splits > kMaxSplits) return 0;
+    return split_workspace_bytes(B, Hq, Nq, d, num_splits);
+}
+
+extern "C" int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                              int Hkv, int Nq, int Nk, int d, float scale, int causal, int num_splits,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+    if (B < 0 || Nq < 0 || Nk < 0 || Hq < 1) return FA_ERR_SHAPE;
+    if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+    if (Hkv < 1 || Hq % Hkv != 0) return FA_ERR_GQA;
+    if (num_splits < 1 || num_splits > kMaxSplits) return FA_ERR_SHAPE;
+    if (B == 0 || Nq == 0) return FA_OK;
+    if (Nk == 0 || (causal && Nk < Nq)) return FA_ERR_SHAPE;
+    if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+        return FA_ERR_ALIGN;
+    if ((long long)B * Hq * Nq > (1ll << 30) || (long long)B * Hkv * Nk > (1ll << 31)) return FA_ERR_SHAPE;
+    if ((long long)B * Hq * Nq * num_splits > (1ll << 31)) return FA_ERR_SHAPE;
+    const size_t need = split_workspace_bytes(B, Hq, Nq, d, num_splits);
+    if (need > 0) {
+        if (!workspace) return FA_ERR_NULL;
+        if (!aligned(workspace, 16)) return FA_ERR_ALIGN;
+        if (workspace_bytes < need) return FA_ERR_SHAPE;
+    }
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_LAUNCH;
+    DeviceState* ds = nullptr;
+    const int st = init_device(dev, &ds);
+    if (st != FA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const SplitShape sh = split_shape(Hq, Hkv, Nq);
+    const int q_off = causal ? Nk - Nq : 0;
+    if (num_splits == 1)
+        return launch_fwd(q, k, v, o, lse, B, sh.Hq, sh.Hkv, sh.N, Nk, q_off, d, scale, causal, nullptr, s,
+                          ds->status, ds->num_sms, sh.qmod);
+    const long long rows = (long long)B * Hq * Nq;
+    float* o_part = static_cast<float*>(workspace);
+    float* lse_part = o_part + static_cast<size_t>(num_splits) * rows * d;
+    const int rc = launch_fwd(q, k, v, o, lse, B, sh.Hq, sh.Hkv, sh.N, Nk, q_off, d, scale, causal, nullptr, s,
+                              ds->status, ds->num_sms, sh.qmod, num_splits, o_part, lse_part);
+    if (rc != FA_OK) return rc;
+    const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
+    if (d == 64)
+        fa_combine_kernel<64><<<grid, 256, 0, s>>>(o_part, lse_part, static_cast<uint16_t*>(o), lse, rows, num_splits);
+    else
+        fa_combine_kernel<128><<<grid, 256, 0, s>>>(o_part, lse_part, static_cast<uint16_t*>(o), lse, rows, num_splits);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
 extern "C" int fa_selftest_watchdog(int timeout_ms, void* stream) {

@@ -31,6 +31,8 @@ one stream; for the packed batch the sequence lengths are drawn first):
 * c5: 16 sequences, lengths uniform in [512, 8192], H=16, d=128, causal
 * p3: a query chunk of 2048 rows (the last positions) against 16384 keys,
   B=1, H=32, d=128, causal -- the chunked-prefill shape
+* dec: one decode step -- 1 query row per (batch, head) against a 32768-key
+  cache, B=8, Hq=32, Hkv=8, d=128 (with one row, causal allows every key)
 """
 from __future__ import annotations
 
@@ -179,6 +181,18 @@ class Workload:
         f = sum(4.0 * L * L * self.d for L in self.lengths) * self.Hq
         return f / 2 if self.causal else f
 
+    @property
+    def decode(self) -> bool:
+        """A query chunk of fewer than 128 rows: the split-key path."""
+        return self.chunk and self.N < 128
+
+    def hbm_bytes(self) -> float:
+        """Bytes the forward must move at least: Q, K, V read once, O (bf16)
+        and lse (fp32) written once."""
+        nq = self.B * self.Hq * self.N if not self.packed else self.Hq * self.N
+        nk = self.B * self.Hkv * (self.Nk if self.chunk else self.N) if not self.packed else self.Hkv * self.N
+        return 2.0 * self.d * (2 * nq + 2 * nk) + 4.0 * nq
+
     def q_shape(self):
         return (self.N, self.Hq, self.d) if self.packed else (self.B, self.Hq, self.N, self.d)
 
@@ -218,7 +232,7 @@ def packed_from_lengths(name, lens, H, d, causal, seed, Hkv=None) -> Workload:
 
 
 def config(name: str) -> Workload:
-    """The named workloads c1, c2nc, c2c, c3, c4, c5 (inputs not yet drawn)."""
+    """The named workloads c1, c2nc, c2c, c3, c4, c5, p3, dec (inputs not yet drawn)."""
     if name == "c1":
         return Workload("c1", 1, 1, 1, 256, 64, False, 1001)
     if name == "c2nc":
@@ -235,7 +249,11 @@ def config(name: str) -> Workload:
         # a 2048-row prefill chunk at the end of a 16384-token sequence,
         # c3's heads and head size
         return Workload("p3", 1, 32, 32, 2048, 128, True, 1006, Nk=16384)
+    if name == "dec":
+        # one new token per sequence of a batch of 8 against a 32768-token
+        # cache, c4's grouped heads
+        return Workload("dec", 8, 32, 8, 1, 128, True, 1007, Nk=32768)
     raise KeyError(name)
 
 
-CONFIGS = ("c1", "c2nc", "c2c", "c3", "c4", "c5", "p3")
+CONFIGS = ("c1", "c2nc", "c2c", "c3", "c4", "c5", "p3", "dec")

@@ -16,6 +16,7 @@
 #ifndef FA_B200_H
 #define FA_B200_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -102,6 +103,52 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 int fa_fwd_kvcache(const void* q, const void* k, const void* v, void* o, float* lse,
                    int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
                    void* stream);
+
+/*
+ * fa_fwd_splitkv -- fa_fwd_kvcache for decode-shaped problems (a few query
+ * rows against a long KV cache), asynchronous on `stream`.  Same arguments,
+ * layouts, masks and result as fa_fwd_kvcache, plus:
+ *
+ *   num_splits       1 .. 256: the key blocks of every query tile are cut
+ *                    into this many contiguous ranges ("splits") that run as
+ *                    separate work items on different SMs.
+ *   workspace        device memory, 16-byte aligned, of at least
+ *                    fa_splitkv_workspace_bytes(B, Hq, Nq, d, num_splits)
+ *                    bytes (0 when num_splits == 1; it may then be NULL).
+ *                    Each split writes its normalised output and logsumexp
+ *                    there in fp32; a second kernel on the same stream merges
+ *                    them with the rescaling of "Online Softmax" (Theorem 2):
+ *                    lse = ln sum_s exp(lse_s), O = sum_s exp(lse_s - lse) O_s.
+ *                    The workspace must not be used by anything else until
+ *                    that kernel is done; nothing in it needs initialising.
+ *
+ * When Hq > Hkv and Nq < 128, the query rows of the Hq / Hkv heads that
+ * share a key/value head are processed in one 128-row tile, so each K/V
+ * block is read once for all of them.  The page gives no decode algorithm;
+ * splitting the keys is the same block-wise combination the method applies
+ * within one sequence (the split results are combined exactly, up to fp32
+ * rounding).  Errors as fa_fwd_kvcache; FA_ERR_SHAPE also for num_splits out
+ * of range or a workspace smaller than required, FA_ERR_NULL for a missing
+ * workspace, FA_ERR_ALIGN for a misaligned one.
+ */
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,
+                   int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                   int num_splits, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fa_splitkv_num_splits -- the split count fa_fwd_splitkv runs best with on
+ * the current device for this shape (from the number of work items and the
+ * device's SM count), >= 1; or a negative fa_status for invalid sizes or no
+ * usable device.
+ */
+int fa_splitkv_num_splits(int B, int Hq, int Hkv, int Nq, int Nk, int d);
+
+/*
+ * fa_splitkv_workspace_bytes -- workspace fa_fwd_splitkv needs:
+ * num_splits * B * Hq * Nq * (d + 1) * 4 bytes, 0 when num_splits == 1 and 0
+ * for invalid arguments.  Needs no device.
+ */
+size_t fa_splitkv_workspace_bytes(int B, int Hq, int Nq, int d, int num_splits);
 
 /*
  * fa_get_device_status -- reads and clears the status word of the current

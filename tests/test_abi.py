@@ -67,6 +67,43 @@ def test_argument_errors_found_on_the_host():
     assert call(N=0, ptrs=(0, 0, 0, 0, 0)) == fa.FA_OK
 
 
+def test_splitkv_argument_errors_found_on_the_host():
+    from exact_tiled_attention_32_b200 import binding as fa
+    p = 1 << 20
+    ok = dict(B=2, Hq=8, Hkv=2, Nq=1, Nk=4096, d=128, scale=0.1, causal=1, S=4)
+
+    def call(ptrs=(p, p, p, p, p), ws=p, wbytes=1 << 30, **kw):
+        a = dict(ok)
+        a.update(kw)
+        return fa.fa_fwd_splitkv(*ptrs, a["B"], a["Hq"], a["Hkv"], a["Nq"], a["Nk"], a["d"], a["scale"],
+                                 a["causal"], a["S"], ws, wbytes, None)
+
+    assert call(d=96) == fa.FA_ERR_HEADDIM
+    assert call(Hkv=3) == fa.FA_ERR_GQA
+    assert call(S=0) == fa.FA_ERR_SHAPE
+    assert call(S=257) == fa.FA_ERR_SHAPE
+    assert call(Nk=0) == fa.FA_ERR_SHAPE
+    assert call(Nq=8, Nk=4) == fa.FA_ERR_SHAPE          # causal chunk longer than the keys
+    assert call(ws=0) == fa.FA_ERR_NULL
+    assert call(ws=p + 4) == fa.FA_ERR_ALIGN
+    need = fa.fa_splitkv_workspace_bytes(2, 8, 1, 128, 4)
+    assert call(wbytes=need - 1) == fa.FA_ERR_SHAPE
+    assert call(ptrs=(p, p, 0, p, p)) == fa.FA_ERR_NULL
+    assert call(B=0, ptrs=(0, 0, 0, 0, 0), ws=0, wbytes=0) == fa.FA_OK
+    # one split needs no workspace
+    assert fa.fa_splitkv_workspace_bytes(2, 8, 1, 128, 1) == 0
+
+
+def test_splitkv_workspace_bytes():
+    from exact_tiled_attention_32_b200 import binding as fa
+    # num_splits x rows x (d + 1) fp32 values
+    assert fa.fa_splitkv_workspace_bytes(2, 8, 3, 128, 4) == 4 * 2 * 8 * 3 * 129 * 4
+    assert fa.fa_splitkv_workspace_bytes(1, 32, 1, 64, 16) == 16 * 32 * 65 * 4
+    assert fa.fa_splitkv_workspace_bytes(1, 1, 1, 96, 2) == 0      # bad head dim
+    assert fa.fa_splitkv_workspace_bytes(1, 1, 1, 64, 0) == 0      # bad split count
+    assert fa.fa_splitkv_workspace_bytes(1, 1, 1, 64, 257) == 0
+
+
 def test_no_device_means_launch_error():
     import torch
     if torch.cuda.is_available():
@@ -75,6 +112,7 @@ def test_no_device_means_launch_error():
     p = 1 << 20
     assert fa.fa_fwd(p, p, p, p, p, 1, 1, 1, 128, 64, 0.1, 0) == fa.FA_ERR_LAUNCH
     assert fa.fa_get_device_status() == fa.FA_ERR_LAUNCH
+    assert fa.fa_splitkv_num_splits(1, 32, 8, 1, 32768, 128) == fa.FA_ERR_LAUNCH
 
 
 def test_binding_refuses_to_run_without_the_library(tmp_path, monkeypatch):
