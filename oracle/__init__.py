@@ -21,6 +21,9 @@ Every function cites the passage of the pages it follows in ``oracle.c``:
 * ``attention_kv``     -- a chunk of queries against a longer key sequence,
                           the chunk's rows being its last positions (xspy.com,
                           section 1, chunked prefill).
+* ``attention_bwd``    -- dQ, dK, dV of standard attention: the derivative of
+                          the forward's definition (the pages name only the
+                          recomputation of the backward pass).
 
 Pins (in ``tests/test_oracle.py``): the worked examples of both pages, row sums
 of one, torch's fp64 scaled-dot-product attention as an independent library
@@ -84,6 +87,11 @@ def bind(path: str):
     lib.oracle_attention_kv.argtypes = [
         u16p, u16p, u16p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
         ctypes.c_int, ctypes.c_double, ctypes.c_int, i64p, ctypes.c_int64, dp, dp, ctypes.c_int,
+    ]
+    lib.oracle_attention_bwd.restype = ctypes.c_int
+    lib.oracle_attention_bwd.argtypes = [
+        u16p, u16p, u16p, u16p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_double, ctypes.c_int, i64p, ctypes.c_int64, dp, dp, dp, ctypes.c_int,
     ]
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_num_threads.argtypes = []
@@ -201,6 +209,32 @@ def attention_kv(q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal, rows=None, nthre
     if rc != 0:
         raise ValueError("oracle_attention_kv: bad arguments or row id out of range")
     return o, lse
+
+
+def attention_bwd(q, k, v, dout, B, Hq, Hkv, N, d, scale, causal, units=None, nthreads=0,
+                  lib=None) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """fp64 gradients (dq, dk, dv) of dense attention for the upstream
+    gradient ``dout``.  q, dout [B,Hq,N,d], k/v [B,Hkv,N,d] as bf16 bits.
+    ``units``: (batch, kv head) units b*Hkv+hk to compute, or None for all.
+    With units=None: dq [B,Hq,N,d], dk/dv [B,Hkv,N,d]; otherwise dq
+    [nunits, Hq/Hkv, N, d] and dk/dv [nunits, N, d]."""
+    q, k, v, dout = _as_bits(q), _as_bits(k), _as_bits(v), _as_bits(dout)
+    g = Hq // Hkv
+    u = None if units is None else np.ascontiguousarray(units, dtype=np.int64)
+    nunits = B * Hkv if u is None else u.size
+    dq = np.zeros((nunits, g, N, d), dtype=np.float64)
+    dk = np.zeros((nunits, N, d), dtype=np.float64)
+    dv = np.zeros((nunits, N, d), dtype=np.float64)
+    rc = _load(lib).oracle_attention_bwd(
+        _ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16), _ptr(v, ctypes.c_uint16),
+        _ptr(dout, ctypes.c_uint16), B, Hq, Hkv, N, d, float(scale), int(bool(causal)),
+        _ptr(u, ctypes.c_int64), nunits, _ptr(dq, ctypes.c_double), _ptr(dk, ctypes.c_double),
+        _ptr(dv, ctypes.c_double), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_attention_bwd: bad arguments or unit out of range")
+    if u is None:
+        return dq.reshape(B, Hq, N, d), dk.reshape(B, Hkv, N, d), dv.reshape(B, Hkv, N, d)
+    return dq, dk, dv
 
 
 def num_threads() -> int:

@@ -412,6 +412,158 @@ int oracle_attention_kv(const uint16_t* q, const uint16_t* k, const uint16_t* v,
     return bad ? -1 : 0;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Gradients of standard attention (dense batches).                         */
+/*                                                                          */
+/* The pages say only that the backward pass recomputes the score matrix    */
+/* from Q, K, V instead of storing it (14cs17 page, "Common Pitfalls",      */
+/* Pitfall 3; fromzero2ai page, "Core Mechanisms of FlashAttention", item   */
+/* 3).  What it computes is the derivative of the forward's definition:     */
+/* with P = softmax(S) row-wise, S = scale Q K^T (masked entries -inf),     */
+/* O = P V and an upstream gradient dO,                                     */
+/*     dV = P^T dO,      dP = dO V^T,                                       */
+/*     dS_ij = P_ij (dP_ij - D_i),  D_i = sum_j P_ij dP_ij                  */
+/*             (the softmax Jacobian applied to row i of dP),               */
+/*     dQ = scale dS K,  dK = scale dS^T Q.                                  */
+/* Grouped-query attention: the Hq / Hkv query heads that read one          */
+/* key/value head all add into that head's dK and dV.                        */
+/*                                                                          */
+/* Pass 1 walks the query rows: it materialises each score row, its         */
+/* softmax, dP and dS in fp64 and forms dQ, keeping lse_i = m + log l and   */
+/* D_i.  Pass 2 walks the keys: P_ij = exp(S_ij - lse_i) is the same        */
+/* softmax entry, recomputed, and dK_j, dV_j sum over the query rows.       */
+/*                                                                          */
+/* units: list of nunits (batch, kv head) units b*Hkv + hk, or NULL for all */
+/* (nunits is then B*Hkv).  Layouts: q, dout [B,Hq,N,d], k, v [B,Hkv,N,d].  */
+/* Outputs per unit, in unit order: dq [group][N][d], dk and dv [N][d]      */
+/* (with units == NULL that is dq [B,Hq,N,d], dk, dv [B,Hkv,N,d]).          */
+/* A query row with no allowed key contributes nothing.  Returns 0, or -1   */
+/* on bad arguments.                                                        */
+/* ------------------------------------------------------------------------ */
+int oracle_attention_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                         const uint16_t* dout, int B, int Hq, int Hkv, int N, int d,
+                         double scale, int causal, const int64_t* units, int64_t nunits,
+                         double* dq, double* dk, double* dv, int nthreads) {
+    if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || N < 0 || B < 0) return -1;
+    const int group = Hq / Hkv;
+    if (!units) nunits = (int64_t)B * Hkv;
+    for (int64_t u = 0; u < nunits; ++u) {
+        const int64_t unit = units ? units[u] : u;
+        if (unit < 0 || unit >= (int64_t)B * Hkv) return -1;
+    }
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+    const int64_t nd = (int64_t)N * d;
+    double* Qw = (double*)malloc(sizeof(double) * (size_t)(group * nd + 1));
+    double* Ow = (double*)malloc(sizeof(double) * (size_t)(group * nd + 1));   /* dO, widened */
+    double* Kw = (double*)malloc(sizeof(double) * (size_t)(nd + 1));
+    double* Vw = (double*)malloc(sizeof(double) * (size_t)(nd + 1));
+    double* lse = (double*)malloc(sizeof(double) * (size_t)(group * (int64_t)N + 1));
+    double* Dr = (double*)malloc(sizeof(double) * (size_t)(group * (int64_t)N + 1));
+    if (!Qw || !Ow || !Kw || !Vw || !lse || !Dr) {
+        free(Qw); free(Ow); free(Kw); free(Vw); free(lse); free(Dr);
+        return -1;
+    }
+    for (int64_t u = 0; u < nunits; ++u) {
+        const int64_t unit = units ? units[u] : u;
+        const int64_t b = unit / Hkv;
+        const int hk = (int)(unit % Hkv);
+        const uint16_t* k0 = k + (b * Hkv + hk) * nd;
+        const uint16_t* v0 = v + (b * Hkv + hk) * nd;
+        for (int64_t e = 0; e < nd; ++e) {
+            Kw[e] = bf16_to_double(k0[e]);
+            Vw[e] = bf16_to_double(v0[e]);
+        }
+        for (int g = 0; g < group; ++g) {
+            const int h = hk * group + g;
+            const uint16_t* q0 = q + (b * Hq + h) * nd;
+            const uint16_t* o0 = dout + (b * Hq + h) * nd;
+            for (int64_t e = 0; e < nd; ++e) {
+                Qw[g * nd + e] = bf16_to_double(q0[e]);
+                Ow[g * nd + e] = bf16_to_double(o0[e]);
+            }
+        }
+        double* dqu = dq + u * group * nd;
+        double* dku = dk + u * nd;
+        double* dvu = dv + u * nd;
+        /* pass 1: query rows */
+#pragma omp parallel
+        {
+            double* p = (double*)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+            double* dp = (double*)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+#pragma omp for schedule(dynamic, 4)
+            for (int64_t gi = 0; gi < (int64_t)group * N; ++gi) {
+                const int64_t g = gi / N, i = gi % N;
+                const double* qi = Qw + g * nd + i * d;
+                const double* doi = Ow + g * nd + i * d;
+                const int64_t nkeys = causal ? i + 1 : N;     /* keys j < nkeys allowed */
+                double m = -INFINITY;
+                for (int64_t j = 0; j < nkeys; ++j) {
+                    double dot = 0.0;
+                    for (int c = 0; c < d; ++c) dot += qi[c] * Kw[j * d + c];
+                    p[j] = scale * dot;
+                    if (p[j] > m) m = p[j];
+                }
+                double* dqi = dqu + g * nd + i * d;
+                for (int c = 0; c < d; ++c) dqi[c] = 0.0;
+                if (m == -INFINITY) { lse[gi] = -INFINITY; Dr[gi] = 0.0; continue; }
+                double l = 0.0;
+                for (int64_t j = 0; j < nkeys; ++j) {
+                    p[j] = exp(p[j] - m);
+                    l += p[j];
+                }
+                double D = 0.0;
+                for (int64_t j = 0; j < nkeys; ++j) {
+                    p[j] /= l;
+                    double dot = 0.0;
+                    for (int c = 0; c < d; ++c) dot += doi[c] * Vw[j * d + c];
+                    dp[j] = dot;
+                    D += p[j] * dp[j];
+                }
+                for (int64_t j = 0; j < nkeys; ++j) {
+                    const double ds = p[j] * (dp[j] - D);
+                    for (int c = 0; c < d; ++c) dqi[c] += scale * ds * Kw[j * d + c];
+                }
+                lse[gi] = m + log(l);
+                Dr[gi] = D;
+            }
+            free(p);
+            free(dp);
+        }
+        /* pass 2: keys */
+#pragma omp parallel for schedule(dynamic, 4)
+        for (int64_t j = 0; j < N; ++j) {
+            double* dkj = dku + j * d;
+            double* dvj = dvu + j * d;
+            for (int c = 0; c < d; ++c) { dkj[c] = 0.0; dvj[c] = 0.0; }
+            const double* kj = Kw + j * d;
+            const double* vj = Vw + j * d;
+            for (int g = 0; g < group; ++g) {
+                for (int64_t i = causal ? j : 0; i < N; ++i) {
+                    const int64_t gi = (int64_t)g * N + i;
+                    if (lse[gi] == -INFINITY) continue;
+                    const double* qi = Qw + g * nd + i * d;
+                    const double* doi = Ow + g * nd + i * d;
+                    double s = 0.0, dp = 0.0;
+                    for (int c = 0; c < d; ++c) {
+                        s += qi[c] * kj[c];
+                        dp += doi[c] * vj[c];
+                    }
+                    const double pij = exp(scale * s - lse[gi]);
+                    const double ds = pij * (dp - Dr[gi]);
+                    for (int c = 0; c < d; ++c) {
+                        dvj[c] += pij * doi[c];
+                        dkj[c] += scale * ds * qi[c];
+                    }
+                }
+            }
+        }
+    }
+    free(Qw); free(Ow); free(Kw); free(Vw); free(lse); free(Dr);
+    return 0;
+}
+
 /* Number of worker threads OpenMP will use (reported by the CPU baseline). */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

@@ -386,6 +386,13 @@ MUTATIONS = {
     "online_no_rescale": ("double carry = (m_run == -INFINITY) ? 0.0 : exp(m_run - m_new);",
                           "double carry = (m_run == -INFINITY) ? 0.0 : 1.0;"),
     "chunk_top_left_mask": ("const int64_t pos = (int64_t)Nk - Nq + i;", "const int64_t pos = i;"),
+    "bwd_dq_without_scale": ("dqi[c] += scale * ds * Kw[j * d + c];", "dqi[c] += ds * Kw[j * d + c];"),
+    "bwd_D_without_p": ("D += p[j] * dp[j];", "D += dp[j];"),
+    "bwd_dk_from_dout": ("dkj[c] += scale * ds * qi[c];", "dkj[c] += scale * ds * doi[c];"),
+    "bwd_dv_from_q": ("dvj[c] += pij * doi[c];", "dvj[c] += pij * qi[c];"),
+    "bwd_flipped_ds": ("const double ds = pij * (dp - Dr[gi]);", "const double ds = pij * (Dr[gi] - dp);"),
+    "bwd_causal_keys_from_zero": ("for (int64_t i = causal ? j : 0; i < N; ++i) {",
+                                  "for (int64_t i = 0; i < N; ++i) {"),
 }
 
 
@@ -424,6 +431,19 @@ def _pin_suite(lib):
         return np.max(np.abs(o - o_t)) < 1e-12 and np.max(np.abs(lse - lse_t)) < 1e-12
 
     checks["torch_chunk"] = chunk_pin
+
+    def bwd_pin(B, Hq, Hkv, N, d, causal):
+        s = syn.Stream(31 + N)
+        q = s.normal_bf16((B, Hq, N, d))
+        k = s.normal_bf16((B, Hkv, N, d))
+        v = s.normal_bf16((B, Hkv, N, d))
+        do = s.normal_bf16((B, Hq, N, d))
+        got = oracle.attention_bwd(q, k, v, do, B, Hq, Hkv, N, d, 0.3, causal, lib=lib)
+        ref = _torch_bwd(q, k, v, do, B, Hq, Hkv, N, d, 0.3, causal)
+        return all(np.max(np.abs(a - b)) < 1e-12 for a, b in zip(got, ref))
+
+    checks["torch_bwd_causal_gqa"] = lambda: bwd_pin(1, 4, 2, 23, 8, True)
+    checks["torch_bwd_dense"] = lambda: bwd_pin(1, 2, 2, 11, 8, False)
     for name, fn in checks.items():
         try:
             ok = bool(fn())
@@ -539,3 +559,115 @@ def test_chunked_prefill_reproduces_the_whole_causal_forward():
         o, l = oracle.attention_kv(qc, kc, vc, B, H, H, b - a, b, d, 0.25, True)
         assert np.array_equal(o.reshape(B, H, b - a, d), o_full[:, :, a:b])
         assert np.array_equal(l.reshape(B, H, b - a), l_full[:, :, a:b])
+
+
+# --------------------------------------------------------------------------
+# gradients (the backward pass): dQ, dK, dV of the forward's definition
+# --------------------------------------------------------------------------
+
+def _torch_bwd(q, k, v, dout, B, Hq, Hkv, N, d, scale, causal):
+    """torch.autograd in fp64 through an explicit masked softmax (an
+    independent differentiation of the same definition)."""
+    qt, kt, vt = (torch.from_numpy(_f64(a)).requires_grad_(True) for a in (q, k, v))
+    g = Hq // Hkv
+    kr, vr = kt.repeat_interleave(g, dim=1), vt.repeat_interleave(g, dim=1)
+    s = scale * qt @ kr.transpose(-1, -2)
+    if causal:
+        mask = torch.ones(N, N, dtype=torch.bool).tril()
+        s = s.masked_fill(~mask, -math.inf)
+    o = torch.softmax(s, dim=-1) @ vr
+    o.backward(torch.from_numpy(_f64(dout)))
+    return qt.grad.numpy(), kt.grad.numpy(), vt.grad.numpy()
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,causal", [
+    (1, 4, 2, 37, 16, True),
+    (2, 2, 2, 20, 16, False),
+    (1, 3, 1, 9, 8, True),
+    (1, 2, 1, 1, 8, True),
+])
+def test_bwd_matches_torch_autograd(B, Hq, Hkv, N, d, causal):
+    s = syn.Stream(81 + N + d)
+    q = s.normal_bf16((B, Hq, N, d))
+    k = s.normal_bf16((B, Hkv, N, d))
+    v = s.normal_bf16((B, Hkv, N, d))
+    do = s.normal_bf16((B, Hq, N, d))
+    dq, dk, dv = oracle.attention_bwd(q, k, v, do, B, Hq, Hkv, N, d, 0.3, causal)
+    tq, tk, tv = _torch_bwd(q, k, v, do, B, Hq, Hkv, N, d, 0.3, causal)
+    assert np.max(np.abs(dq - tq)) < 1e-12
+    assert np.max(np.abs(dk - tk)) < 1e-12
+    assert np.max(np.abs(dv - tv)) < 1e-12
+
+
+def test_bwd_central_differences():
+    """Brute-force derivative of L = sum(dO * O), O from the oracle forward:
+    inputs are multiples of 1/8, so x +- 1/64 is exact in bf16; the central
+    difference error is O(h^2)."""
+    B, Hq, Hkv, N, d, scale = 1, 2, 1, 5, 4, 0.7
+    rng = np.random.default_rng(5)
+
+    def grid(shape):
+        return rng.integers(-8, 9, size=shape).astype(np.float64) / 8.0
+
+    qf, kf, vf = grid((B, Hq, N, d)), grid((B, Hkv, N, d)), grid((B, Hkv, N, d))
+    do = syn.fp64_to_bf16_bits(grid((B, Hq, N, d)))
+    dof = _f64(do).reshape(-1, d)
+    bits = syn.fp64_to_bf16_bits
+    h = 1.0 / 64
+    for causal in (False, True):
+        def loss(qx, kx, vx):
+            o, _ = oracle.attention(bits(qx), bits(kx), bits(vx), B, Hq, Hkv, N, d, scale, causal)
+            return float(np.sum(o * dof))
+
+        dq, dk, dv = oracle.attention_bwd(bits(qf), bits(kf), bits(vf), do, B, Hq, Hkv, N, d, scale, causal)
+        for which, base, grad in (("q", qf, dq), ("k", kf, dk), ("v", vf, dv)):
+            for idx in np.ndindex(base.shape):
+                xp, xm = base.copy(), base.copy()
+                xp[idx] += h
+                xm[idx] -= h
+                args_p = {"q": (xp, kf, vf), "k": (qf, xp, vf), "v": (qf, kf, xp)}[which]
+                args_m = {"q": (xm, kf, vf), "k": (qf, xm, vf), "v": (qf, kf, xm)}[which]
+                fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
+                assert abs(fd - grad[idx]) < 2e-3, (which, idx, fd, grad[idx], causal)
+
+
+def test_bwd_invariants():
+    """Every softmax row sums to one, so sum_j dS_ij = 0: the key gradients of
+    a (sequence, kv head) sum to zero, and the value gradients sum to the
+    upstream gradients of the query rows (of all heads in the group)."""
+    B, Hq, Hkv, N, d = 2, 4, 2, 50, 16
+    s = syn.Stream(91)
+    q = s.normal_bf16((B, Hq, N, d))
+    k = s.normal_bf16((B, Hkv, N, d))
+    v = s.normal_bf16((B, Hkv, N, d))
+    do = s.normal_bf16((B, Hq, N, d))
+    for causal in (False, True):
+        dq, dk, dv = oracle.attention_bwd(q, k, v, do, B, Hq, Hkv, N, d, 0.25, causal)
+        assert np.max(np.abs(dk.sum(axis=2))) < 1e-11
+        dos = _f64(do).reshape(B, Hkv, Hq // Hkv, N, d).sum(axis=(2, 3))
+        assert np.max(np.abs(dv.sum(axis=2) - dos)) < 1e-11
+
+
+def test_bwd_single_visible_key():
+    """Causal row 0 sees only key 0: P = [1], so dS = 0 there, and with N = 1
+    dQ = dK = 0 while dV = the group's summed dO."""
+    B, Hq, Hkv, N, d = 1, 3, 1, 1, 8
+    s = syn.Stream(92)
+    q, k, v = s.normal_bf16((B, Hq, N, d)), s.normal_bf16((B, Hkv, N, d)), s.normal_bf16((B, Hkv, N, d))
+    do = s.normal_bf16((B, Hq, N, d))
+    dq, dk, dv = oracle.attention_bwd(q, k, v, do, B, Hq, Hkv, N, d, 0.5, True)
+    assert np.all(dq == 0) and np.all(dk == 0)
+    assert np.max(np.abs(dv[0, 0] - _f64(do)[0].sum(axis=0))) < 1e-15
+
+
+def test_bwd_units_subset():
+    B, Hq, Hkv, N, d = 2, 4, 2, 30, 8
+    s = syn.Stream(93)
+    q = s.normal_bf16((B, Hq, N, d))
+    k = s.normal_bf16((B, Hkv, N, d))
+    v = s.normal_bf16((B, Hkv, N, d))
+    do = s.normal_bf16((B, Hq, N, d))
+    dq, dk, dv = oracle.attention_bwd(q, k, v, do, B, Hq, Hkv, N, d, 0.4, True)
+    sq, sk, sv = oracle.attention_bwd(q, k, v, do, B, Hq, Hkv, N, d, 0.4, True, units=[3, 0])
+    assert np.array_equal(sq[0], dq[1, 2:4]) and np.array_equal(sq[1], dq[0, 0:2])
+    assert np.array_equal(sk[0], dk[1, 1]) and np.array_equal(sv[1], dv[0, 0])
