@@ -29,7 +29,8 @@ FA_ERR_DEVICE_TIMEOUT = -8
 FA_ERR_SEQLENS = -9
 
 EXPORTED = ("fa_fwd", "fa_get_device_status", "fa_status_string", "fa_fwd_noalloc", "fa_fwd_kvcache",
-            "fa_selftest_watchdog", "fa_fwd_splitkv", "fa_splitkv_num_splits", "fa_splitkv_workspace_bytes")
+            "fa_selftest_watchdog", "fa_fwd_splitkv", "fa_splitkv_num_splits", "fa_splitkv_workspace_bytes",
+            "fa_bwd", "fa_bwd_workspace_bytes")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -59,6 +60,12 @@ _lib.fa_splitkv_num_splits.restype = ctypes.c_int
 _lib.fa_splitkv_num_splits.argtypes = [ctypes.c_int] * 6
 _lib.fa_splitkv_workspace_bytes.restype = ctypes.c_size_t
 _lib.fa_splitkv_workspace_bytes.argtypes = [ctypes.c_int] * 5
+_lib.fa_bwd.restype = ctypes.c_int
+_lib.fa_bwd.argtypes = [ctypes.c_void_p] * 9 + [ctypes.c_int] * 5 + [
+    ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+]
+_lib.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
+_lib.fa_bwd_workspace_bytes.argtypes = [ctypes.c_int] * 4
 _lib.fa_selftest_watchdog.restype = ctypes.c_int
 _lib.fa_selftest_watchdog.argtypes = [ctypes.c_int, ctypes.c_void_p]
 _lib.fa_get_device_status.restype = ctypes.c_int
@@ -192,6 +199,51 @@ def attention_forward_splitkv(q, k, v, *, causal: bool = False, scale: float | N
     if rc != FA_OK:
         raise FAError(rc, "fa_fwd_splitkv")
     return out, lse
+
+
+def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, workspace, workspace_bytes,
+           stream=None) -> int:
+    """The C entry point of the backward pass; returns the status."""
+    return _lib.fa_bwd(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), _addr(dout), _addr(dq), _addr(dk),
+                       _addr(dv), int(B), int(Hq), int(Hkv), int(N), int(d), float(scale), int(bool(causal)),
+                       _addr(workspace), int(workspace_bytes), _stream(stream))
+
+
+def fa_bwd_workspace_bytes(B, Hq, N, d) -> int:
+    """Workspace bytes fa_bwd needs (0 for bad arguments)."""
+    return int(_lib.fa_bwd_workspace_bytes(int(B), int(Hq), int(N), int(d)))
+
+
+def attention_backward(q, k, v, o, lse, dout, *, causal: bool = False, scale: float | None = None,
+                       workspace=None):
+    """dq, dk, dv for the dense forward O, lse = attention_forward(q, k, v)
+    and the upstream gradient ``dout`` (bf16 CUDA tensors, layouts of the
+    dense forward).  The workspace is allocated with torch unless given."""
+    import torch
+
+    for t in (q, k, v, o, dout):
+        if t.dtype != torch.bfloat16:
+            raise TypeError("q, k, v, o, dout must be bfloat16")
+    if lse.dtype != torch.float32:
+        raise TypeError("lse must be float32")
+    q, k, v, o, dout, lse = (t.contiguous() for t in (q, k, v, o, dout, lse))
+    if q.dim() != 4 or k.shape != v.shape or o.shape != q.shape or dout.shape != q.shape:
+        raise ValueError("dense layout: q, o, dout [B,Hq,N,d], k/v [B,Hkv,N,d]")
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = fa_bwd_workspace_bytes(B, Hq, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    rc = fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, workspace,
+                workspace.numel() * workspace.element_size(), torch.cuda.current_stream(q.device))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_bwd")
+    return dq, dk, dv
 
 
 def fa_selftest_watchdog(timeout_ms: int, stream=None) -> int:

@@ -1,0 +1,718 @@
+// fa_bwd.cu -- attention backward (dQ, dK, dV) for B200 (sm_100a) and its C ABI.
+//
+// The method's backward pass keeps the forward's memory saving: it does not
+// store the score matrix, it recomputes the scores block by block from Q and
+// K (pages: "Flash Attention", 14cs17.netlify.app, "Common Pitfalls",
+// Pitfall 3; fromzero2ai.dev, "Core Mechanisms of FlashAttention", item 3).
+// The gradients are those of the forward's definition: with
+// P = softmax(scale Q K^T) (masked), O = P V and the upstream gradient dO,
+//     dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),  D_i = sum_j dO_ij O_ij,
+//     dQ = scale dS K,  dK = scale dS^T Q,
+// and P_ij = exp(scale q_i.k_j - lse_i) from the logsumexp the forward saved.
+//
+// Three kernels on the caller's stream:
+//   1. fa_bwd_prep_kernel: D_i = rowsum(dO * O) and lse_i * log2(e) per query
+//      row, in row-padded fp32 arrays, and the fp32 dQ accumulator cleared.
+//   2. fa_bwd_kernel: one persistent CTA per SM; a work item is one 128-key
+//      block K_j, V_j of one (batch, kv head).  It keeps dK_j and dV_j in TMEM
+//      while it walks the query blocks Q_i, dO_i of every query head of the
+//      group (under the causal mask, i >= j only); per block it recomputes
+//      S^T = K_j Q_i^T, forms P^T and dS^T, accumulates dV_j and dK_j, and
+//      adds dQ_i's share into the fp32 accumulator with vector reductions.
+//   3. fa_bwd_dq_kernel: dQ = scale * accumulator, rounded to bf16.
+//
+// fa_bwd_kernel roles (384 threads):
+//   warps 0-3   P/dS warpgroup, one thread per key row: tcgen05.ld of S^T,
+//               P^T = exp2(S^T scale log2e - lse log2e) (masked), bf16 P^T
+//               back into TMEM; then tcgen05.ld of dP^T, dS^T = P^T (dP^T - D)
+//               to shared memory (bf16, 128-byte swizzled K-major tile).
+//   warps 4-7   dQ warpgroup, one thread per query row: tcgen05.ld of the
+//               block's dQ_i share and red.global.add.v4.f32 into the
+//               accumulator; at the end of an item, dK_j and dV_j from TMEM to
+//               HBM (bf16).
+//   warp 9      MMA issuer (one thread); warp 10 TMA producer (one thread);
+//   warp 8      TMEM allocation.
+//
+// TMEM columns (512): X [0,128) S^T, then P^T (bf16) in [0,64);
+// Y [128,256) dP^T, then the block's dQ_i share; dV [256,256+D); dK [384,384+D).
+// Shared memory: K_j, V_j, two Q slots (with their lse and D slices), one dO
+// slot and the dS tile.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace fa_sm100 {
+namespace bwd {
+
+constexpr int kBlock = 128;            // keys per item, queries per step
+constexpr int kThreads = 384;
+constexpr int kAllocWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kLoadWarp = 10;
+constexpr uint32_t kPdsRegs = 232;     // setmaxnreg: 128 x 232 + 128 x 168 + 128 x 104 = 384 x 168
+constexpr uint32_t kOtherRegs = 104;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kBoxBytes = kBlock * 64 * 2;   // one 128-row x 64-column bf16 TMA box
+constexpr uint32_t kColX = 0, kColY = 128, kColDV = 256, kColDK = 384;
+
+enum WaitSite : int {
+    kSiteKvEmpty = 11, kSiteKvFull, kSiteQEmpty, kSiteQFull, kSiteDoEmpty, kSiteDoFull, kSiteS, kSiteP, kSiteDp,
+    kSiteDs, kSiteDsFree, kSiteDq, kSiteYFree, kSiteAccDone, kSiteAccFree
+};
+
+struct alignas(64) Params {
+    CUtensorMap tm_q, tm_k, tm_v, tm_do;
+    const float* lse2;      // [B, Hq, Npad]: lse * log2(e); +inf on padding rows
+    const float* Dvec;      // [B, Hq, Npad]: rowsum(dO * O); 0 on padding rows
+    float* dq_acc;          // [B, Hq, Npad, d] fp32, cleared by the prep kernel
+    uint16_t* dk;           // [B, Hkv, N, d] bf16
+    uint16_t* dv;           // [B, Hkv, N, d] bf16
+    int* status;
+    int B, Hq, Hkv, N, Npad, group, causal;
+    float scale_log2, scale;
+    unsigned long long timeout_ns;
+};
+
+struct Misc {
+    uint64_t kv_full, kv_empty, q_full[2], q_empty[2], do_full, do_empty;
+    uint64_t s_full, p_full, dp_full, ds_full, ds_free, dq_full, y_free, acc_done, acc_free, drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+template <int D>
+struct Cfg {
+    static_assert(D == 64 || D == 128, "head dim");
+    static constexpr int kTileBytes = kBlock * D * 2;
+    static constexpr int kBoxes = D / 64;
+    static constexpr int kKOff = 0;
+    static constexpr int kVOff = kKOff + kTileBytes;
+    static constexpr int kQOff = kVOff + kTileBytes;              // two slots
+    static constexpr int kDoOff = kQOff + 2 * kTileBytes;
+    static constexpr int kDsOff = kDoOff + kTileBytes;            // 128 x 128 bf16
+    static constexpr int kVecOff = kDsOff + kBlock * kBlock * 2;  // lse2[2][128], D[2][128]
+    static constexpr int kMiscOff = kVecOff + 4 * kBlock * 4;
+    static constexpr int kSmemBytes = kMiscOff + (int)sizeof(Misc) + 1024;
+    static_assert(kSmemBytes <= 232448, "shared memory");
+};
+
+// One work item: key block j of one (batch, kv head).
+struct Item {
+    int b, hk, j;
+    int i0;       // first query block (causal: j)
+    int nq;       // query blocks per head
+    int niter;    // group * (nq - i0)
+};
+
+__device__ __forceinline__ int item_of_round(int r) {
+    const int G = gridDim.x;
+    return r * G + ((r & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+}
+
+// Items in increasing key block (under the causal mask the early key blocks
+// see the most query blocks: heaviest first), then (batch, kv head).
+__device__ __forceinline__ Item decode_item(int idx, const Params& p) {
+    Item it;
+    const int units = p.B * p.Hkv;
+    it.j = idx / units;
+    const int u = idx - it.j * units;
+    it.b = u / p.Hkv;
+    it.hk = u - it.b * p.Hkv;
+    it.nq = (p.N + kBlock - 1) / kBlock;
+    it.i0 = p.causal ? it.j : 0;
+    it.niter = p.group * (it.nq - it.i0);
+    return it;
+}
+
+// Iteration n of an item: query head h (of the group) and query block i.
+__device__ __forceinline__ void iter_of(const Item& it, int n, const Params& p, int& h, int& i) {
+    const int per = it.nq - it.i0;
+    const int g = n / per;
+    h = it.hk * p.group + g;
+    i = it.i0 + (n - g * per);
+}
+
+#ifndef FA_SUSPEND_NS
+#define FA_SUSPEND_NS 20000u
+#endif
+
+// Bounded wait: gives up after timeout_ns (recording the site in the status
+// word and raising the CTA's abort flag) or as soon as another role aborted.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Params& p, Misc& ms, int site) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait_sleep(bar, parity, FA_SUSPEND_NS)) return true;
+        if (*reinterpret_cast<volatile int*>(&ms.abort_flag)) return false;
+        if (globaltimer_ns() - t0 > p.timeout_ns) {
+            *reinterpret_cast<volatile int*>(&ms.abort_flag) = 1;
+            if (atomicCAS(p.status, 0, FA_ERR_DEVICE_TIMEOUT) == 0) {
+                p.status[1] = site;
+                p.status[2] = blockIdx.x;
+            }
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, const Params& p) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > p.timeout_ns) return;
+    }
+}
+
+// ---------------------------------------------------------------- producer
+template <int D>
+__device__ void load_role(const Params& p, Misc& ms, uint8_t* smem, int total) {
+    using C = Cfg<D>;
+    const uint64_t pol_keep = policy_evict_last();
+    const uint32_t s_k = smem_u32(smem + C::kKOff), s_v = smem_u32(smem + C::kVOff);
+    const uint32_t s_q = smem_u32(smem + C::kQOff), s_do = smem_u32(smem + C::kDoOff);
+    const uint32_t s_vec = smem_u32(smem + C::kVecOff);
+    uint32_t item_n = 0, ng = 0;
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+        const int idx = item_of_round(r);
+        if (idx >= total) break;
+        const Item it = decode_item(idx, p);
+        if (!(ok = wait_bar(smem_u32(&ms.kv_empty), (item_n & 1) ^ 1, p, ms, kSiteKvEmpty))) break;
+        mbar_arrive_expect_tx(smem_u32(&ms.kv_full), 2 * C::kTileBytes);
+        for (int bx = 0; bx < C::kBoxes; ++bx) {
+            tma_load_4d(s_k + bx * kBoxBytes, &p.tm_k, smem_u32(&ms.kv_full), bx * 64, it.j * kBlock, it.hk, it.b,
+                        pol_keep);
+            tma_load_4d(s_v + bx * kBoxBytes, &p.tm_v, smem_u32(&ms.kv_full), bx * 64, it.j * kBlock, it.hk, it.b,
+                        pol_keep);
+        }
+        ++item_n;
+        for (int n = 0; n < it.niter && ok; ++n, ++ng) {
+            int h, i;
+            iter_of(it, n, p, h, i);
+            const uint32_t slot = ng & 1;
+            // Q_i with its lse and D slices
+            if (!(ok = wait_bar(smem_u32(&ms.q_empty[slot]), ((ng >> 1) & 1) ^ 1, p, ms, kSiteQEmpty))) break;
+            const uint32_t qbar = smem_u32(&ms.q_full[slot]);
+            mbar_arrive_expect_tx(qbar, C::kTileBytes + 2 * kBlock * 4);
+            for (int bx = 0; bx < C::kBoxes; ++bx)
+                tma_load_4d(s_q + slot * C::kTileBytes + bx * kBoxBytes, &p.tm_q, qbar, bx * 64, i * kBlock, h, it.b,
+                            pol_keep);
+            const size_t row0 = (static_cast<size_t>(it.b) * p.Hq + h) * p.Npad + static_cast<size_t>(i) * kBlock;
+            bulk_load(s_vec + slot * kBlock * 4, p.lse2 + row0, kBlock * 4, qbar);
+            bulk_load(s_vec + (2 + slot) * kBlock * 4, p.Dvec + row0, kBlock * 4, qbar);
+            // dO_i
+            if (!(ok = wait_bar(smem_u32(&ms.do_empty), (ng & 1) ^ 1, p, ms, kSiteDoEmpty))) break;
+            const uint32_t dbar = smem_u32(&ms.do_full);
+            mbar_arrive_expect_tx(dbar, C::kTileBytes);
+            for (int bx = 0; bx < C::kBoxes; ++bx)
+                tma_load_4d(s_do + bx * kBoxBytes, &p.tm_do, dbar, bx * 64, i * kBlock, h, it.b, pol_keep);
+        }
+    }
+    if (!ok) {
+        // let the copies already issued land before the CTA goes away
+        if (item_n > 0) drain_bar(smem_u32(&ms.kv_full), (item_n - 1) & 1, p);
+        for (uint32_t g = (ng > 2 ? ng - 2 : 0); g <= ng; ++g) {
+            drain_bar(smem_u32(&ms.q_full[g & 1]), (g >> 1) & 1, p);
+            drain_bar(smem_u32(&ms.do_full), g & 1, p);
+        }
+    }
+}
+
+// ------------------------------------------------------------- MMA issuer
+template <int D>
+__device__ __forceinline__ void mma_qk(uint32_t d_tmem, uint64_t a, uint64_t b) {
+    constexpr uint32_t idesc = idesc_bf16_f32(kBlock, kBlock, false);
+    if constexpr (D == 128)
+        umma_ss_k128_x8(d_tmem, a, b, idesc);
+    else
+        umma_ss_k64_x4(d_tmem, a, b, idesc);
+}
+
+template <int D>
+__device__ void mma_role(const Params& p, Misc& ms, uint8_t* smem, uint32_t tmem, int total) {
+    using C = Cfg<D>;
+    constexpr uint64_t kTileStep = C::kTileBytes >> 4;
+    // K-major views (inner dimension d inside the swizzled rows)
+    const uint64_t dk_k = smem_desc_sw128(smem_u32(smem + C::kKOff), 16, 1024);
+    const uint64_t dv_k = smem_desc_sw128(smem_u32(smem + C::kVOff), 16, 1024);
+    const uint64_t dq_k0 = smem_desc_sw128(smem_u32(smem + C::kQOff), 16, 1024);
+    const uint64_t ddo_k = smem_desc_sw128(smem_u32(smem + C::kDoOff), 16, 1024);
+    const uint64_t dds_k = smem_desc_sw128(smem_u32(smem + C::kDsOff), 16, 1024);
+    // MN-major views (rows are the reduction dimension)
+    const uint64_t dk_mn = smem_desc_sw128(smem_u32(smem + C::kKOff), kBoxBytes, 1024);
+    const uint64_t dq_mn0 = smem_desc_sw128(smem_u32(smem + C::kQOff), kBoxBytes, 1024);
+    const uint64_t ddo_mn = smem_desc_sw128(smem_u32(smem + C::kDoOff), kBoxBytes, 1024);
+    const uint64_t dds_mn = smem_desc_sw128(smem_u32(smem + C::kDsOff), kBoxBytes, 1024);
+    constexpr uint32_t id_dv = idesc_bf16_f32(kBlock, D, true);          // P^T (TMEM) x dO (MN)
+    constexpr uint32_t id_dk = idesc_bf16_f32(kBlock, D, true);          // dS^T (K-major) x Q (MN)
+    constexpr uint32_t id_dq = idesc_bf16_f32(kBlock, D, true, true);    // dS (MN) x K (MN)
+    uint32_t item_n = 0, ng = 0;
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+        const int idx = item_of_round(r);
+        if (idx >= total) break;
+        const Item it = decode_item(idx, p);
+        if (!(ok = wait_bar(smem_u32(&ms.kv_full), item_n & 1, p, ms, kSiteKvFull))) break;
+        tc_fence_after();
+        for (int n = 0; n < it.niter && ok; ++n, ++ng) {
+            const uint32_t slot = ng & 1;
+            if (n == 0) {          // S^T of the item's first block
+                if (!(ok = wait_bar(smem_u32(&ms.q_full[slot]), (ng >> 1) & 1, p, ms, kSiteQFull))) break;
+                tc_fence_after();
+                mma_qk<D>(tmem + kColX, dk_k, dq_k0 + slot * kTileStep);
+                umma_commit(smem_u32(&ms.s_full));
+            }
+            // dV_j += P^T dO_i, once P^T is in TMEM
+            if (!(ok = wait_bar(smem_u32(&ms.p_full), ng & 1, p, ms, kSiteP))) break;
+            if (n == 0 && !(ok = wait_bar(smem_u32(&ms.acc_free), (item_n & 1) ^ 1, p, ms, kSiteAccFree))) break;
+            if (!(ok = wait_bar(smem_u32(&ms.do_full), ng & 1, p, ms, kSiteDoFull))) break;
+            tc_fence_after();
+            umma_ts_kv128_x8(tmem + kColDV, tmem + kColX, ddo_mn, id_dv, n > 0 ? 1u : 0u);
+            // dP^T = V_j dO_i^T, once the previous dQ share has left Y
+            if (!(ok = wait_bar(smem_u32(&ms.y_free), (ng & 1) ^ 1, p, ms, kSiteYFree))) break;
+            tc_fence_after();
+            mma_qk<D>(tmem + kColY, dv_k, ddo_k);
+            umma_commit(smem_u32(&ms.dp_full));
+            umma_commit(smem_u32(&ms.do_empty));
+            // S^T of the next block (X is free once dV has read P^T: in order)
+            if (n + 1 < it.niter) {
+                const uint32_t ns = (ng + 1) & 1;
+                if (!(ok = wait_bar(smem_u32(&ms.q_full[ns]), ((ng + 1) >> 1) & 1, p, ms, kSiteQFull))) break;
+                tc_fence_after();
+                mma_qk<D>(tmem + kColX, dk_k, dq_k0 + ns * kTileStep);
+                umma_commit(smem_u32(&ms.s_full));
+            }
+            // dK_j += dS^T Q_i and dQ_i share = dS K_j, once dS is in shared memory
+            if (!(ok = wait_bar(smem_u32(&ms.ds_full), ng & 1, p, ms, kSiteDs))) break;
+            tc_fence_after();
+            umma_ss_kA_mnB_k128_x8(tmem + kColDK, dds_k, dq_mn0 + slot * kTileStep, id_dk, n > 0 ? 1u : 0u);
+            umma_ss_mnA_mnB_k128_x8(tmem + kColY, dds_mn, dk_mn, id_dq);
+            umma_commit(smem_u32(&ms.dq_full));
+            umma_commit(smem_u32(&ms.ds_free));
+            umma_commit(smem_u32(&ms.q_empty[slot]));
+            if (n == it.niter - 1) {
+                umma_commit(smem_u32(&ms.acc_done));
+                umma_commit(smem_u32(&ms.kv_empty));
+            }
+        }
+        ++item_n;
+    }
+    umma_commit(smem_u32(&ms.drain));
+    drain_bar(smem_u32(&ms.drain), 0, p);
+}
+
+// -------------------------------------------------- P / dS warpgroup
+// Byte offset of 16-byte chunk `c16` (8 bf16 columns, 0..15) of row `r` in a
+// 128-row x 128-column bf16 tile stored as two 128-byte-swizzled 64-column
+// boxes (the layout TMA writes, read K-major or MN-major by the MMAs).
+__device__ __forceinline__ uint32_t sw128_chunk(int r, int c16) {
+    return static_cast<uint32_t>((c16 >> 3) * kBoxBytes + r * 128 + (((c16 & 7) ^ (r & 7)) << 4));
+}
+
+template <int D>
+__device__ void pds_role(const Params& p, Misc& ms, uint8_t* smem, uint32_t tmem, int warp, int lane, int total) {
+    using C = Cfg<D>;
+    const int r = warp * 32 + lane;                     // key row inside the block
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tx = tmem + lane_off + kColX, ty = tmem + lane_off + kColY;
+    const float* vec = reinterpret_cast<const float*>(smem + C::kVecOff);
+    uint8_t* ds_tile = smem + C::kDsOff;
+    const float sl2 = p.scale_log2;
+    uint32_t ng = 0;
+    bool ok = true;
+    for (int rr = 0; ok; ++rr) {
+        const int idx = item_of_round(rr);
+        if (idx >= total) break;
+        const Item it = decode_item(idx, p);
+        const bool key_valid = it.j * kBlock + r < p.N;
+        for (int n = 0; n < it.niter; ++n, ++ng) {
+            int h, i;
+            iter_of(it, n, p, h, i);
+            const uint32_t slot = ng & 1;
+            const float* lse2 = vec + slot * kBlock;
+            const float* dvec = vec + (2 + slot) * kBlock;
+            ok = wait_bar(smem_u32(&ms.s_full), ng & 1, p, ms, kSiteS);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t s[128];
+            tmem_ld128_sync(tx, s);
+            // P^T = exp2(S^T * scale * log2 e - lse * log2 e); key r vs query c
+            const bool diag = p.causal && i == it.j;
+#pragma unroll
+            for (int c = 0; c < 128; c += 4) {
+                const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c);
+                float e0 = ex2_approx(fmaf(__uint_as_float(s[c]), sl2, -l4.x));
+                float e1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), sl2, -l4.y));
+                float e2 = ex2_approx(fmaf(__uint_as_float(s[c + 2]), sl2, -l4.z));
+                float e3 = ex2_approx(fmaf(__uint_as_float(s[c + 3]), sl2, -l4.w));
+                if (diag) {        // query c sees key r only if r <= c
+                    if (c < r) e0 = 0.f;
+                    if (c + 1 < r) e1 = 0.f;
+                    if (c + 2 < r) e2 = 0.f;
+                    if (c + 3 < r) e3 = 0.f;
+                }
+                if (!key_valid) e0 = e1 = e2 = e3 = 0.f;
+                s[c] = __float_as_uint(e0);
+                s[c + 1] = __float_as_uint(e1);
+                s[c + 2] = __float_as_uint(e2);
+                s[c + 3] = __float_as_uint(e3);
+            }
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int t = 0; t < 32; ++t)
+                    pk[t] = pack_bf16x2(__uint_as_float(s[64 * hf + 2 * t]), __uint_as_float(s[64 * hf + 2 * t + 1]));
+                tmem_st32(tx + 32 * hf, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ms.p_full));
+            // dS^T = P^T (dP^T - D), into the shared dS tile
+            ok = wait_bar(smem_u32(&ms.dp_full), ng & 1, p, ms, kSiteDp);
+            ok = ok && wait_bar(smem_u32(&ms.ds_free), (ng & 1) ^ 1, p, ms, kSiteDsFree);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                uint32_t dp[32];
+                tmem_ld32_sync(ty + 32 * q4, dp);
+                uint32_t pk[16];
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    const int c = 32 * q4 + 2 * t;
+                    const float2 d2 = *reinterpret_cast<const float2*>(dvec + c);
+                    const float a = __uint_as_float(s[c]) * (__uint_as_float(dp[2 * t]) - d2.x);
+                    const float b = __uint_as_float(s[c + 1]) * (__uint_as_float(dp[2 * t + 1]) - d2.y);
+                    pk[t] = pack_bf16x2(a, b);
+                }
+#pragma unroll
+                for (int t = 0; t < 4; ++t)
+                    *reinterpret_cast<uint4*>(ds_tile + sw128_chunk(r, 4 * q4 + t)) =
+                        make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ms.ds_full));
+        }
+    }
+}
+
+// ------------------------------------------------------- dQ warpgroup
+template <int D>
+__device__ void dq_role(const Params& p, Misc& ms, uint32_t tmem, int wq, int lane, int total) {
+    const int r = wq * 32 + lane;                       // query row (dQ) or key row (dK, dV)
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t ty = tmem + lane_off + kColY;
+    uint32_t item_n = 0, ng = 0;
+    bool ok = true;
+    for (int rr = 0; ok; ++rr) {
+        const int idx = item_of_round(rr);
+        if (idx >= total) break;
+        const Item it = decode_item(idx, p);
+        for (int n = 0; n < it.niter; ++n, ++ng) {
+            int h, i;
+            iter_of(it, n, p, h, i);
+            ok = wait_bar(smem_u32(&ms.dq_full), ng & 1, p, ms, kSiteDq);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            float* dst = p.dq_acc + ((static_cast<size_t>(it.b) * p.Hq + h) * p.Npad + static_cast<size_t>(i) * kBlock + r) * D;
+            uint32_t a[32], b[32];
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) {
+                tmem_ld64_sync(ty + 64 * c, a, b);
+                if (c == D / 64 - 1) {
+                    // Y may take the next dP once every lane has its values
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&ms.y_free));
+                }
+#pragma unroll
+                for (int t = 0; t < 8; ++t)
+                    red_add_v4(dst + 64 * c + 4 * t, __uint_as_float(a[4 * t]), __uint_as_float(a[4 * t + 1]),
+                               __uint_as_float(a[4 * t + 2]), __uint_as_float(a[4 * t + 3]));
+#pragma unroll
+                for (int t = 0; t < 8; ++t)
+                    red_add_v4(dst + 64 * c + 32 + 4 * t, __uint_as_float(b[4 * t]), __uint_as_float(b[4 * t + 1]),
+                               __uint_as_float(b[4 * t + 2]), __uint_as_float(b[4 * t + 3]));
+            }
+        }
+        if (!ok) break;
+        // dK_j, dV_j of the item: TMEM -> bf16 -> HBM
+        ok = wait_bar(smem_u32(&ms.acc_done), item_n & 1, p, ms, kSiteAccDone);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        ++item_n;
+        tc_fence_after();
+        const int key = it.j * kBlock + r;
+        const size_t row = (static_cast<size_t>(it.b) * p.Hkv + it.hk) * p.N + key;
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+            const float mul = which == 0 ? 1.f : p.scale;
+            uint16_t* out = (which == 0 ? p.dv : p.dk) + row * D;
+            const uint32_t col = which == 0 ? kColDV : kColDK;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32_sync(tmem + lane_off + col + 32 * c, v);
+                uint32_t pk[16];
+#pragma unroll
+                for (int t = 0; t < 16; ++t)
+                    pk[t] = pack_bf16x2(__uint_as_float(v[2 * t]) * mul, __uint_as_float(v[2 * t + 1]) * mul);
+                if (key < p.N) {
+                    uint4* o4 = reinterpret_cast<uint4*>(out + 32 * c);
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) o4[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+                }
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&ms.acc_free));
+    }
+}
+
+// ------------------------------------------------------------------ kernel
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) fa_bwd_kernel(const __grid_constant__ Params p) {
+    using C = Cfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Misc& ms = *reinterpret_cast<Misc*>(smem + C::kMiscOff);
+    const int tid = threadIdx.x;
+    const int warp = tid / 32, lane = tid % 32;
+    if (tid == 0) {
+        mbar_init(smem_u32(&ms.kv_full), 1);
+        mbar_init(smem_u32(&ms.kv_empty), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_u32(&ms.q_full[s]), 1);
+            mbar_init(smem_u32(&ms.q_empty[s]), 1);
+        }
+        mbar_init(smem_u32(&ms.do_full), 1);
+        mbar_init(smem_u32(&ms.do_empty), 1);
+        mbar_init(smem_u32(&ms.s_full), 1);
+        mbar_init(smem_u32(&ms.p_full), 4);       // one arrival per warp of the P/dS warpgroup
+        mbar_init(smem_u32(&ms.dp_full), 1);
+        mbar_init(smem_u32(&ms.ds_full), 4);
+        mbar_init(smem_u32(&ms.ds_free), 1);
+        mbar_init(smem_u32(&ms.dq_full), 1);
+        mbar_init(smem_u32(&ms.y_free), 4);       // one arrival per warp of the dQ warpgroup
+        mbar_init(smem_u32(&ms.acc_done), 1);
+        mbar_init(smem_u32(&ms.acc_free), 4);
+        mbar_init(smem_u32(&ms.drain), 1);
+        ms.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kLoadWarp && lane == 0) {
+        prefetch_tensormap(&p.tm_q);
+        prefetch_tensormap(&p.tm_k);
+        prefetch_tensormap(&p.tm_v);
+        prefetch_tensormap(&p.tm_do);
+    }
+    if (warp == kAllocWarp) {
+        tmem_alloc(smem_u32(&ms.tmem_base), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ms.tmem_base;
+    const int total = ((p.N + kBlock - 1) / kBlock) * p.B * p.Hkv;
+
+    if (warp < 4) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kPdsRegs));
+        pds_role<D>(p, ms, smem, tmem, warp, lane, total);
+    } else if (warp < 8) {
+        dq_role<D>(p, ms, tmem, warp - 4, lane, total);
+    } else {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
+        if (warp == kMmaWarp) {
+            if (lane == 0) mma_role<D>(p, ms, smem, tmem, total);
+            __syncwarp();
+        } else if (warp == kLoadWarp) {
+            if (lane == 0) load_role<D>(p, ms, smem, total);
+            __syncwarp();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kAllocWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// D_i = sum_c dO_ic O_ic (fp32 from bf16), lse_i * log2(e), on rows padded to
+// a multiple of 128 (padding: D = 0, lse2 = +inf so that P = 0 there); and
+// the dQ accumulator cleared.  One warp per padded row.
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
+                                                          const float* __restrict__ lse, float* lse2, float* Dvec,
+                                                          float* dq_acc, int N, int Npad, long long rows_pad) {
+    const long long row = static_cast<long long>(blockIdx.x) * 8 + threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    if (row >= rows_pad) return;
+    const long long bh = row / Npad;
+    const int t = static_cast<int>(row - bh * Npad);
+    float* acc = dq_acc + row * D;
+    for (int c = lane * 4; c < D; c += 128) *reinterpret_cast<float4*>(acc + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+    float dsum = 0.f;
+    if (t < N) {
+        const size_t src = (static_cast<size_t>(bh) * N + t) * D;
+        for (int c = lane * 2; c < D; c += 64) {
+            const uint32_t ov = *reinterpret_cast<const uint32_t*>(o + src + c);
+            const uint32_t dv = *reinterpret_cast<const uint32_t*>(dout + src + c);
+            dsum += __uint_as_float(ov << 16) * __uint_as_float(dv << 16) +
+                    __uint_as_float(ov & 0xFFFF0000u) * __uint_as_float(dv & 0xFFFF0000u);
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
+    if (lane == 0) {
+        float l2 = INFINITY;
+        if (t < N) {
+            const float l = lse[static_cast<size_t>(bh) * N + t];
+            l2 = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+        }
+        lse2[row] = l2;
+        Dvec[row] = t < N ? dsum : 0.f;
+    }
+}
+
+// dQ = scale * accumulator -> bf16, rows < N.  One thread per 4 values.
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float* __restrict__ dq_acc, uint16_t* dq, float scale,
+                                                        int N, int Npad, long long total4) {
+    const long long e4 = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
+    if (e4 >= total4) return;
+    const long long e = e4 * 4;
+    const long long row = e / D;               // row of [B*Hq, N]
+    const int c = static_cast<int>(e - row * D);
+    const long long bh = row / N;
+    const long long t = row - bh * N;
+    const float4 v = *reinterpret_cast<const float4*>(dq_acc + (bh * Npad + t) * D + c);
+    *reinterpret_cast<uint2*>(dq + e) = make_uint2(pack_bf16x2(v.x * scale, v.y * scale), pack_bf16x2(v.z * scale, v.w * scale));
+}
+
+static std::mutex g_bwd_mu;
+static bool g_bwd_ready[kMaxDevices];
+
+static int bwd_setup(int dev) {
+    std::lock_guard<std::mutex> lock(g_bwd_mu);
+    if (g_bwd_ready[dev]) return FA_OK;
+    bool good = cudaFuncSetAttribute(fa_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Cfg<64>::kSmemBytes) == cudaSuccess;
+    good = good && cudaFuncSetAttribute(fa_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        Cfg<128>::kSmemBytes) == cudaSuccess;
+    if (!good) return FA_ERR_LAUNCH;
+    g_bwd_ready[dev] = true;
+    return FA_OK;
+}
+
+static size_t workspace_bytes(int B, int Hq, int N, int d) {
+    const size_t npad = (static_cast<size_t>(N) + kBlock - 1) / kBlock * kBlock;
+    return static_cast<size_t>(B) * Hq * npad * (d + 2) * sizeof(float);
+}
+
+static bool aligned(const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) == 0; }
+
+}  // namespace bwd
+}  // namespace fa_sm100
+
+using namespace fa_sm100;
+
+extern "C" size_t fa_bwd_workspace_bytes(int B, int Hq, int N, int d) {
+    if (B < 0 || Hq < 1 || N < 0 || (d != 64 && d != 128)) return 0;
+    return bwd::workspace_bytes(B, Hq, N, d);
+}
+
+extern "C" int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                      void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+    using namespace bwd;
+    if (B < 0 || N < 0 || Hq < 1) return FA_ERR_SHAPE;
+    if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+    if (Hkv < 1 || Hq % Hkv != 0) return FA_ERR_GQA;
+    if (B == 0 || N == 0) return FA_OK;
+    if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return FA_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
+        !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) || !aligned(workspace, 16))
+        return FA_ERR_ALIGN;
+    const long long npad = (static_cast<long long>(N) + kBlock - 1) / kBlock * kBlock;
+    if ((long long)B * Hq * npad > (1ll << 30) || (long long)B * Hkv * ((N + kBlock - 1) / kBlock) > (1ll << 30))
+        return FA_ERR_SHAPE;
+    if (workspace_bytes < bwd::workspace_bytes(B, Hq, N, d)) return FA_ERR_SHAPE;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_LAUNCH;
+    DeviceState* ds = nullptr;
+    int st = init_device(dev, &ds);
+    if (st != FA_OK) return st;
+    if ((st = bwd_setup(dev)) != FA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    const long long rows_pad = (long long)B * Hq * npad;
+    float* dq_acc = static_cast<float*>(workspace);
+    float* lse2 = dq_acc + rows_pad * d;
+    float* Dvec = lse2 + rows_pad;
+
+    Params P;
+    std::memset(&P, 0, sizeof(P));
+    {
+        const uint64_t e = 2;
+        const uint32_t box[4] = {64, (uint32_t)kBlock, 1, 1};
+        const uint64_t dq_[4] = {(uint64_t)d, (uint64_t)N, (uint64_t)Hq, (uint64_t)B};
+        const uint64_t sq[3] = {d * e, (uint64_t)N * d * e, (uint64_t)Hq * N * d * e};
+        const uint64_t dk_[4] = {(uint64_t)d, (uint64_t)N, (uint64_t)Hkv, (uint64_t)B};
+        const uint64_t sk[3] = {d * e, (uint64_t)N * d * e, (uint64_t)Hkv * N * d * e};
+        if (!encode_map(&P.tm_q, q, dq_, sq, box) || !encode_map(&P.tm_do, dout, dq_, sq, box) ||
+            !encode_map(&P.tm_k, k, dk_, sk, box) || !encode_map(&P.tm_v, v, dk_, sk, box))
+            return FA_ERR_LAUNCH;
+    }
+    P.lse2 = lse2;
+    P.Dvec = Dvec;
+    P.dq_acc = dq_acc;
+    P.dk = static_cast<uint16_t*>(dk);
+    P.dv = static_cast<uint16_t*>(dv);
+    P.status = ds->status;
+    P.B = B;
+    P.Hq = Hq;
+    P.Hkv = Hkv;
+    P.N = N;
+    P.Npad = (int)npad;
+    P.group = Hq / Hkv;
+    P.causal = causal ? 1 : 0;
+    P.scale = scale;
+    P.scale_log2 = scale * 1.4426950408889634f;
+    P.timeout_ns = 2000000000ull;
+
+    const unsigned prep_grid = static_cast<unsigned>((rows_pad + 7) / 8);
+    const long long items = (long long)B * Hkv * ((N + kBlock - 1) / kBlock);
+    const int grid = (int)std::min<long long>(items, ds->num_sms);
+    const long long total4 = (long long)B * Hq * N * d / 4;
+    const unsigned post_grid = static_cast<unsigned>((total4 + 255) / 256);
+    if (d == 64) {
+        fa_bwd_prep_kernel<64><<<prep_grid, 256, 0, s>>>(static_cast<const uint16_t*>(o),
+                                                          static_cast<const uint16_t*>(dout), lse, lse2, Dvec, dq_acc,
+                                                          N, (int)npad, rows_pad);
+        fa_bwd_kernel<64><<<grid, kThreads, Cfg<64>::kSmemBytes, s>>>(P);
+        fa_bwd_dq_kernel<64><<<post_grid, 256, 0, s>>>(dq_acc, static_cast<uint16_t*>(dq), scale, N, (int)npad, total4);
+    } else {
+        fa_bwd_prep_kernel<128><<<prep_grid, 256, 0, s>>>(static_cast<const uint16_t*>(o),
+                                                           static_cast<const uint16_t*>(dout), lse, lse2, Dvec, dq_acc,
+                                                           N, (int)npad, rows_pad);
+        fa_bwd_kernel<128><<<grid, kThreads, Cfg<128>::kSmemBytes, s>>>(P);
+        fa_bwd_dq_kernel<128><<<post_grid, 256, 0, s>>>(dq_acc, static_cast<uint16_t*>(dq), scale, N, (int)npad,
+                                                        total4);
+    }
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}

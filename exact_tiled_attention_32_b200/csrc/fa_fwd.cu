@@ -38,6 +38,7 @@
 #include <mutex>
 
 #include "fa.h"
+#include "fa_internal.cuh"
 #include "sm100_ptx.cuh"
 
 namespace fa_sm100 {
@@ -869,19 +870,11 @@ __global__ void fa_watchdog_probe_kernel(const __grid_constant__ Params p) {
 }
 
 // =================================================================== host
-struct DeviceState {
-    bool init = false;
-    int status_code = FA_OK;
-    int num_sms = 0;
-    int* status = nullptr;        // device: [0] code, [1] wait site, [2] block
-};
-
-constexpr int kMaxDevices = 64;
 static DeviceState g_dev[kMaxDevices];
 static std::mutex g_mu;
 static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
-static int init_device(int dev, DeviceState** out) {
+int init_device(int dev, DeviceState** out) {
     if (dev < 0 || dev >= kMaxDevices) return FA_ERR_LAUNCH;
     std::lock_guard<std::mutex> lock(g_mu);
     DeviceState& ds = g_dev[dev];
@@ -925,8 +918,8 @@ static int init_device(int dev, DeviceState** out) {
 }
 
 // 4-D bf16 tensor map with a 64 x rows box, 128-byte swizzle.
-static bool encode_map(CUtensorMap* m, const void* base, const uint64_t dims[4], const uint64_t strides[3],
-                       const uint32_t box[4]) {
+bool encode_map(CUtensorMap* m, const void* base, const uint64_t dims[4], const uint64_t strides[3],
+                const uint32_t box[4]) {
     const cuuint32_t elem[4] = {1, 1, 1, 1};
     CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
                           elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

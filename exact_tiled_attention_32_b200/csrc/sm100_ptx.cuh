@@ -210,6 +210,54 @@ __device__ __forceinline__ void umma_ts_kv64_x4(uint32_t d_tmem, uint32_t a_tmem
         : "memory");
 }
 
+// D (+)= A B over K = 128 with A K-major (K inside the 128-byte rows: +2 per
+// 16-element step in the start-address field, +1024 for the second 64-column
+// box) and B MN-major (K along the rows: 16 rows = 2 KB = +128 per step).
+// The first MMA accumulates only if `accumulate` is nonzero.
+__device__ __forceinline__ void umma_ss_kA_mnB_k128_x8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                      uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p0, pt;\n\t.reg .b64 a1, a2, a3, a4, a5, a6, a7, b1, b2, b3, b4, b5, b6, b7;\n\t"
+        "setp.ne.b32 p0, %4, 0;\n\tsetp.eq.b32 pt, %3, %3;\n\t"
+        "add.s64 a1, %1, 2;\n\tadd.s64 b1, %2, 128;\n\tadd.s64 a2, %1, 4;\n\tadd.s64 b2, %2, 256;\n\t"
+        "add.s64 a3, %1, 6;\n\tadd.s64 b3, %2, 384;\n\tadd.s64 a4, %1, 1024;\n\tadd.s64 b4, %2, 512;\n\t"
+        "add.s64 a5, %1, 1026;\n\tadd.s64 b5, %2, 640;\n\tadd.s64 a6, %1, 1028;\n\tadd.s64 b6, %2, 768;\n\t"
+        "add.s64 a7, %1, 1030;\n\tadd.s64 b7, %2, 896;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %3, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %3, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a4, b4, %3, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a5, b5, %3, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a6, b6, %3, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a7, b7, %3, pt;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// D = A B over K = 128 with A and B both MN-major (K along the rows of both:
+// +128 per 16-row step in each start-address field); the first MMA
+// overwrites D.
+__device__ __forceinline__ void umma_ss_mnA_mnB_k128_x8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                       uint32_t idesc) {
+    asm volatile(
+        "{\n\t.reg .pred pf, pt;\n\t.reg .b64 a1, a2, a3, a4, a5, a6, a7, b1, b2, b3, b4, b5, b6, b7;\n\t"
+        "setp.ne.b32 pf, %3, %3;\n\tsetp.eq.b32 pt, %3, %3;\n\t"
+        "add.s64 a1, %1, 128;\n\tadd.s64 b1, %2, 128;\n\tadd.s64 a2, %1, 256;\n\tadd.s64 b2, %2, 256;\n\t"
+        "add.s64 a3, %1, 384;\n\tadd.s64 b3, %2, 384;\n\tadd.s64 a4, %1, 512;\n\tadd.s64 b4, %2, 512;\n\t"
+        "add.s64 a5, %1, 640;\n\tadd.s64 b5, %2, 640;\n\tadd.s64 a6, %1, 768;\n\tadd.s64 b6, %2, 768;\n\t"
+        "add.s64 a7, %1, 896;\n\tadd.s64 b7, %2, 896;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, pf;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %3, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %3, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a4, b4, %3, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a5, b5, %3, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a6, b6, %3, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a7, b7, %3, pt;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc)
+        : "memory");
+}
+
 // arrive once on `bar` when every tcgen05 op issued so far by this thread is done
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -233,10 +281,11 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo_
 }
 
 // Instruction descriptor for kind::f16: fp32 accumulator (bits 4-5 = 1),
-// A and B bf16 (bits 7-9, 10-12 = 1), B major-ness in bit 16 (1 = MN-major),
-// N >> 3 in bits 17-22, M >> 4 in bits 24-28.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+// A and B bf16 (bits 7-9, 10-12 = 1), A and B major-ness in bits 15 and 16
+// (1 = MN-major; A from TMEM is always K-major), N >> 3 in bits 17-22,
+// M >> 4 in bits 24-28.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major, bool a_mn_major = false) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
            (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
@@ -304,6 +353,25 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
         "r"(r[29]), "r"(r[30]), "r"(r[31])
         : "memory");
+}
+
+// Untiled bulk copy global -> this CTA's shared memory (no multicast);
+// completion as transaction bytes on `bar`.  Both addresses 16-byte aligned,
+// size a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (tensor-core operand reads) before it signals them.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Four fp32 additions into global memory, one 16-byte reduction.
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
 }
 
 // ------------------------------------------------------------- arithmetic

@@ -151,6 +151,56 @@ int fa_splitkv_num_splits(int B, int Hq, int Hkv, int Nq, int Nk, int d);
 size_t fa_splitkv_workspace_bytes(int B, int Hq, int Nq, int d, int num_splits);
 
 /*
+ * fa_bwd -- gradients of fa_fwd (dense batches), asynchronous on `stream`.
+ * The backward pass recomputes the scores block by block from Q and K and the
+ * logsumexp that fa_fwd saved, instead of storing them ("Flash Attention",
+ * 14cs17.netlify.app, "Common Pitfalls", Pitfall 3; fromzero2ai.dev, "Core
+ * Mechanisms of FlashAttention", item 3).  The gradients are those of the
+ * forward's definition: with P = softmax(scale Q K^T) (masked) and the
+ * upstream gradient dO,
+ *     dV = P^T dO,  dS = P * (dO V^T - D),  D_i = sum_c dO_ic O_ic,
+ *     dQ = scale dS K,  dK = scale dS^T Q,
+ * the query heads of a group adding into their key/value head's dK and dV.
+ *
+ *   q, k, v, o, lse   the forward's inputs and outputs (o bf16, lse fp32 as
+ *                     fa_fwd wrote them), device memory, read only.
+ *   dout              bf16 upstream gradient, same layout as o.
+ *   dq                bf16 output, layout of q.
+ *   dk, dv            bf16 outputs, layout of k (written, not accumulated).
+ *   workspace         device memory, 16-byte aligned, at least
+ *                     fa_bwd_workspace_bytes(B, Hq, N, d) bytes: an fp32 dQ
+ *                     accumulator and two per-row fp32 vectors, on rows padded
+ *                     to a multiple of 128.  Nothing in it needs initialising;
+ *                     it must not be used by anything else until the call's
+ *                     kernels have finished on `stream`.
+ *   B, Hq, Hkv, N, d, scale, causal   as fa_fwd (dense layout only:
+ *                     q, o, dout, dq [B, Hq, N, d]; k, v, dk, dv
+ *                     [B, Hkv, N, d]; lse [B, Hq, N]).
+ *
+ * Three kernels run on `stream`: a pass computing D and clearing the
+ * accumulator, the main kernel (one 128-key block of one (batch, kv head)
+ * per work item, dK and dV kept in tensor memory, each block's dQ share
+ * added into the accumulator with fp32 reductions), and the dQ conversion.
+ * The order of the fp32 reductions varies from run to run, so dQ may differ
+ * in its last bits between runs; dK and dV do not.
+ *
+ * Errors as fa_fwd (FA_ERR_NULL also for a missing workspace, FA_ERR_ALIGN for
+ * a misaligned one, FA_ERR_SHAPE for one that is too small).  B == 0 or N == 0
+ * is an empty problem (FA_OK, nothing launched).
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dout, void* dq, void* dk, void* dv,
+           int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fa_bwd_workspace_bytes -- workspace fa_bwd needs:
+ * B * Hq * Npad * (d + 2) * 4 bytes with Npad = N rounded up to 128; 0 for
+ * invalid arguments.  Needs no device.
+ */
+size_t fa_bwd_workspace_bytes(int B, int Hq, int N, int d);
+
+/*
  * fa_get_device_status -- reads and clears the status word of the current
  * device.  Synchronises `stream` (a cudaStream_t) first, so it reports every
  * fa_fwd launched on that stream before the call.  Returns FA_OK, a negative

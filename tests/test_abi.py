@@ -104,6 +104,28 @@ def test_splitkv_workspace_bytes():
     assert fa.fa_splitkv_workspace_bytes(1, 1, 1, 64, 257) == 0
 
 
+def test_bwd_argument_errors_and_workspace_bytes():
+    from exact_tiled_attention_32_b200 import binding as fa
+    p = 1 << 20
+    # B * Hq * Npad * (d + 2) * 4 with Npad = N rounded up to 128
+    assert fa.fa_bwd_workspace_bytes(2, 4, 300, 128) == 2 * 4 * 384 * 130 * 4
+    assert fa.fa_bwd_workspace_bytes(1, 1, 128, 64) == 128 * 66 * 4
+    assert fa.fa_bwd_workspace_bytes(1, 1, 128, 96) == 0
+
+    def call(ptrs=(p,) * 9, ws=p, wb=1 << 30, B=1, Hq=4, Hkv=2, N=100, d=128):
+        return fa.fa_bwd(*ptrs, B, Hq, Hkv, N, d, 0.1, 1, ws, wb)
+
+    assert call(d=96) == fa.FA_ERR_HEADDIM
+    assert call(Hkv=3) == fa.FA_ERR_GQA
+    assert call(N=-1) == fa.FA_ERR_SHAPE
+    assert call(ws=0) == fa.FA_ERR_NULL
+    assert call(ptrs=(p,) * 8 + (0,)) == fa.FA_ERR_NULL
+    assert call(ws=p + 4) == fa.FA_ERR_ALIGN
+    assert call(ptrs=(p + 2,) + (p,) * 8) == fa.FA_ERR_ALIGN
+    assert call(wb=fa.fa_bwd_workspace_bytes(1, 4, 100, 128) - 16) == fa.FA_ERR_SHAPE
+    assert call(B=0, ptrs=(0,) * 9, ws=0, wb=0) == fa.FA_OK
+
+
 def test_no_device_means_launch_error():
     import torch
     if torch.cuda.is_available():
