@@ -21,22 +21,25 @@
 //      adds dQ_i's share into the fp32 accumulator with vector reductions.
 //   3. fa_bwd_dq_kernel: dQ = scale * accumulator, rounded to bf16.
 //
-// fa_bwd_kernel roles (384 threads):
-//   warps 0-3   P/dS warpgroup, one thread per key row: tcgen05.ld of S^T,
+// fa_bwd_kernel roles (512 threads):
+//   warps 0-7   two P/dS warpgroups, one thread per key row, warpgroup g
+//               taking query columns 64g .. 64g+63: tcgen05.ld of S^T,
 //               P^T = exp2(S^T scale log2e - lse log2e) (masked), bf16 P^T
 //               back into TMEM; then tcgen05.ld of dP^T, dS^T = P^T (dP^T - D)
 //               to shared memory (bf16, 128-byte swizzled K-major tile).
-//   warps 4-7   dQ warpgroup, one thread per query row: tcgen05.ld of the
-//               block's dQ_i share and red.global.add.v4.f32 into the
-//               accumulator; at the end of an item, dK_j and dV_j from TMEM to
-//               HBM (bf16).
-//   warp 9      MMA issuer (one thread); warp 10 TMA producer (one thread);
-//   warp 8      TMEM allocation.
+//   warps 8-11  dQ warpgroup, one thread per query row: tcgen05.ld of the
+//               block's dQ_i share, staged through shared memory so that each
+//               red.global.add.v4.f32 instruction covers whole 128-byte rows
+//               of the accumulator; at the end of an item, dK_j and dV_j from
+//               TMEM to HBM (bf16).
+//   warp 13     MMA issuer (one thread); warps 14 and 15 TMA producers (one
+//               thread each: K, V, Q and the lse / D slices; dO);
+//   warp 12     TMEM allocation.
 //
 // TMEM columns (512): X [0,128) S^T, then P^T (bf16) in [0,64);
 // Y [128,256) dP^T, then the block's dQ_i share; dV [256,256+D); dK [384,384+D).
 // Shared memory: K_j, V_j, two Q slots (with their lse and D slices), one dO
-// slot and the dS tile.
+// slot, the dS tile and the dQ staging tiles.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -54,20 +57,39 @@
 namespace fa_sm100 {
 namespace bwd {
 
+// Optional pipeline timeline (compile with -DFA_TRACE): CTA 0 records clock64
+// stamps as [role][iteration][event], 256 iterations and 8 events per role;
+// the buffer is set with fa_bwd_trace_set.
+#ifdef FA_TRACE
+__device__ unsigned long long* g_btrace = nullptr;
+#define BWD_TRACE(role, it, ev)                                                                          \
+    do {                                                                                                 \
+        if (blockIdx.x == 0 && g_btrace && (it) < 256) g_btrace[((role) * 256 + (it)) * 8 + (ev)] = clock64(); \
+    } while (0)
+#else
+#define BWD_TRACE(role, it, ev) \
+    do {                        \
+    } while (0)
+#endif
+
 constexpr int kBlock = 128;            // keys per item, queries per step
-constexpr int kThreads = 384;
-constexpr int kAllocWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kLoadWarp = 10;
-constexpr uint32_t kPdsRegs = 232;     // setmaxnreg: 128 x 232 + 128 x 168 + 128 x 104 = 384 x 168
-constexpr uint32_t kOtherRegs = 104;
+constexpr int kThreads = 512;
+constexpr int kDqWarp0 = 8;            // warps 8-11: dQ warpgroup
+constexpr int kAllocWarp = 12;
+constexpr int kMmaWarp = 13;
+constexpr int kLoadWarp = 14;
+// setmaxnreg split of the 512 x 128 registers: 2 x 128 x 144 (P/dS) +
+// 128 x 160 (dQ) + 128 x 64 (control) = 512 x 128
+constexpr uint32_t kPdsRegs = 144;
+constexpr uint32_t kDqRegs = 160;
+constexpr uint32_t kOtherRegs = 64;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBoxBytes = kBlock * 64 * 2;   // one 128-row x 64-column bf16 TMA box
 constexpr uint32_t kColX = 0, kColY = 128, kColDV = 256, kColDK = 384;
 
 enum WaitSite : int {
     kSiteKvEmpty = 11, kSiteKvFull, kSiteQEmpty, kSiteQFull, kSiteDoEmpty, kSiteDoFull, kSiteS, kSiteP, kSiteDp,
-    kSiteDs, kSiteDsFree, kSiteDq, kSiteYFree, kSiteAccDone, kSiteAccFree
+    kSiteDs, kSiteDsFree, kSiteDq, kSiteYFree, kSiteAccDone, kSiteAccFree, kSiteAlign, kSiteStage
 };
 
 struct alignas(64) Params {
@@ -98,12 +120,16 @@ struct Cfg {
     static constexpr int kKOff = 0;
     static constexpr int kVOff = kKOff + kTileBytes;
     static constexpr int kQOff = kVOff + kTileBytes;              // two slots
-    static constexpr int kDoOff = kQOff + 2 * kTileBytes;
+    static constexpr int kDoOff = kQOff + 2 * kTileBytes;         // one slot
     static constexpr int kDsOff = kDoOff + kTileBytes;            // 128 x 128 bf16
     static constexpr int kVecOff = kDsOff + kBlock * kBlock * 2;  // lse2[2][128], D[2][128]
-    static constexpr int kMiscOff = kVecOff + 4 * kBlock * 4;
-    static constexpr int kSmemBytes = kMiscOff + (int)sizeof(Misc) + 1024;
-    static_assert(kSmemBytes <= 232448, "shared memory");
+    static constexpr int kStageOff = kVecOff + 4 * kBlock * 4;    // dQ staging: 4 warps x 32 rows x 128 B
+    static constexpr int kMiscOff = kStageOff + 4 * 32 * 128;
+    static constexpr int kLayoutBytes = kMiscOff + (int)sizeof(Misc);
+    static_assert(kLayoutBytes <= 232448, "shared memory");
+    // the tiles need a 1024-byte aligned base: request room for the padding
+    // where it fits; the kernel checks that the padding it needs fits
+    static constexpr int kSmemBytes = kLayoutBytes + 1024 <= 232448 ? kLayoutBytes + 1024 : 232448;
 };
 
 // One work item: key block j of one (batch, kv head).
@@ -119,27 +145,48 @@ __device__ __forceinline__ int item_of_round(int r) {
     return r * G + ((r & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
 }
 
-// Items in increasing key block (under the causal mask the early key blocks
-// see the most query blocks: heaviest first), then (batch, kv head).
-__device__ __forceinline__ Item decode_item(int idx, const Params& p) {
-    Item it;
-    const int units = p.B * p.Hkv;
-    it.j = idx / units;
-    const int u = idx - it.j * units;
+// Work units: key blocks j and nk-1-j of one (batch, kv head), run one after
+// the other by one CTA.  Under the causal mask block j visits nk - j query
+// blocks, so every pair visits nk + 1 (the middle block of an odd count is
+// alone).  Units are numbered (batch, kv head)-major, so the CTAs running at
+// the same time share few heads and those heads' dQ accumulators stay in L2.
+__device__ __forceinline__ int num_work_units(const Params& p) {
+    const int nk = (p.N + kBlock - 1) / kBlock;
+    return ((nk + 1) / 2) * p.B * p.Hkv;
+}
+
+// Slot r of this CTA's sequence: element r % 2 of work unit
+// item_of_round(r / 2).  Returns 0 past the last unit, 2 for the missing
+// second element of a lone middle block, 1 with `it` filled in.
+__device__ __forceinline__ int next_item(int r, const Params& p, int total_wu, Item& it) {
+    const int w = item_of_round(r >> 1);
+    if (w >= total_wu) return 0;
+    const int nk = (p.N + kBlock - 1) / kBlock;
+    const int npairs = (nk + 1) / 2;
+    const int u = w / npairs;
+    const int pr = w - u * npairs;
+    const int j = (r & 1) ? nk - 1 - pr : pr;
+    if ((r & 1) && j == pr) return 2;
     it.b = u / p.Hkv;
     it.hk = u - it.b * p.Hkv;
-    it.nq = (p.N + kBlock - 1) / kBlock;
-    it.i0 = p.causal ? it.j : 0;
+    it.j = j;
+    it.nq = nk;
+    it.i0 = p.causal ? j : 0;
     it.niter = p.group * (it.nq - it.i0);
-    return it;
+    return 1;
 }
 
 // Iteration n of an item: query head h (of the group) and query block i.
+// The query blocks of a head are walked from a starting point that depends
+// on the key block, so that CTAs working on the same head at the same time
+// add into different rows of the dQ accumulator.
 __device__ __forceinline__ void iter_of(const Item& it, int n, const Params& p, int& h, int& i) {
     const int per = it.nq - it.i0;
     const int g = n / per;
     h = it.hk * p.group + g;
-    i = it.i0 + (n - g * per);
+    int t = n - g * per + (it.j * 7) % per;
+    if (t >= per) t -= per;
+    i = it.i0 + t;
 }
 
 #ifndef FA_SUSPEND_NS
@@ -172,8 +219,11 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, const P
 }
 
 // ---------------------------------------------------------------- producer
+// Two producer threads: `which` 0 loads K_j, V_j per item and Q_i with its
+// lse and D slices per iteration; `which` 1 loads dO_i.  Each runs ahead as
+// far as its own buffer slots allow.
 template <int D>
-__device__ void load_role(const Params& p, Misc& ms, uint8_t* smem, int total) {
+__device__ void load_role(const Params& p, Misc& ms, uint8_t* smem, int total, int which) {
     using C = Cfg<D>;
     const uint64_t pol_keep = policy_evict_last();
     const uint32_t s_k = smem_u32(smem + C::kKOff), s_v = smem_u32(smem + C::kVOff);
@@ -182,46 +232,57 @@ __device__ void load_role(const Params& p, Misc& ms, uint8_t* smem, int total) {
     uint32_t item_n = 0, ng = 0;
     bool ok = true;
     for (int r = 0; ok; ++r) {
-        const int idx = item_of_round(r);
-        if (idx >= total) break;
-        const Item it = decode_item(idx, p);
-        if (!(ok = wait_bar(smem_u32(&ms.kv_empty), (item_n & 1) ^ 1, p, ms, kSiteKvEmpty))) break;
-        mbar_arrive_expect_tx(smem_u32(&ms.kv_full), 2 * C::kTileBytes);
-        for (int bx = 0; bx < C::kBoxes; ++bx) {
-            tma_load_4d(s_k + bx * kBoxBytes, &p.tm_k, smem_u32(&ms.kv_full), bx * 64, it.j * kBlock, it.hk, it.b,
-                        pol_keep);
-            tma_load_4d(s_v + bx * kBoxBytes, &p.tm_v, smem_u32(&ms.kv_full), bx * 64, it.j * kBlock, it.hk, it.b,
-                        pol_keep);
+        Item it;
+        const int st = next_item(r, p, total, it);
+        if (st == 0) break;
+        if (st == 2) continue;
+        if (which == 0) {
+            if (!(ok = wait_bar(smem_u32(&ms.kv_empty), (item_n & 1) ^ 1, p, ms, kSiteKvEmpty))) break;
+            mbar_arrive_expect_tx(smem_u32(&ms.kv_full), 2 * C::kTileBytes);
+            for (int bx = 0; bx < C::kBoxes; ++bx) {
+                tma_load_4d(s_k + bx * kBoxBytes, &p.tm_k, smem_u32(&ms.kv_full), bx * 64, it.j * kBlock, it.hk, it.b,
+                            pol_keep);
+                tma_load_4d(s_v + bx * kBoxBytes, &p.tm_v, smem_u32(&ms.kv_full), bx * 64, it.j * kBlock, it.hk, it.b,
+                            pol_keep);
+            }
+            ++item_n;
         }
-        ++item_n;
         for (int n = 0; n < it.niter && ok; ++n, ++ng) {
             int h, i;
             iter_of(it, n, p, h, i);
             const uint32_t slot = ng & 1;
-            // Q_i with its lse and D slices
-            if (!(ok = wait_bar(smem_u32(&ms.q_empty[slot]), ((ng >> 1) & 1) ^ 1, p, ms, kSiteQEmpty))) break;
-            const uint32_t qbar = smem_u32(&ms.q_full[slot]);
-            mbar_arrive_expect_tx(qbar, C::kTileBytes + 2 * kBlock * 4);
-            for (int bx = 0; bx < C::kBoxes; ++bx)
-                tma_load_4d(s_q + slot * C::kTileBytes + bx * kBoxBytes, &p.tm_q, qbar, bx * 64, i * kBlock, h, it.b,
-                            pol_keep);
-            const size_t row0 = (static_cast<size_t>(it.b) * p.Hq + h) * p.Npad + static_cast<size_t>(i) * kBlock;
-            bulk_load(s_vec + slot * kBlock * 4, p.lse2 + row0, kBlock * 4, qbar);
-            bulk_load(s_vec + (2 + slot) * kBlock * 4, p.Dvec + row0, kBlock * 4, qbar);
-            // dO_i
-            if (!(ok = wait_bar(smem_u32(&ms.do_empty), (ng & 1) ^ 1, p, ms, kSiteDoEmpty))) break;
-            const uint32_t dbar = smem_u32(&ms.do_full);
-            mbar_arrive_expect_tx(dbar, C::kTileBytes);
-            for (int bx = 0; bx < C::kBoxes; ++bx)
-                tma_load_4d(s_do + bx * kBoxBytes, &p.tm_do, dbar, bx * 64, i * kBlock, h, it.b, pol_keep);
+            if (which == 0) {
+                // Q_i with its lse and D slices
+                BWD_TRACE(3, ng, 0);
+                if (!(ok = wait_bar(smem_u32(&ms.q_empty[slot]), ((ng >> 1) & 1) ^ 1, p, ms, kSiteQEmpty))) break;
+                BWD_TRACE(3, ng, 1);
+                const uint32_t qbar = smem_u32(&ms.q_full[slot]);
+                mbar_arrive_expect_tx(qbar, C::kTileBytes + 2 * kBlock * 4);
+                for (int bx = 0; bx < C::kBoxes; ++bx)
+                    tma_load_4d(s_q + slot * C::kTileBytes + bx * kBoxBytes, &p.tm_q, qbar, bx * 64, i * kBlock, h, it.b,
+                                pol_keep);
+                const size_t row0 = (static_cast<size_t>(it.b) * p.Hq + h) * p.Npad + static_cast<size_t>(i) * kBlock;
+                bulk_load(s_vec + slot * kBlock * 4, p.lse2 + row0, kBlock * 4, qbar);
+                bulk_load(s_vec + (2 + slot) * kBlock * 4, p.Dvec + row0, kBlock * 4, qbar);
+            } else {
+                // dO_i
+                if (!(ok = wait_bar(smem_u32(&ms.do_empty), (ng & 1) ^ 1, p, ms, kSiteDoEmpty))) break;
+                BWD_TRACE(3, ng, 2);
+                const uint32_t dbar = smem_u32(&ms.do_full);
+                mbar_arrive_expect_tx(dbar, C::kTileBytes);
+                for (int bx = 0; bx < C::kBoxes; ++bx)
+                    tma_load_4d(s_do + bx * kBoxBytes, &p.tm_do, dbar, bx * 64, i * kBlock, h, it.b, pol_keep);
+            }
         }
     }
     if (!ok) {
-        // let the copies already issued land before the CTA goes away
-        if (item_n > 0) drain_bar(smem_u32(&ms.kv_full), (item_n - 1) & 1, p);
-        for (uint32_t g = (ng > 2 ? ng - 2 : 0); g <= ng; ++g) {
-            drain_bar(smem_u32(&ms.q_full[g & 1]), (g >> 1) & 1, p);
-            drain_bar(smem_u32(&ms.do_full), g & 1, p);
+        // let the copies already issued land before the CTA goes away: the
+        // last item's K/V and the last two slots' loads
+        if (which == 0 && item_n > 0) drain_bar(smem_u32(&ms.kv_full), (item_n - 1) & 1, p);
+        if (which == 0) {
+            for (uint32_t g = (ng > 2 ? ng - 2 : 0); g < ng; ++g) drain_bar(smem_u32(&ms.q_full[g & 1]), (g >> 1) & 1, p);
+        } else if (ng > 0) {
+            drain_bar(smem_u32(&ms.do_full), (ng - 1) & 1, p);
         }
     }
 }
@@ -244,12 +305,12 @@ __device__ void mma_role(const Params& p, Misc& ms, uint8_t* smem, uint32_t tmem
     const uint64_t dk_k = smem_desc_sw128(smem_u32(smem + C::kKOff), 16, 1024);
     const uint64_t dv_k = smem_desc_sw128(smem_u32(smem + C::kVOff), 16, 1024);
     const uint64_t dq_k0 = smem_desc_sw128(smem_u32(smem + C::kQOff), 16, 1024);
-    const uint64_t ddo_k = smem_desc_sw128(smem_u32(smem + C::kDoOff), 16, 1024);
+    const uint64_t ddo_k0 = smem_desc_sw128(smem_u32(smem + C::kDoOff), 16, 1024);
     const uint64_t dds_k = smem_desc_sw128(smem_u32(smem + C::kDsOff), 16, 1024);
     // MN-major views (rows are the reduction dimension)
     const uint64_t dk_mn = smem_desc_sw128(smem_u32(smem + C::kKOff), kBoxBytes, 1024);
     const uint64_t dq_mn0 = smem_desc_sw128(smem_u32(smem + C::kQOff), kBoxBytes, 1024);
-    const uint64_t ddo_mn = smem_desc_sw128(smem_u32(smem + C::kDoOff), kBoxBytes, 1024);
+    const uint64_t ddo_mn0 = smem_desc_sw128(smem_u32(smem + C::kDoOff), kBoxBytes, 1024);
     const uint64_t dds_mn = smem_desc_sw128(smem_u32(smem + C::kDsOff), kBoxBytes, 1024);
     constexpr uint32_t id_dv = idesc_bf16_f32(kBlock, D, true);          // P^T (TMEM) x dO (MN)
     constexpr uint32_t id_dk = idesc_bf16_f32(kBlock, D, true);          // dS^T (K-major) x Q (MN)
@@ -257,9 +318,10 @@ __device__ void mma_role(const Params& p, Misc& ms, uint8_t* smem, uint32_t tmem
     uint32_t item_n = 0, ng = 0;
     bool ok = true;
     for (int r = 0; ok; ++r) {
-        const int idx = item_of_round(r);
-        if (idx >= total) break;
-        const Item it = decode_item(idx, p);
+        Item it;
+        const int st = next_item(r, p, total, it);
+        if (st == 0) break;
+        if (st == 2) continue;
         if (!(ok = wait_bar(smem_u32(&ms.kv_full), item_n & 1, p, ms, kSiteKvFull))) break;
         tc_fence_after();
         for (int n = 0; n < it.niter && ok; ++n, ++ng) {
@@ -270,18 +332,32 @@ __device__ void mma_role(const Params& p, Misc& ms, uint8_t* smem, uint32_t tmem
                 mma_qk<D>(tmem + kColX, dk_k, dq_k0 + slot * kTileStep);
                 umma_commit(smem_u32(&ms.s_full));
             }
-            // dV_j += P^T dO_i, once P^T is in TMEM
-            if (!(ok = wait_bar(smem_u32(&ms.p_full), ng & 1, p, ms, kSiteP))) break;
-            if (n == 0 && !(ok = wait_bar(smem_u32(&ms.acc_free), (item_n & 1) ^ 1, p, ms, kSiteAccFree))) break;
+            // dP^T = V_j dO_i^T (once the previous dQ share has left Y) and
+            // dV_j += P^T dO_i (once P^T is in TMEM), whichever is ready first
+            BWD_TRACE(0, ng, 0);
             if (!(ok = wait_bar(smem_u32(&ms.do_full), ng & 1, p, ms, kSiteDoFull))) break;
+            BWD_TRACE(0, ng, 1);
+            const uint64_t ddo_k = ddo_k0, ddo_mn = ddo_mn0;
+            bool dp_issued = false;
+            if (mbar_try_wait(smem_u32(&ms.y_free), (ng & 1) ^ 1)) {
+                tc_fence_after();
+                mma_qk<D>(tmem + kColY, dv_k, ddo_k);
+                umma_commit(smem_u32(&ms.dp_full));
+                dp_issued = true;
+            }
+            if (!(ok = wait_bar(smem_u32(&ms.p_full), ng & 1, p, ms, kSiteP))) break;
+            BWD_TRACE(0, ng, 2);
+            if (n == 0 && !(ok = wait_bar(smem_u32(&ms.acc_free), (item_n & 1) ^ 1, p, ms, kSiteAccFree))) break;
             tc_fence_after();
             umma_ts_kv128_x8(tmem + kColDV, tmem + kColX, ddo_mn, id_dv, n > 0 ? 1u : 0u);
-            // dP^T = V_j dO_i^T, once the previous dQ share has left Y
-            if (!(ok = wait_bar(smem_u32(&ms.y_free), (ng & 1) ^ 1, p, ms, kSiteYFree))) break;
-            tc_fence_after();
-            mma_qk<D>(tmem + kColY, dv_k, ddo_k);
-            umma_commit(smem_u32(&ms.dp_full));
+            if (!dp_issued) {
+                if (!(ok = wait_bar(smem_u32(&ms.y_free), (ng & 1) ^ 1, p, ms, kSiteYFree))) break;
+                tc_fence_after();
+                mma_qk<D>(tmem + kColY, dv_k, ddo_k);
+                umma_commit(smem_u32(&ms.dp_full));
+            }
             umma_commit(smem_u32(&ms.do_empty));
+            BWD_TRACE(0, ng, 3);
             // S^T of the next block (X is free once dV has read P^T: in order)
             if (n + 1 < it.niter) {
                 const uint32_t ns = (ng + 1) & 1;
@@ -291,13 +367,18 @@ __device__ void mma_role(const Params& p, Misc& ms, uint8_t* smem, uint32_t tmem
                 umma_commit(smem_u32(&ms.s_full));
             }
             // dK_j += dS^T Q_i and dQ_i share = dS K_j, once dS is in shared memory
+            BWD_TRACE(0, ng, 4);
             if (!(ok = wait_bar(smem_u32(&ms.ds_full), ng & 1, p, ms, kSiteDs))) break;
+            BWD_TRACE(0, ng, 5);
             tc_fence_after();
-            umma_ss_kA_mnB_k128_x8(tmem + kColDK, dds_k, dq_mn0 + slot * kTileStep, id_dk, n > 0 ? 1u : 0u);
+            // dQ first: the dQ warpgroup can start reading Y while dK runs
             umma_ss_mnA_mnB_k128_x8(tmem + kColY, dds_mn, dk_mn, id_dq);
             umma_commit(smem_u32(&ms.dq_full));
+            umma_ss_kA_mnB_k128_x8(tmem + kColDK, dds_k, dq_mn0 + slot * kTileStep, id_dk, n > 0 ? 1u : 0u);
             umma_commit(smem_u32(&ms.ds_free));
             umma_commit(smem_u32(&ms.q_empty[slot]));
+            BWD_TRACE(0, ng, 6);
+            if (dp_issued) BWD_TRACE(0, ng, 7);
             if (n == it.niter - 1) {
                 umma_commit(smem_u32(&ms.acc_done));
                 umma_commit(smem_u32(&ms.kv_empty));
@@ -320,132 +401,171 @@ __device__ __forceinline__ uint32_t sw128_chunk(int r, int c16) {
 template <int D>
 __device__ void pds_role(const Params& p, Misc& ms, uint8_t* smem, uint32_t tmem, int warp, int lane, int total) {
     using C = Cfg<D>;
-    const int r = warp * 32 + lane;                     // key row inside the block
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const int g = warp / 4;                              // warpgroup: query columns 64g .. 64g+63
+    const int wq = warp % 4;                             // TMEM lane quarter
+    const int r = wq * 32 + lane;                        // key row inside the block
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tx = tmem + lane_off + kColX, ty = tmem + lane_off + kColY;
-    const float* vec = reinterpret_cast<const float*>(smem + C::kVecOff);
-    uint8_t* ds_tile = smem + C::kDsOff;
+    const uint32_t vec = smem_u32(smem + C::kVecOff);
+    const uint32_t ds_tile = smem_u32(smem + C::kDsOff);
     const float sl2 = p.scale_log2;
     uint32_t ng = 0;
     bool ok = true;
     for (int rr = 0; ok; ++rr) {
-        const int idx = item_of_round(rr);
-        if (idx >= total) break;
-        const Item it = decode_item(idx, p);
+        Item it;
+        const int st = next_item(rr, p, total, it);
+        if (st == 0) break;
+        if (st == 2) continue;
         const bool key_valid = it.j * kBlock + r < p.N;
         for (int n = 0; n < it.niter; ++n, ++ng) {
             int h, i;
             iter_of(it, n, p, h, i);
             const uint32_t slot = ng & 1;
-            const float* lse2 = vec + slot * kBlock;
-            const float* dvec = vec + (2 + slot) * kBlock;
+            const uint32_t lse2 = vec + (slot * kBlock + 64 * g) * 4;
+            const uint32_t dvec = vec + ((2 + slot) * kBlock + 64 * g) * 4;
+            if (r == 0 && g == 0) BWD_TRACE(1, ng, 0);
             ok = wait_bar(smem_u32(&ms.s_full), ng & 1, p, ms, kSiteS);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
-            uint32_t s[128];
-            tmem_ld128_sync(tx, s);
-            // P^T = exp2(S^T * scale * log2 e - lse * log2 e); key r vs query c
-            const bool diag = p.causal && i == it.j;
-#pragma unroll
-            for (int c = 0; c < 128; c += 4) {
-                const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c);
-                float e0 = ex2_approx(fmaf(__uint_as_float(s[c]), sl2, -l4.x));
-                float e1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), sl2, -l4.y));
-                float e2 = ex2_approx(fmaf(__uint_as_float(s[c + 2]), sl2, -l4.z));
-                float e3 = ex2_approx(fmaf(__uint_as_float(s[c + 3]), sl2, -l4.w));
-                if (diag) {        // query c sees key r only if r <= c
-                    if (c < r) e0 = 0.f;
-                    if (c + 1 < r) e1 = 0.f;
-                    if (c + 2 < r) e2 = 0.f;
-                    if (c + 3 < r) e3 = 0.f;
-                }
-                if (!key_valid) e0 = e1 = e2 = e3 = 0.f;
-                s[c] = __float_as_uint(e0);
-                s[c + 1] = __float_as_uint(e1);
-                s[c + 2] = __float_as_uint(e2);
-                s[c + 3] = __float_as_uint(e3);
+            uint32_t s[64];
+            {
+                uint32_t (&sa)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
+                uint32_t (&sb)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32]);
+                tmem_ld64_sync(tx + 64 * g, sa, sb);
             }
+            // P^T = exp2(S^T * scale * log2 e - lse * log2 e) for key r and query
+            // 64g + c; masked: query < key on the diagonal block, and every
+            // query of a key row past the sequence end
+            const int cmin = !key_valid ? 64 : ((p.causal && i == it.j) ? r - 64 * g : 0);
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
+            for (int c0 = 0; c0 < 64; c0 += 32) {
+                float4 l4[8];
+#pragma unroll
+                for (int t = 0; t < 8; ++t) l4[t] = lds_f4(lse2 + (c0 + 4 * t) * 4);
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    const int c = c0 + 4 * t;
+                    const float e0 = ex2_approx(fmaf(__uint_as_float(s[c]), sl2, -l4[t].x));
+                    const float e1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), sl2, -l4[t].y));
+                    const float e2 = ex2_approx(fmaf(__uint_as_float(s[c + 2]), sl2, -l4[t].z));
+                    const float e3 = ex2_approx(fmaf(__uint_as_float(s[c + 3]), sl2, -l4[t].w));
+                    s[c] = __float_as_uint(c < cmin ? 0.f : e0);
+                    s[c + 1] = __float_as_uint(c + 1 < cmin ? 0.f : e1);
+                    s[c + 2] = __float_as_uint(c + 2 < cmin ? 0.f : e2);
+                    s[c + 3] = __float_as_uint(c + 3 < cmin ? 0.f : e3);
+                }
+            }
+            {
                 uint32_t pk[32];
 #pragma unroll
-                for (int t = 0; t < 32; ++t)
-                    pk[t] = pack_bf16x2(__uint_as_float(s[64 * hf + 2 * t]), __uint_as_float(s[64 * hf + 2 * t + 1]));
-                tmem_st32(tx + 32 * hf, pk);
+                for (int t = 0; t < 32; ++t) pk[t] = pack_bf16x2(__uint_as_float(s[2 * t]), __uint_as_float(s[2 * t + 1]));
+                tmem_st32(tx + 32 * g, pk);
             }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&ms.p_full));
-            // dS^T = P^T (dP^T - D), into the shared dS tile
+            if (r == 0 && g == 0) BWD_TRACE(1, ng, 3);
+            // dS^T = P^T (dP^T - D), into box g of the shared dS tile
             ok = wait_bar(smem_u32(&ms.dp_full), ng & 1, p, ms, kSiteDp);
+            if (r == 0 && g == 0) BWD_TRACE(1, ng, 4);
             ok = ok && wait_bar(smem_u32(&ms.ds_free), (ng & 1) ^ 1, p, ms, kSiteDsFree);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            if (r == 0 && g == 0) BWD_TRACE(1, ng, 5);
             tc_fence_after();
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
+            for (int q4 = 0; q4 < 2; ++q4) {
                 uint32_t dp[32];
-                tmem_ld32_sync(ty + 32 * q4, dp);
-                uint32_t pk[16];
+                tmem_ld32_sync(ty + 64 * g + 32 * q4, dp);
 #pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    const int c = 32 * q4 + 2 * t;
-                    const float2 d2 = *reinterpret_cast<const float2*>(dvec + c);
-                    const float a = __uint_as_float(s[c]) * (__uint_as_float(dp[2 * t]) - d2.x);
-                    const float b = __uint_as_float(s[c + 1]) * (__uint_as_float(dp[2 * t + 1]) - d2.y);
-                    pk[t] = pack_bf16x2(a, b);
+                for (int hq = 0; hq < 2; ++hq) {
+                    float4 d4[4];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) d4[t] = lds_f4(dvec + (32 * q4 + 16 * hq + 4 * t) * 4);
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const int c = 32 * q4 + 16 * hq + 4 * t;
+                        const int e = 16 * hq + 4 * t;
+                        pk[2 * t] = pack_bf16x2(__uint_as_float(s[c]) * (__uint_as_float(dp[e]) - d4[t].x),
+                                                __uint_as_float(s[c + 1]) * (__uint_as_float(dp[e + 1]) - d4[t].y));
+                        pk[2 * t + 1] = pack_bf16x2(__uint_as_float(s[c + 2]) * (__uint_as_float(dp[e + 2]) - d4[t].z),
+                                                    __uint_as_float(s[c + 3]) * (__uint_as_float(dp[e + 3]) - d4[t].w));
+                    }
+                    const int c16 = 8 * g + 4 * q4 + 2 * hq;
+                    sts_u4(ds_tile + sw128_chunk(r, c16), pk[0], pk[1], pk[2], pk[3]);
+                    sts_u4(ds_tile + sw128_chunk(r, c16 + 1), pk[4], pk[5], pk[6], pk[7]);
                 }
-#pragma unroll
-                for (int t = 0; t < 4; ++t)
-                    *reinterpret_cast<uint4*>(ds_tile + sw128_chunk(r, 4 * q4 + t)) =
-                        make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
             }
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&ms.ds_full));
+            if (r == 0 && g == 0) BWD_TRACE(1, ng, 6);
         }
     }
 }
 
 // ------------------------------------------------------- dQ warpgroup
 template <int D>
-__device__ void dq_role(const Params& p, Misc& ms, uint32_t tmem, int wq, int lane, int total) {
+__device__ void dq_role(const Params& p, Misc& ms, uint8_t* smem, uint32_t tmem, int wq, int lane, int total) {
+    using C = Cfg<D>;
     const int r = wq * 32 + lane;                       // query row (dQ) or key row (dK, dV)
+    // this warp's 32 x 32 fp32 staging tile: 128-byte rows, 16-byte chunks
+    // XOR-swizzled by row; rows go in by thread and come out by row
+    const uint32_t stage = smem_u32(smem + C::kStageOff) + wq * 32 * 128;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t ty = tmem + lane_off + kColY;
     uint32_t item_n = 0, ng = 0;
     bool ok = true;
     for (int rr = 0; ok; ++rr) {
-        const int idx = item_of_round(rr);
-        if (idx >= total) break;
-        const Item it = decode_item(idx, p);
+        Item it;
+        const int st = next_item(rr, p, total, it);
+        if (st == 0) break;
+        if (st == 2) continue;
         for (int n = 0; n < it.niter; ++n, ++ng) {
             int h, i;
             iter_of(it, n, p, h, i);
+            if (r == 0) BWD_TRACE(2, ng, 0);
             ok = wait_bar(smem_u32(&ms.dq_full), ng & 1, p, ms, kSiteDq);
+            if (r == 0) BWD_TRACE(2, ng, 1);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
+            // row r of the block's dQ share: into registers first, so that Y can
+            // take the next dP before the reductions go out
             float* dst = p.dq_acc + ((static_cast<size_t>(it.b) * p.Hq + h) * p.Npad + static_cast<size_t>(i) * kBlock + r) * D;
-            uint32_t a[32], b[32];
-#pragma unroll
-            for (int c = 0; c < D / 64; ++c) {
-                tmem_ld64_sync(ty + 64 * c, a, b);
-                if (c == D / 64 - 1) {
-                    // Y may take the next dP once every lane has its values
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_u32(&ms.y_free));
-                }
-#pragma unroll
-                for (int t = 0; t < 8; ++t)
-                    red_add_v4(dst + 64 * c + 4 * t, __uint_as_float(a[4 * t]), __uint_as_float(a[4 * t + 1]),
-                               __uint_as_float(a[4 * t + 2]), __uint_as_float(a[4 * t + 3]));
-#pragma unroll
-                for (int t = 0; t < 8; ++t)
-                    red_add_v4(dst + 64 * c + 32 + 4 * t, __uint_as_float(b[4 * t]), __uint_as_float(b[4 * t + 1]),
-                               __uint_as_float(b[4 * t + 2]), __uint_as_float(b[4 * t + 3]));
+            uint32_t v[D];
+            if constexpr (D == 128) {
+                tmem_ld128_sync(ty, v);
+            } else {
+                uint32_t (&va)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
+                uint32_t (&vb)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
+                tmem_ld64_sync(ty, va, vb);
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ms.y_free));
+            if (r == 0) BWD_TRACE(2, ng, 2);
+            // 32 columns at a time through the staging tile: each reduction
+            // instruction of the warp then covers 4 rows x 128 bytes
+            float* dst0 = dst - static_cast<size_t>(lane) * D;          // row wq*32 of the share
+            const int rsub = lane >> 3, k = lane & 7;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+#pragma unroll
+                for (int t = 0; t < 8; ++t)
+                    sts_u4(stage + lane * 128 + ((t ^ (lane & 7)) << 4), v[32 * c + 4 * t], v[32 * c + 4 * t + 1],
+                           v[32 * c + 4 * t + 2], v[32 * c + 4 * t + 3]);
+                __syncwarp();
+#pragma unroll
+                for (int rr = 0; rr < 8; ++rr) {
+                    const int row = 4 * rr + rsub;
+                    const float4 x = lds_f4(stage + row * 128 + ((k ^ (row & 7)) << 4));
+                    red_add_v4(dst0 + static_cast<size_t>(row) * D + 32 * c + 4 * k, x.x, x.y, x.z, x.w);
+                }
+                __syncwarp();
+            }
+            if (r == 0) BWD_TRACE(2, ng, 3);
         }
         if (!ok) break;
         // dK_j, dV_j of the item: TMEM -> bf16 -> HBM
@@ -487,6 +607,14 @@ __global__ void __launch_bounds__(kThreads, 1) fa_bwd_kernel(const __grid_consta
     using C = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    if (smem - smem_raw > C::kSmemBytes - C::kLayoutBytes) {
+        // the launch's shared memory cannot hold the aligned layout: report, do nothing
+        if (threadIdx.x == 0 && atomicCAS(p.status, 0, FA_ERR_LAUNCH) == 0) {
+            p.status[1] = kSiteAlign;
+            p.status[2] = blockIdx.x;
+        }
+        return;
+    }
     Misc& ms = *reinterpret_cast<Misc*>(smem + C::kMiscOff);
     const int tid = threadIdx.x;
     const int warp = tid / 32, lane = tid % 32;
@@ -500,9 +628,9 @@ __global__ void __launch_bounds__(kThreads, 1) fa_bwd_kernel(const __grid_consta
         mbar_init(smem_u32(&ms.do_full), 1);
         mbar_init(smem_u32(&ms.do_empty), 1);
         mbar_init(smem_u32(&ms.s_full), 1);
-        mbar_init(smem_u32(&ms.p_full), 4);       // one arrival per warp of the P/dS warpgroup
+        mbar_init(smem_u32(&ms.p_full), 8);       // one arrival per warp of the two P/dS warpgroups
         mbar_init(smem_u32(&ms.dp_full), 1);
-        mbar_init(smem_u32(&ms.ds_full), 4);
+        mbar_init(smem_u32(&ms.ds_full), 8);
         mbar_init(smem_u32(&ms.ds_free), 1);
         mbar_init(smem_u32(&ms.dq_full), 1);
         mbar_init(smem_u32(&ms.y_free), 4);       // one arrival per warp of the dQ warpgroup
@@ -526,20 +654,24 @@ __global__ void __launch_bounds__(kThreads, 1) fa_bwd_kernel(const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ms.tmem_base;
-    const int total = ((p.N + kBlock - 1) / kBlock) * p.B * p.Hkv;
+    const int total = num_work_units(p);
 
-    if (warp < 4) {
+    if (warp < kDqWarp0) {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kPdsRegs));
         pds_role<D>(p, ms, smem, tmem, warp, lane, total);
-    } else if (warp < 8) {
-        dq_role<D>(p, ms, tmem, warp - 4, lane, total);
+    } else if (warp < kDqWarp0 + 4) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kDqRegs));
+        dq_role<D>(p, ms, smem, tmem, warp - kDqWarp0, lane, total);
     } else {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
         if (warp == kMmaWarp) {
             if (lane == 0) mma_role<D>(p, ms, smem, tmem, total);
             __syncwarp();
         } else if (warp == kLoadWarp) {
-            if (lane == 0) load_role<D>(p, ms, smem, total);
+            if (lane == 0) load_role<D>(p, ms, smem, total, 0);
+            __syncwarp();
+        } else if (warp == kLoadWarp + 1) {
+            if (lane == 0) load_role<D>(p, ms, smem, total, 1);
             __syncwarp();
         }
     }
@@ -630,6 +762,13 @@ static bool aligned(const void* ptr, uintptr_t a) { return (reinterpret_cast<uin
 
 using namespace fa_sm100;
 
+#ifdef FA_TRACE
+extern "C" int fa_bwd_trace_set(void* ptr) {
+    unsigned long long* q = static_cast<unsigned long long*>(ptr);
+    return cudaMemcpyToSymbol(fa_sm100::bwd::g_btrace, &q, sizeof(q)) == cudaSuccess ? 0 : -1;
+}
+#endif
+
 extern "C" size_t fa_bwd_workspace_bytes(int B, int Hq, int N, int d) {
     if (B < 0 || Hq < 1 || N < 0 || (d != 64 && d != 128)) return 0;
     return bwd::workspace_bytes(B, Hq, N, d);
@@ -696,8 +835,8 @@ extern "C" int fa_bwd(const void* q, const void* k, const void* v, const void* o
     P.timeout_ns = 2000000000ull;
 
     const unsigned prep_grid = static_cast<unsigned>((rows_pad + 7) / 8);
-    const long long items = (long long)B * Hkv * ((N + kBlock - 1) / kBlock);
-    const int grid = (int)std::min<long long>(items, ds->num_sms);
+    const long long units = (long long)B * Hkv * (((N + kBlock - 1) / kBlock + 1) / 2);
+    const int grid = (int)std::min<long long>(units, ds->num_sms);
     const long long total4 = (long long)B * Hq * N * d / 4;
     const unsigned post_grid = static_cast<unsigned>((total4 + 255) / 256);
     if (d == 64) {
