@@ -2,6 +2,7 @@
 """Benchmark of the exact attention forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config c3] [--impl ours|reference]
+                    [--pass fwd|bwd]
 
 A step is one fa_fwd call over the whole workload (default: causal B=1, H=32,
 N=16384, d=128, the configuration the throughput target is quoted on).  The
@@ -15,6 +16,11 @@ weak; the timing is the maximum over ranks.
 Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle
 on the host cores instead (rank 0 only), each step a bounded sample of the same
 workload's query rows.
+
+``--pass bwd`` times the backward pass instead (fa_bwd: dQ, dK, dV from the
+forward's O and logsumexp and a seeded upstream gradient), counted as 2.5x the
+forward's FLOPs (five matrix products per block instead of two); its CPU
+baseline is the fp64 gradient oracle on one (batch, kv head) unit.
 """
 from __future__ import annotations
 
@@ -33,6 +39,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "attention fwd TFLOP/s (bf16) and % of B200 dense BF16 tensor peak"
+METRIC_BWD = "attention bwd TFLOP/s (bf16; 2.5x the forward's FLOPs) and % of B200 dense BF16 tensor peak"
+BWD_FLOP_FACTOR = 2.5
 UNIT = "TFLOP/s"
 FALLBACK_PEAK_TFLOPS = 1590.0
 
@@ -48,6 +56,7 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU time budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd")
     return ap.parse_args()
 
 
@@ -98,24 +107,28 @@ def load_hbm_peak():
         return 6650.0, "fallback"
 
 
-def source_sha():
+def source_sha(kernel="fwd"):
+    """sha256[:16] of the source files of the forward (fa_fwd.cu) or backward
+    (fa_bwd.cu) kernel, with the shared PTX wrappers."""
     h = hashlib.sha256()
-    for rel in ("exact_tiled_attention_32_b200/csrc/fa_fwd.cu", "exact_tiled_attention_32_b200/csrc/sm100_ptx.cuh"):
+    main = "fa_fwd.cu" if kernel == "fwd" else "fa_bwd.cu"
+    for rel in (f"exact_tiled_attention_32_b200/csrc/{main}", "exact_tiled_attention_32_b200/csrc/sm100_ptx.cuh"):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(config_name):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel source; else None."""
+def profiled_traffic(key, kernel="fwd"):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary (row `key`), if it was taken on the current kernel source; else
+    None."""
     path = os.path.join(ROOT, "profiles", "fa_fwd_kernel_traffic.md")
     if not os.path.exists(path):
         return None
-    sha = source_sha()
+    sha = source_sha(kernel)
     for line in open(path):
-        m = re.match(r"\|\s*(\w+)\s*\|\s*([0-9a-f]{16})\s*\|\s*([0-9.eE+]+)\s*\|", line)
-        if m and m.group(1) == config_name and m.group(2) == sha:
+        m = re.match(r"\|\s*([\w-]+)\s*\|\s*([0-9a-f]{16})\s*\|\s*([0-9.eE+]+)\s*\|", line)
+        if m and m.group(1) == key and m.group(2) == sha:
             return float(m.group(3))
     return None
 
@@ -239,9 +252,60 @@ def time_oracle(w, seconds, seed=0):
                       f"{dt:.1f} s on the host cores"}
 
 
+def bwd_unit_flops(w):
+    """Backward FLOPs of one (batch, kv head) unit: 2.5x the forward's."""
+    return BWD_FLOP_FACTOR * w.flops() / (w.B * w.Hkv)
+
+
+def time_oracle_bwd(w, do, seconds):
+    """The gradient oracle on whole (batch, kv head) units until ``seconds``
+    have passed (at least one unit)."""
+    import oracle
+    units = 0
+    t0 = time.perf_counter()
+    while True:
+        oracle.attention_bwd(w.q, w.k, w.v, do, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal,
+                             units=[units % (w.B * w.Hkv)])
+        units += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": units * bwd_unit_flops(w) / dt / 1e12, "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": f"{units} whole (batch, kv head) units of the workload's gradients "
+                                        f"(fp64, materialised score rows), {dt:.1f} s on the host cores"}
+
+
+def bwd_dout(w):
+    """The seeded upstream gradient of the backward bench (bf16 N(0,1))."""
+    from exact_tiled_attention_32_b200 import synthetic as syn
+    return syn.Stream(w.seed + 77).normal_bf16(w.q_shape())
+
+
 def run_reference(args, rank):
     """--impl reference: the oracle timed on the host cores (rank 0 only)."""
     if rank != 0:
+        return
+    if getattr(args, "pass_", "fwd") == "bwd":
+        from exact_tiled_attention_32_b200 import synthetic as syn
+        import oracle
+        w = syn.config(args.config).draw()
+        do = bwd_dout(w)
+        t0 = time.perf_counter()
+        for k in range(args.steps):
+            oracle.attention_bwd(w.q, w.k, w.v, do, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal,
+                                 units=[k % (w.B * w.Hkv)])
+        dt = time.perf_counter() - t0
+        value = args.steps * bwd_unit_flops(w) / dt / 1e12
+        line = {
+            "impl": "reference", "metric": METRIC_BWD, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / max(args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(w, {"pass": "bwd", "step": "one whole (batch, kv head) unit per step"}),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": f"{args.steps} (batch, kv head) units"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
         return
     import numpy as np
     import oracle
@@ -318,6 +382,10 @@ def main():
     w = syn.config(args.config)
     w.seed += rank              # independent problem per rank
     w.draw()
+    if args.pass_ == "bwd":
+        if w.packed or w.chunk:
+            raise SystemExit("--pass bwd runs on dense workloads (c1, c2nc, c2c, c3, c4)")
+        return run_bwd(args, w, rank, world, dev)
     q = torch.from_numpy(w.q.view(np.int16)).view(torch.bfloat16).to(dev)
     k = torch.from_numpy(w.k.view(np.int16)).view(torch.bfloat16).to(dev)
     v = torch.from_numpy(w.v.view(np.int16)).view(torch.bfloat16).to(dev)
@@ -464,6 +532,127 @@ def main():
         "e2e": e2e,
         "gpu_launches": args.steps * launches_per_step,
         "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_bwd(args, w, rank, world, dev):
+    """The backward pass (fa_bwd) timed like the forward: CUDA events over K
+    steps, each step one fa_bwd call (three kernel launches) on resident
+    inputs."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from exact_tiled_attention_32_b200 import binding as fa
+
+    def dev_bits(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    do_bits = bwd_dout(w)
+    q, k, v, do = dev_bits(w.q), dev_bits(w.k), dev_bits(w.v), dev_bits(do_bits)
+    o, lse = fa.attention_forward(q, k, v, causal=w.causal, scale=w.scale)
+    ws_bytes = fa.fa_bwd_workspace_bytes(w.B, w.Hq, w.N, w.d)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    stream = torch.cuda.current_stream(dev)
+    flops = BWD_FLOP_FACTOR * w.flops()
+
+    def step():
+        rc = fa.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal, ws,
+                       ws_bytes, stream)
+        if rc != 0:
+            raise fa.FAError(rc, "fa_bwd")
+
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.3)
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    t_host0 = time.time()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    ev1.synchronize()
+    torch.cuda.synchronize(dev)
+    t_host1 = time.time()
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+    sampler.stop()
+    status = fa.fa_get_device_status(stream)
+    if status != 0:
+        raise fa.FAError(status, "device status after the timed region")
+    ms_per_step = ms / max(args.steps, 1)
+    value = whole_job_tflops(flops, world, args.steps, ms)
+    achieved = flops / (ms_per_step / 1e3) / 1e12
+    peak, peak_sustained, peak_kind = load_peak()
+
+    e2e = None
+    if args.e2e_steps > 0:
+        host = [torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()
+                for a in (w.q, w.k, w.v, do_bits)]
+        oh = o.cpu().pin_memory()
+        lh = lse.cpu().pin_memory()
+        outs = [torch.empty(t.shape, dtype=torch.bfloat16).pin_memory() for t in (dq, dk, dv)]
+
+        def e2e_step():
+            qd, kd, vd, dod = (t.to(dev, non_blocking=True) for t in host)
+            od = oh.to(dev, non_blocking=True)
+            ld = lh.to(dev, non_blocking=True)
+            grads = fa.attention_backward(qd, kd, vd, od, ld, dod, causal=w.causal, scale=w.scale, workspace=ws)
+            for dst, src in zip(outs, grads):
+                dst.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        e1.synchronize()
+        ems = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": whole_job_tflops(flops, world, args.e2e_steps, ems), "unit": UNIT,
+               "h2d_bytes_per_step": int(sum(t.nbytes for t in host) + oh.nbytes + lh.nbytes),
+               "d2h_bytes_per_step": int(sum(t.nbytes for t in outs)),
+               "ms_per_step": ems / args.e2e_steps, "steps": args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = time_oracle_bwd(w, do_bits, args.cpu_seconds)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC_BWD, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_dict(w, {"pass": "bwd", "flops_per_step": flops,
+                                  "parallelism": f"replicas x{world} (independent problems, no collective)"}),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                     "frac": achieved / peak, "traffic": profiled_traffic(f"{args.config}-bwd", "bwd"),
+                     "peak_source": f"MEASURED_PEAKS.json bf16_tflops (burst), of {peak_kind}",
+                     "frac_of_sustained": (achieved / peak_sustained) if peak_sustained else None,
+                     "timed": "whole step: D / accumulator prep, the backward kernel, dQ conversion"},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 3 * args.steps,
+        "clocks": sampler.summary(t_host0, t_host1),
     }
     print(json.dumps(line), flush=True)
 

@@ -69,3 +69,16 @@ def test_reference_arm_runs_on_rank0_only(capsys, monkeypatch):
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_reference_arm_of_the_backward(capsys):
+    """--impl reference --pass bwd: the gradient oracle on whole units."""
+    import bench
+
+    class A:
+        config, steps, warmup, gpus, pass_ = "c1", 1, 0, 1, "bwd"
+    bench.run_reference(A, rank=0)
+    import json
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC_BWD and line["value"] > 0
+    assert line["config"]["pass"] == "bwd" and line["cpu_baseline"]["kind"] == "oracle"
