@@ -33,6 +33,10 @@ one stream; for the packed batch the sequence lengths are drawn first):
   B=1, H=32, d=128, causal -- the chunked-prefill shape
 * dec: one decode step -- 1 query row per (batch, head) against a 32768-key
   cache, B=8, Hq=32, Hkv=8, d=128 (with one row, causal allows every key)
+* c3f8: c3's shape with Q, K, V drawn as N(0,1) times 32 and rounded to
+  nearest-even FP8 E4M3 (per-tensor scale 1/32)
+* E4M3: 1 sign, 4 exponent bits (bias 7), 3 mantissa bits, subnormals in
+  steps of 2^-9; the encoder rounds half to even and saturates at 448
 """
 from __future__ import annotations
 
@@ -43,6 +47,7 @@ from dataclasses import dataclass, field
 import numpy as np
 
 GAMMA = np.uint64(0x9E3779B97F4A7C15)
+FP8_SCALE = 1.0 / 32.0      # per-tensor scale of the E4M3 workloads (a power of two)
 _M1 = np.uint64(0xBF58476D1CE4E5B9)
 _M2 = np.uint64(0x94D049BB133111EB)
 _CHUNK = 1 << 22
@@ -86,6 +91,31 @@ def fp64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     return (f32.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
 
 
+def fp64_to_e4m3_bits(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to nearest-even FP8 E4M3 (OCP FP8: 1 sign, 4
+    exponent bits with bias 7, 3 mantissa bits, subnormals, no infinities, the
+    one NaN pattern per sign never produced): finite values beyond 448 saturate
+    to +-448.  Returns the 8-bit patterns."""
+    x = np.asarray(x, dtype=np.float64)
+    sign = (np.signbit(x)).astype(np.uint8) << np.uint8(7)
+    a = np.abs(x)
+    code = np.zeros(a.shape, dtype=np.int64)
+    sub = a < 2.0 ** -6
+    # subnormals (and zero): multiples of 2^-9, rounded half to even
+    code[sub] = np.rint(a[sub] * 512.0).astype(np.int64)
+    norm = ~sub
+    if norm.any():
+        f, ex = np.frexp(a[norm])                      # a = f 2^ex, f in [0.5, 1)
+        e = ex.astype(np.int64) - 1                     # a = (1 + m) 2^e
+        mq = np.rint((2.0 * f - 1.0) * 8.0).astype(np.int64)
+        carry = mq == 8
+        e[carry] += 1
+        mq[carry] = 0
+        c = ((e + 7) << 3) | mq
+        code[norm] = np.minimum(c, 0x7E)               # 0x7E = 448; larger values saturate
+    return (code.astype(np.uint8) | sign).astype(np.uint8)
+
+
 def bf16_bits_to_float(bits: np.ndarray) -> np.ndarray:
     """Widen bf16 bit patterns to fp32 (exact)."""
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
@@ -103,6 +133,32 @@ class Stream:
         self.pos += n
         span = np.uint64(hi - lo + 1)
         return (x % span).astype(np.int64) + lo
+
+    def normal_e4m3(self, shape, inv_scale: float, threads: int = 8) -> np.ndarray:
+        """E4M3 bit patterns of i.i.d. N(0,1) draws times ``inv_scale`` (the
+        tensor's quantisation: value = code * (1 / inv_scale)), C order."""
+        n = int(np.prod(shape))
+        draws = n + (n & 1)
+        if self.pos & 1:
+            self.pos += 1
+        base = self.pos
+        out = np.empty(n, dtype=np.uint8)
+
+        def work(c0):
+            c1 = min(c0 + _CHUNK, draws)
+            z = _normals_chunk(self.seed, base + c0, c1 - c0)
+            e = min(c1, n)
+            out[c0:e] = fp64_to_e4m3_bits(z[: e - c0] * inv_scale)
+
+        starts = range(0, draws, _CHUNK)
+        if threads > 1 and draws > _CHUNK:
+            with ThreadPoolExecutor(threads) as ex:
+                list(ex.map(work, starts))
+        else:
+            for c0 in starts:
+                work(c0)
+        self.pos += draws
+        return out.reshape(shape)
 
     def normal_bf16(self, shape, threads: int = 8) -> np.ndarray:
         """bf16 bit patterns of i.i.d. N(0,1) draws, in C order of ``shape``."""
@@ -143,6 +199,7 @@ class Workload:
     seed: int
     seqlens: list[int] | None = None
     Nk: int | None = None   # dense query chunk: keys per sequence (the chunk is the last N positions)
+    fp8: bool = False       # Q, K, V as E4M3 codes with per-tensor scale FP8_SCALE (see draw)
     q: np.ndarray | None = field(default=None, repr=False)
     k: np.ndarray | None = field(default=None, repr=False)
     v: np.ndarray | None = field(default=None, repr=False)
@@ -208,6 +265,14 @@ class Workload:
         s = Stream(self.seed)
         if self.packed:
             s.pos = self._len_draws
+        if self.fp8:
+            # N(0,1) samples times 1 / FP8_SCALE = 32 use E4M3's range (|x| <= ~180
+            # of 448) while keeping small values out of the subnormals
+            inv = 1.0 / FP8_SCALE
+            self.q = s.normal_e4m3(self.q_shape(), inv, threads)
+            self.k = s.normal_e4m3(self.kv_shape(), inv, threads)
+            self.v = s.normal_e4m3(self.kv_shape(), inv, threads)
+            return self
         self.q = s.normal_bf16(self.q_shape(), threads)
         self.k = s.normal_bf16(self.kv_shape(), threads)
         self.v = s.normal_bf16(self.kv_shape(), threads)
@@ -232,7 +297,7 @@ def packed_from_lengths(name, lens, H, d, causal, seed, Hkv=None) -> Workload:
 
 
 def config(name: str) -> Workload:
-    """The named workloads c1, c2nc, c2c, c3, c4, c5, p3, dec (inputs not yet drawn)."""
+    """The named workloads c1, c2nc, c2c, c3, c4, c5, p3, dec, c3f8 (inputs not yet drawn)."""
     if name == "c1":
         return Workload("c1", 1, 1, 1, 256, 64, False, 1001)
     if name == "c2nc":
@@ -249,6 +314,9 @@ def config(name: str) -> Workload:
         # a 2048-row prefill chunk at the end of a 16384-token sequence,
         # c3's heads and head size
         return Workload("p3", 1, 32, 32, 2048, 128, True, 1006, Nk=16384)
+    if name == "c3f8":
+        # c3 with Q, K, V in E4M3 (per-tensor scale 1/32)
+        return Workload("c3f8", 1, 32, 32, 16384, 128, True, 1008, fp8=True)
     if name == "dec":
         # one new token per sequence of a batch of 8 against a 32768-token
         # cache, c4's grouped heads
@@ -256,4 +324,4 @@ def config(name: str) -> Workload:
     raise KeyError(name)
 
 
-CONFIGS = ("c1", "c2nc", "c2c", "c3", "c4", "c5", "p3", "dec")
+CONFIGS = ("c1", "c2nc", "c2c", "c3", "c4", "c5", "p3", "dec", "c3f8")

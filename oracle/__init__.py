@@ -24,6 +24,11 @@ Every function cites the passage of the pages it follows in ``oracle.c``:
 * ``attention_bwd``    -- dQ, dK, dV of standard attention: the derivative of
                           the forward's definition (the pages name only the
                           recomputation of the backward pass).
+* ``e4m3_decode``, ``attention_fp8`` -- FP8 (E4M3) inputs: each code decoded
+                          by the format's definition and multiplied by its
+                          tensor's scale, then standard attention in fp64
+                          (the pages name FP8 only as FlashAttention-3's; the
+                          reading is attention of the dequantised inputs).
 
 Pins (in ``tests/test_oracle.py``): the worked examples of both pages, row sums
 of one, torch's fp64 scaled-dot-product attention as an independent library
@@ -235,6 +240,46 @@ def attention_bwd(q, k, v, dout, B, Hq, Hkv, N, d, scale, causal, units=None, nt
     if u is None:
         return dq.reshape(B, Hq, N, d), dk.reshape(B, Hkv, N, d), dv.reshape(B, Hkv, N, d)
     return dq, dk, dv
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """FP8 E4M3 codes -> fp64 by the format's definition: sign bit 7,
+    exponent bits 6..3 with bias 7, mantissa bits 2..0; exponent field 0 is
+    subnormal (mantissa * 2^-9); exponent 15 with mantissa 7 is NaN (no
+    infinities)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    val = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    val = np.where((e == 15) & ((c & 0x7) == 7), np.nan, val)
+    return sign * val
+
+
+def _exact_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Bit patterns of values that bf16 holds exactly (checked)."""
+    f = np.ascontiguousarray(x, dtype=np.float32)
+    if not np.array_equal(f.astype(np.float64), x):
+        raise ValueError("value not exact in fp32")
+    u = f.view(np.uint32)
+    if np.any(u & 0xFFFF):
+        raise ValueError("dequantised value not exact in bf16: use a power-of-two scale")
+    return (u >> 16).astype(np.uint16)
+
+
+def attention_fp8(q8, k8, v8, q_scale, k_scale, v_scale, B, Hq, Hkv, N, d, scale, causal, rows=None,
+                  nthreads=0, lib=None, abs_v=False) -> tuple[np.ndarray, np.ndarray]:
+    """Standard attention, in fp64, of the dequantised E4M3 inputs
+    (value = e4m3_decode(code) * tensor scale).  Dense layouts as
+    ``attention``.  With power-of-two scales every dequantised value is exact
+    in bf16, so the fp64 materialised attention of ``oracle.c`` runs on them
+    unchanged.  ``abs_v``: use |V| (gives sum_j p_j |v_j| per row, the
+    weight the FP8 tolerance is stated in)."""
+    qb = _exact_bf16_bits(e4m3_decode(q8) * q_scale)
+    kb = _exact_bf16_bits(e4m3_decode(k8) * k_scale)
+    vv = e4m3_decode(v8) * v_scale
+    vb = _exact_bf16_bits(np.abs(vv) if abs_v else vv)
+    return attention(qb, kb, vb, B, Hq, Hkv, N, d, scale, causal, rows=rows, nthreads=nthreads, lib=lib)
 
 
 def num_threads() -> int:

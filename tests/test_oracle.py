@@ -671,3 +671,77 @@ def test_bwd_units_subset():
     sq, sk, sv = oracle.attention_bwd(q, k, v, do, B, Hq, Hkv, N, d, 0.4, True, units=[3, 0])
     assert np.array_equal(sq[0], dq[1, 2:4]) and np.array_equal(sq[1], dq[0, 0:2])
     assert np.array_equal(sk[0], dk[1, 1]) and np.array_equal(sv[1], dv[0, 0])
+
+
+# --------------------------------------------------------------------------
+# FP8 (E4M3) inputs
+# --------------------------------------------------------------------------
+
+def test_e4m3_decode_matches_torch_on_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = oracle.e4m3_decode(codes)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan) and nan.sum() == 2
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+def test_e4m3_encoder_of_the_inputs_round_trips():
+    """The input generator's encoder and the oracle's decoder agree: decoding
+    an encoded value gives the nearest E4M3 value (checked against torch's
+    rounding), and re-encoding a decoded code gives the code back."""
+    x = np.random.default_rng(7).normal(size=20000) * 60
+    codes = syn.fp64_to_e4m3_bits(x)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(oracle.e4m3_decode(codes), ref)
+    finite = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    assert np.array_equal(syn.fp64_to_e4m3_bits(oracle.e4m3_decode(finite)), finite)
+
+
+def test_fp8_attention_brute_force():
+    """Tiny E4M3 problem against a pure-Python evaluation of softmax(QK^T)V
+    on torch-decoded inputs (no max shift)."""
+    B, Hq, Hkv, N, d, scale = 1, 2, 1, 6, 8, 0.35
+    s = syn.Stream(5)
+    inv = 32.0
+    q8, k8, v8 = s.normal_e4m3((B, Hq, N, d), inv), s.normal_e4m3((B, Hkv, N, d), inv), s.normal_e4m3((B, Hkv, N, d), inv)
+    dec = lambda a: torch.from_numpy(a).view(torch.float8_e4m3fn).to(torch.float64).numpy() / inv
+    qf, kf, vf = dec(q8)[0], dec(k8)[0], dec(v8)[0]
+    for causal in (False, True):
+        o, lse = oracle.attention_fp8(q8, k8, v8, 1 / inv, 1 / inv, 1 / inv, B, Hq, Hkv, N, d, scale, causal)
+        for h in range(Hq):
+            for i in range(N):
+                keys = range(i + 1) if causal else range(N)
+                w = [math.exp(scale * float(np.dot(qf[h, i], kf[0, j]))) for j in keys]
+                ref = sum(wj * vf[0, j] for wj, j in zip(w, keys)) / sum(w)
+                assert np.max(np.abs(o[h * N + i] - ref)) < 1e-12
+                assert abs(lse[h * N + i] - math.log(sum(w))) < 1e-12
+
+
+def test_fp8_attention_rejects_inexact_scales():
+    q8 = np.full((1, 1, 2, 4), 0x39, dtype=np.uint8)     # 1.125
+    with pytest.raises(ValueError):
+        oracle.attention_fp8(q8, q8, q8, 0.1, 1.0, 1.0, 1, 1, 1, 2, 4, 1.0, False)
+
+
+@pytest.mark.parametrize("old,new", [
+    ("np.exp2(e.astype(np.float64) - 7.0)", "np.exp2(e.astype(np.float64) - 8.0)"),     # exponent bias
+    ("m * 2.0 ** -9", "m * 2.0 ** -10"),                                                   # subnormal step
+    ("(1.0 + m / 8.0)", "(1.0 + m / 16.0)"),                                               # mantissa width
+])
+def test_planted_mistake_in_e4m3_decode_is_caught(old, new, tmp_path):
+    """Each mistake planted into a copy of the oracle's decoder breaks the
+    torch pin."""
+    import importlib.util
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "__init__.py")).read()
+    assert old in src
+    path = tmp_path / "oracle_mut.py"
+    path.write_text(src.replace(old, new, 1))
+    spec = importlib.util.spec_from_file_location("oracle_mut", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = mod.e4m3_decode(codes)
+    nan = np.isnan(ref)
+    assert not np.array_equal(got[~nan], ref[~nan])
