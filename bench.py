@@ -65,6 +65,9 @@ def workload_desc(w):
         return (f"{w.name}: {'causal' if w.causal else 'non-causal'} query chunk of {w.N} rows (the last "
                 f"positions) against {w.Nk} keys, B={w.B} Hq={w.Hq} Hkv={w.Hkv} d={w.d}, bf16 N(0,1), "
                 "scale=1/sqrt(d)")
+    if w.fp8:
+        return (f"{w.name}: {'causal' if w.causal else 'non-causal'} B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d}, "
+                "Q/K/V E4M3 codes of N(0,1)*32 (per-tensor scale 1/32), scale=1/sqrt(d)")
     if w.packed:
         shape = f"packed {w.B} sequences (lengths {min(w.seqlens)}..{max(w.seqlens)}), H={w.Hq}"
     else:
@@ -224,6 +227,11 @@ def row_flops(w, rows):
 def oracle_rows(w, rows):
     """The oracle on the given query rows of workload ``w``."""
     import oracle
+    if w.fp8:
+        from exact_tiled_attention_32_b200 import synthetic as syn
+        s = syn.FP8_SCALE
+        return oracle.attention_fp8(w.q, w.k, w.v, s, s, s, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal,
+                                    rows=rows)
     if w.chunk:
         return oracle.attention_kv(w.q, w.k, w.v, w.B, w.Hq, w.Hkv, w.N, w.Nk, w.d, w.scale, w.causal,
                                    rows=rows)
@@ -386,11 +394,14 @@ def main():
         if w.packed or w.chunk:
             raise SystemExit("--pass bwd runs on dense workloads (c1, c2nc, c2c, c3, c4)")
         return run_bwd(args, w, rank, world, dev)
-    q = torch.from_numpy(w.q.view(np.int16)).view(torch.bfloat16).to(dev)
-    k = torch.from_numpy(w.k.view(np.int16)).view(torch.bfloat16).to(dev)
-    v = torch.from_numpy(w.v.view(np.int16)).view(torch.bfloat16).to(dev)
+    if w.fp8:
+        q, k, v = (torch.from_numpy(a).to(dev) for a in (w.q, w.k, w.v))      # E4M3 codes
+    else:
+        q = torch.from_numpy(w.q.view(np.int16)).view(torch.bfloat16).to(dev)
+        k = torch.from_numpy(w.k.view(np.int16)).view(torch.bfloat16).to(dev)
+        v = torch.from_numpy(w.v.view(np.int16)).view(torch.bfloat16).to(dev)
     cu = None if w.cu_seqlens is None else torch.from_numpy(w.cu_seqlens).to(dev)
-    o = torch.empty_like(q)
+    o = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
     lse_shape = (w.Hq, w.N) if w.packed else (w.B, w.Hq, w.N)
     lse = torch.empty(lse_shape, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -402,8 +413,13 @@ def main():
         ws_bytes = fa.fa_splitkv_workspace_bytes(w.B, w.Hq, w.N, w.d, splits)
         ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
 
+    fp8_scale = syn.FP8_SCALE
+
     def step():
-        if w.decode:
+        if w.fp8:
+            rc = fa.fa_fwd_fp8(q, k, v, o, lse, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal, fp8_scale, fp8_scale,
+                               fp8_scale, stream)
+        elif w.decode:
             rc = fa.fa_fwd_splitkv(q, k, v, o, lse, w.B, w.Hq, w.Hkv, w.N, w.Nk, w.d, w.scale, w.causal,
                                    splits, ws, ws_bytes, stream)
         elif w.chunk:
@@ -456,9 +472,12 @@ def main():
     # ---- end to end through the public call, host buffers, copies timed
     e2e = None
     if args.e2e_steps > 0:
-        qh = torch.from_numpy(w.q.view(np.int16)).view(torch.bfloat16).pin_memory()
-        kh = torch.from_numpy(w.k.view(np.int16)).view(torch.bfloat16).pin_memory()
-        vh = torch.from_numpy(w.v.view(np.int16)).view(torch.bfloat16).pin_memory()
+        if w.fp8:
+            qh, kh, vh = (torch.from_numpy(a).pin_memory() for a in (w.q, w.k, w.v))
+        else:
+            qh = torch.from_numpy(w.q.view(np.int16)).view(torch.bfloat16).pin_memory()
+            kh = torch.from_numpy(w.k.view(np.int16)).view(torch.bfloat16).pin_memory()
+            vh = torch.from_numpy(w.v.view(np.int16)).view(torch.bfloat16).pin_memory()
         oh = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
         lh = torch.empty(lse_shape, dtype=torch.float32).pin_memory()
 
@@ -466,7 +485,10 @@ def main():
             qd = qh.to(dev, non_blocking=True)
             kd = kh.to(dev, non_blocking=True)
             vd = vh.to(dev, non_blocking=True)
-            if w.decode:
+            if w.fp8:
+                od, ld = fa.attention_forward_fp8(qd, kd, vd, fp8_scale, fp8_scale, fp8_scale, causal=w.causal,
+                                                  scale=w.scale)
+            elif w.decode:
                 od, ld = fa.attention_forward_splitkv(qd, kd, vd, causal=w.causal, scale=w.scale,
                                                       num_splits=splits, workspace=ws)
             elif w.chunk:
@@ -516,6 +538,12 @@ def main():
                     "peak_source": f"MEASURED_PEAKS.json hbm_gbs, of {hbm_kind}",
                     "algorithmic_bytes": w.hbm_bytes(),
                     "timed": f"whole step: split-key forward + merge of {splits} splits"}
+    elif w.fp8:
+        # the FP8 peak: the measured bf16 peak times the nominal FP8 / BF16 ratio (4.5 / 2.25)
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": 2 * peak, "unit": UNIT,
+                    "frac": achieved / (2 * peak), "traffic": profiled_traffic(args.config),
+                    "peak_source": f"2 x MEASURED_PEAKS.json bf16_tflops (burst; nominal fp8/bf16 ratio), of {peak_kind}",
+                    "frac_of_sustained": (achieved / (2 * peak_sustained)) if peak_sustained else None}
     else:
         roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
                     "frac": achieved / peak, "traffic": profiled_traffic(args.config),
@@ -524,7 +552,7 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if w.fp8 else "bf16", "data": "synthetic",
         "config": config_dict(w, {"parallelism": f"replicas x{world} (independent problems, no collective)",
                                   **({"num_splits": splits} if w.decode else {})}),
         "roofline": roofline,

@@ -30,7 +30,7 @@ FA_ERR_SEQLENS = -9
 
 EXPORTED = ("fa_fwd", "fa_get_device_status", "fa_status_string", "fa_fwd_noalloc", "fa_fwd_kvcache",
             "fa_selftest_watchdog", "fa_fwd_splitkv", "fa_splitkv_num_splits", "fa_splitkv_workspace_bytes",
-            "fa_bwd", "fa_bwd_workspace_bytes")
+            "fa_bwd", "fa_bwd_workspace_bytes", "fa_fwd_fp8")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -66,6 +66,9 @@ _lib.fa_bwd.argtypes = [ctypes.c_void_p] * 9 + [ctypes.c_int] * 5 + [
 ]
 _lib.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
 _lib.fa_bwd_workspace_bytes.argtypes = [ctypes.c_int] * 4
+_lib.fa_fwd_fp8.restype = ctypes.c_int
+_lib.fa_fwd_fp8.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_int] + \
+    [ctypes.c_float] * 3 + [ctypes.c_void_p]
 _lib.fa_selftest_watchdog.restype = ctypes.c_int
 _lib.fa_selftest_watchdog.argtypes = [ctypes.c_int, ctypes.c_void_p]
 _lib.fa_get_device_status.restype = ctypes.c_int
@@ -244,6 +247,41 @@ def attention_backward(q, k, v, o, lse, dout, *, causal: bool = False, scale: fl
     if rc != FA_OK:
         raise FAError(rc, "fa_bwd")
     return dq, dk, dv
+
+
+def fa_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, q_scale, k_scale, v_scale, stream=None) -> int:
+    """The C entry point of the FP8 (E4M3) forward; returns the status."""
+    return _lib.fa_fwd_fp8(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), int(B), int(Hq), int(Hkv), int(N),
+                           int(d), float(scale), int(bool(causal)), float(q_scale), float(k_scale), float(v_scale),
+                           _stream(stream))
+
+
+def attention_forward_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: float, *, causal: bool = False,
+                          scale: float | None = None):
+    """O (bf16), lse for E4M3 q [B, Hq, N, d], k/v [B, Hkv, N, d] (CUDA tensors
+    of dtype torch.float8_e4m3fn or uint8 holding E4M3 codes) with per-tensor
+    scales: the values are code * scale."""
+    import torch
+
+    for t in (q, k, v):
+        if t.dtype not in (torch.uint8, getattr(torch, "float8_e4m3fn", torch.uint8)):
+            raise TypeError("q, k, v must be float8_e4m3fn (or uint8 E4M3 codes)")
+    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    if q.dim() != 4 or k.dim() != 4 or k.shape != v.shape:
+        raise ValueError("dense layout: q [B,Hq,N,d], k/v [B,Hkv,N,d]")
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape[0] != B or k.shape[2] != N or k.shape[3] != d:
+        raise ValueError("k/v shape does not match q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = torch.empty((B, Hq, N, d), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    rc = fa_fwd_fp8(q, k, v, out, lse, B, Hq, Hkv, N, d, scale, causal, q_scale, k_scale, v_scale,
+                    torch.cuda.current_stream(q.device))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_fwd_fp8")
+    return out, lse
 
 
 def fa_selftest_watchdog(timeout_ms: int, stream=None) -> int:

@@ -82,7 +82,8 @@ struct alignas(64) Params {
     int group;                 // Hq / Hkv
     int group_units;           // dense: (batch, head) units scheduled together
     int causal, packed;
-    float scale_log2;          // scale * log2(e)
+    float scale_log2;          // scale * log2(e) (FP8: times the Q and K scales)
+    float o_scale;             // FP8: the V scale, applied to O in the epilogue
     unsigned long long timeout_ns;
     unsigned long long* trace;     // FA_TRACE builds: per-role clock64 stamps of CTA 0
 };
@@ -123,13 +124,16 @@ struct SeqTables {
     int pstart[kMaxPairs];     // first item index at pair level p
 };
 
-template <int D, bool PK>
+template <int D, bool PK, bool F8 = false>
 struct Cfg {
     static_assert(D == 64 || D == 128, "head dim");
-    static constexpr int kTileBytes = kBlockM * D * 2;     // one 128 x D bf16 tile
-    static constexpr int kBoxes = D / 64;
+    static_assert(!F8 || (D == 128 && !PK), "FP8: dense batches, d = 128");
+    static constexpr int kElem = F8 ? 1 : 2;                // bytes per element
+    static constexpr int kTileBytes = kBlockM * D * kElem;  // one 128 x D tile
+    static constexpr int kBoxes = D * kElem / 128;          // 128-byte-wide TMA boxes per tile row
+    static constexpr int kBoxCols = 128 / kElem;            // elements per box row
     // K/V ring depth: what fits next to the two Q tiles (and the packed tables)
-    static constexpr int kStages = (D == 128) ? (PK ? 4 : 5) : 10;
+    static constexpr int kStages = F8 ? 10 : ((D == 128) ? (PK ? 4 : 5) : 10);
     static_assert(kStages <= kMaxStages, "ring");
     static constexpr int kQOff = 0;
     static constexpr int kKVOff = 2 * kTileBytes;
@@ -284,10 +288,10 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, const P
 }
 
 // ---------------------------------------------------------------- producer
-template <int D, bool PK>
+template <int D, bool PK, bool F8 = false>
 __device__ void load_role(const Params& p, Misc& ms, const SeqTables& tab, uint32_t smem_q, uint32_t smem_kv,
                           int total) {
-    using C = Cfg<D, PK>;
+    using C = Cfg<D, PK, F8>;
     const uint64_t pol_kv = policy_evict_last();
     const uint64_t pol_q = policy_evict_first();
     uint32_t kv_it = 0, item_n = 0;
@@ -307,9 +311,9 @@ __device__ void load_role(const Params& p, Misc& ms, const SeqTables& tab, uint3
             for (int b = 0; b < C::kBoxes; ++b) {
                 const uint32_t dst = smem_q + t * C::kTileBytes + b * kBoxBytes;
                 if constexpr (!PK)
-                    tma_load_4d(dst, &p.tm_q, qbar, b * 64, row, it.h, it.seq, pol_q);
+                    tma_load_4d(dst, &p.tm_q, qbar, b * C::kBoxCols, row, it.h, it.seq, pol_q);
                 else
-                    tma_load_4d(dst, &p.tm_q, qbar, b * 64, it.h, it.tok0 + row, 0, pol_q);
+                    tma_load_4d(dst, &p.tm_q, qbar, b * C::kBoxCols, it.h, it.tok0 + row, 0, pol_q);
             }
         }
         ++item_n;
@@ -325,9 +329,9 @@ __device__ void load_role(const Params& p, Misc& ms, const SeqTables& tab, uint3
                     const uint32_t dst = smem_kv + st * C::kTileBytes + b * kBoxBytes;
                     const int key0 = (it.j0 + j) * kBlockN;
                     if constexpr (!PK)
-                        tma_load_4d(dst, map, bar, b * 64, key0, kvh, it.seq, pol_kv);
+                        tma_load_4d(dst, map, bar, b * C::kBoxCols, key0, kvh, it.seq, pol_kv);
                     else
-                        tma_load_4d(dst, map, bar, b * 64, kvh, it.tok0 + key0, 0, pol_kv);
+                        tma_load_4d(dst, map, bar, b * C::kBoxCols, kvh, it.tok0 + key0, 0, pol_kv);
                 }
                 ++kv_it;
                 if (++st == (uint32_t)C::kStages) {
@@ -349,30 +353,40 @@ __device__ void load_role(const Params& p, Misc& ms, const SeqTables& tab, uint3
 // ------------------------------------------------------------- MMA issuer
 // S_t = Q_t K^T over K = d (steps of 16), both operands K-major, 128-byte
 // swizzle; O_t (+)= P_t V with P read from TMEM.  Each is one asm block.
-template <int D>
+template <int D, bool F8 = false>
 __device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint64_t dq, uint64_t dk) {
-    constexpr uint32_t idesc = idesc_bf16_f32(kBlockM, kBlockN, false);
-    if constexpr (D == 128)
-        umma_ss_k128_x8(tmem_s, dq, dk, idesc);
-    else
-        umma_ss_k64_x4(tmem_s, dq, dk, idesc);
+    if constexpr (F8) {
+        umma_f8_ss_k128_x4(tmem_s, dq, dk, idesc_e4m3_f32(kBlockM, kBlockN, false));
+    } else {
+        constexpr uint32_t idesc = idesc_bf16_f32(kBlockM, kBlockN, false);
+        if constexpr (D == 128)
+            umma_ss_k128_x8(tmem_s, dq, dk, idesc);
+        else
+            umma_ss_k64_x4(tmem_s, dq, dk, idesc);
+    }
 }
-// Half h of O_t (+)= P_t V: keys 64h .. 64h+63 (P columns 32h.., V rows 64h..)
-template <int D>
+// Half h of O_t (+)= P_t V: keys 64h .. 64h+63 (bf16: P columns 32h.., FP8:
+// P columns 16h..; V rows 64h.. of 128 bytes each)
+template <int D, bool F8 = false>
 __device__ __forceinline__ void issue_pv_half(uint32_t tmem_o, uint32_t tmem_p, uint64_t dv, int h, bool accumulate) {
-    constexpr uint32_t idesc = idesc_bf16_f32(kBlockM, D, true);
-    umma_ts_kv64_x4(tmem_o, tmem_p + 32 * h, dv + static_cast<uint64_t>(h * ((64 * 128) >> 4)), idesc,
-                    accumulate ? 1u : 0u);
+    if constexpr (F8) {
+        umma_f8_ts_kv64_x2(tmem_o, tmem_p + 16 * h, dv + static_cast<uint64_t>(h * ((64 * 128) >> 4)),
+                           idesc_e4m3_f32(kBlockM, D, true), accumulate ? 1u : 0u);
+    } else {
+        constexpr uint32_t idesc = idesc_bf16_f32(kBlockM, D, true);
+        umma_ts_kv64_x4(tmem_o, tmem_p + 32 * h, dv + static_cast<uint64_t>(h * ((64 * 128) >> 4)), idesc,
+                        accumulate ? 1u : 0u);
+    }
 }
 
 // The MMA issuer.  Per work item it walks j = 0 .. nmax (nmax = the larger
 // block count of the two tiles): O_t += P_t V_{j-1} for each tile that had
 // block j-1, then S_t = Q_t K_j^T for each tile that has block j, tile 0
 // before tile 1 -- the order that keeps the two softmax warpgroups out of phase.
-template <int D, bool PK>
+template <int D, bool PK, bool F8 = false>
 __device__ void mma_role(const Params& p, Misc& ms, const SeqTables& tab, uint32_t tmem, uint32_t smem_q,
                          uint32_t smem_kv, int total) {
-    using C = Cfg<D, PK>;
+    using C = Cfg<D, PK, F8>;
     // descriptors of Q tile 0 and of ring stage 0; other tiles/stages are offsets
     const uint64_t dq0 = smem_desc_sw128(smem_q, 16, 1024);
     const uint64_t dk0 = smem_desc_sw128(smem_kv, 16, 1024);              // K-major (K tiles)
@@ -408,8 +422,8 @@ __device__ void mma_role(const Params& p, Misc& ms, const SeqTables& tab, uint32
                         if (!(ok = wait_bar(smem_u32(&ms.bar_p_half[t][h]), pc[t] & 1, p, ms, kSitePFull))) break;
                         tc_fence_after();
                         if (h == 0) FA_TRACE_EV(2, (item_n == 1 ? j : kTraceIters), 2 + 2 * t);
-                        issue_pv_half<D>(tmem + 256 + t * 128, tmem + t * 128, dv0 + vst * kTileStep, h,
-                                         h > 0 || j - 1 > 0);
+                        issue_pv_half<D, F8>(tmem + 256 + t * 128, tmem + t * 128, dv0 + vst * kTileStep, h,
+                                             h > 0 || j - 1 > 0);
                     }
                     if (!ok) break;
                     ++pc[t];
@@ -421,7 +435,7 @@ __device__ void mma_role(const Params& p, Misc& ms, const SeqTables& tab, uint32
                         tc_fence_after();
                         k_ready = true;
                     }
-                    issue_qk<D>(tmem + t * 128, dq0 + t * kTileStep, dk0 + kst * kTileStep);
+                    issue_qk<D, F8>(tmem + t * 128, dq0 + t * kTileStep, dk0 + kst * kTileStep);
                     umma_commit(smem_u32(&ms.bar_s_full[t]));
                     FA_TRACE_EV(2, (item_n == 1 ? j : kTraceIters), 3 + 2 * t);
                 }
@@ -477,7 +491,7 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
     return f2_pack(q0, q1);
 }
 
-template <int D, bool PK>
+template <int D, bool PK, bool F8 = false>
 __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, uint32_t tmem, int warp, int lane,
                              int total) {
     const int t = warp / 4;                          // query tile of this warpgroup
@@ -538,7 +552,10 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
             }
             const float m_new = fmaxf(m_used, mx * sl2);
             if (lane == 0 && wq == 0) FA_TRACE_EV(t, sc - 1, 3);
-            const bool need = m_new > m_used + kRescaleThreshold;
+            // FP8: exact running maximum (threshold 0), so that P <= 1 before the
+            // 2^8 shift below; bf16: lazy rescale
+            constexpr float kThr = F8 ? 0.f : kRescaleThreshold;
+            const bool need = m_new > m_used + kThr;
             if (j > 0 && __any_sync(0xffffffffu, need)) {
                 // Theorem 2: rescale the partial output when the max grows.
                 // S_t(j) was issued after O_t += P_t V_{j-1}, so O_t is final here.
@@ -563,12 +580,18 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
                 l *= (m_used == -INFINITY) ? 0.f : ex2_approx(m_used - m_new);
                 m_used = m_new;
             }
-            const float msub = (m_used == -INFINITY) ? 0.f : m_used;
+            // FP8: P is computed as 2^8 * exp2(x - m) in (0, 256], so that E4M3
+            // holds every entry above 2^-14 of the row maximum as a normal
+            // number (relative rounding error <= 2^-4); l carries the same
+            // factor, and lse takes it back out
+            constexpr float kPShift = F8 ? 8.f : 0.f;
+            const float msub = ((m_used == -INFINITY) ? 0.f : m_used) - kPShift;
             const uint64_t nm2 = f2_pack(-msub, -msub);
             uint64_t acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0;   // packed row sums (+0.0f pairs)
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                uint32_t pk[32];
+                uint32_t pk[32];             // bf16: 32 pairs; FP8: pk[0..15], four per word
+                float e_prev = 0.f, e_prev1 = 0.f;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int gi = 32 * half + i;       // pair of columns 2gi, 2gi+1
@@ -590,9 +613,23 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
                     }
                     float e0, e1;
                     f2_unpack(e, e0, e1);
-                    pk[i] = pack_bf16x2(e0, e1);
+                    if constexpr (F8) {
+                        // P <= 2^8 fits E4M3's range (448)
+                        if (i & 1)
+                            pk[i >> 1] = pack_e4m3x4(e_prev, e_prev1, e0, e1);
+                        else {
+                            e_prev = e0;
+                            e_prev1 = e1;
+                        }
+                    } else {
+                        pk[i] = pack_bf16x2(e0, e1);
+                    }
                 }
-                tmem_st32(taddr_s + half * 32, pk);
+                if constexpr (F8) {
+                    tmem_st16(taddr_s + half * 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
+                } else {
+                    tmem_st32(taddr_s + half * 32, pk);
+                }
                 if (half == 0) {
                     // keys 0-63 of P are ready: the tensor core can start on them
                     tmem_wait_st();
@@ -619,7 +656,8 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
         ++oc;
         tc_fence_after();
         const bool valid = row < it.len;
-        const float inv = l > 0.f ? 1.f / l : 0.f;
+        float inv = l > 0.f ? 1.f / l : 0.f;
+        if constexpr (F8) inv *= p.o_scale;
         uint16_t* orow;
         float* lrow;
         if constexpr (!PK) {
@@ -645,7 +683,7 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
                 if (valid) {
                     float lg;
                     asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg) : "f"(l));
-                    p.lse_part[prid] = (l > 0.f) ? (m_used + lg) * 0.69314718055994531f : -INFINITY;
+                    p.lse_part[prid] = (l > 0.f) ? (m_used + lg - (F8 ? 8.f : 0.f)) * 0.69314718055994531f : -INFINITY;
                 }
                 tc_fence_before();
                 continue;
@@ -675,16 +713,16 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
         if (valid) {
             float lg;
             asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg) : "f"(l));
-            *lrow = (l > 0.f) ? (m_used + lg) * 0.69314718055994531f : -INFINITY;
+            *lrow = (l > 0.f) ? (m_used + lg - (F8 ? 8.f : 0.f)) * 0.69314718055994531f : -INFINITY;
         }
         tc_fence_before();
     }
 }
 
 // ------------------------------------------------------------------ kernel
-template <int D, bool PK>
+template <int D, bool PK, bool F8 = false>
 __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_constant__ Params p) {
-    using C = Cfg<D, PK>;
+    using C = Cfg<D, PK, F8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Misc& ms = *reinterpret_cast<Misc*>(smem + C::kMiscOff);
@@ -782,14 +820,14 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
 
     if (warp < kNumSoftmaxWarps) {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
-        softmax_role<D, PK>(p, ms, tab, tmem, warp, lane, total);
+        softmax_role<D, PK, F8>(p, ms, tab, tmem, warp, lane, total);
     } else {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
         if (warp == kMmaWarp) {
-            if (lane == 0) mma_role<D, PK>(p, ms, tab, tmem, smem_q, smem_kv, total);
+            if (lane == 0) mma_role<D, PK, F8>(p, ms, tab, tmem, smem_q, smem_kv, total);
             __syncwarp();
         } else if (warp == kLoadWarp) {
-            if (lane == 0) load_role<D, PK>(p, ms, tab, smem_q, smem_kv, total);
+            if (lane == 0) load_role<D, PK, F8>(p, ms, tab, smem_q, smem_kv, total);
             __syncwarp();
         }
     }
@@ -910,6 +948,9 @@ int init_device(int dev, DeviceState** out) {
             good = good && cudaFuncSetAttribute(fa_fwd_kernel<128, true>,
                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 Cfg<128, true>::kSmemBytes) == cudaSuccess;
+            good = good && cudaFuncSetAttribute(fa_fwd_kernel<128, false, true>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                Cfg<128, false, true>::kSmemBytes) == cudaSuccess;
             ds.status_code = good ? FA_OK : FA_ERR_LAUNCH;
         }
     }
@@ -919,33 +960,34 @@ int init_device(int dev, DeviceState** out) {
 
 // 4-D bf16 tensor map with a 64 x rows box, 128-byte swizzle.
 bool encode_map(CUtensorMap* m, const void* base, const uint64_t dims[4], const uint64_t strides[3],
-                const uint32_t box[4]) {
+                const uint32_t box[4], bool bytes) {
     const cuuint32_t elem[4] = {1, 1, 1, 1};
-    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+    CUresult r = g_encode(m, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                          const_cast<void*>(base), dims, strides, box,
                           elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
 static bool make_maps(Params& P, const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int N,
-                      int Nk, int d, bool packed) {
-    const uint64_t e = 2;
+                      int Nk, int d, bool packed, bool fp8 = false) {
+    const uint64_t e = fp8 ? 1 : 2;
     if (!packed) {
         const uint64_t dq[4] = {(uint64_t)d, (uint64_t)N, (uint64_t)Hq, (uint64_t)B};
         const uint64_t sq[3] = {d * e, (uint64_t)N * d * e, (uint64_t)Hq * N * d * e};
         const uint64_t dk[4] = {(uint64_t)d, (uint64_t)Nk, (uint64_t)Hkv, (uint64_t)B};
         const uint64_t sk[3] = {d * e, (uint64_t)Nk * d * e, (uint64_t)Hkv * Nk * d * e};
-        const uint32_t box[4] = {64, (uint32_t)kBlockM, 1, 1};
-        return encode_map(&P.tm_q, q, dq, sq, box) && encode_map(&P.tm_k, k, dk, sk, box) &&
-               encode_map(&P.tm_v, v, dk, sk, box);
+        const uint32_t box[4] = {(uint32_t)(128 / e), (uint32_t)kBlockM, 1, 1};    // 128-byte box rows
+        return encode_map(&P.tm_q, q, dq, sq, box, fp8) && encode_map(&P.tm_k, k, dk, sk, box, fp8) &&
+               encode_map(&P.tm_v, v, dk, sk, box, fp8);
     }
     const uint64_t dq[4] = {(uint64_t)d, (uint64_t)Hq, (uint64_t)N, 1};
     const uint64_t sq[3] = {d * e, (uint64_t)Hq * d * e, (uint64_t)N * Hq * d * e};
     const uint64_t dk[4] = {(uint64_t)d, (uint64_t)Hkv, (uint64_t)N, 1};
     const uint64_t sk[3] = {d * e, (uint64_t)Hkv * d * e, (uint64_t)N * Hkv * d * e};
     const uint32_t box[4] = {64, 1, (uint32_t)kBlockM, 1};
-    return encode_map(&P.tm_q, q, dq, sq, box) && encode_map(&P.tm_k, k, dk, sk, box) &&
-           encode_map(&P.tm_v, v, dk, sk, box);
+    return encode_map(&P.tm_q, q, dq, sq, box, false) && encode_map(&P.tm_k, k, dk, sk, box, false) &&
+           encode_map(&P.tm_v, v, dk, sk, box, false);
 }
 
 #ifndef FA_L2_GROUP_MIB
@@ -966,11 +1008,12 @@ static bool aligned(const void* ptr, uintptr_t a) { return (reinterpret_cast<uin
 static int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                       int N, int Nk, int q_off, int d, float scale, int causal, const int32_t* cu_seqlens,
                       cudaStream_t s, int* status, int num_sms, int qmod = 0, int splits = 1,
-                      float* o_part = nullptr, float* lse_part = nullptr) {
+                      float* o_part = nullptr, float* lse_part = nullptr, bool fp8 = false,
+                      float qk_scale = 1.f, float v_scale = 1.f) {
     const bool packed = cu_seqlens != nullptr;
     Params P;
     std::memset(&P, 0, sizeof(P));
-    if (!make_maps(P, q, k, v, B, Hq, Hkv, N, Nk, d, packed)) return FA_ERR_LAUNCH;
+    if (!make_maps(P, q, k, v, B, Hq, Hkv, N, Nk, d, packed, fp8)) return FA_ERR_LAUNCH;
     P.o = o;
     P.lse = lse;
     P.cu_seqlens = cu_seqlens;
@@ -992,7 +1035,8 @@ static int launch_fwd(const void* q, const void* k, const void* v, void* o, floa
     }
     P.causal = causal ? 1 : 0;
     P.packed = packed ? 1 : 0;
-    P.scale_log2 = scale * 1.4426950408889634f;
+    P.scale_log2 = scale * qk_scale * 1.4426950408889634f;
+    P.o_scale = v_scale;
     P.timeout_ns = 2000000000ull;
     P.qmod = qmod;
     P.splits = splits;
@@ -1008,7 +1052,9 @@ static int launch_fwd(const void* q, const void* k, const void* v, void* o, floa
         items = (long long)num_sms;    // exact count is known only on the device
     }
     const int grid = (int)std::min<long long>(items, num_sms);
-    if (d == 64 && !packed)
+    if (fp8)
+        fa_fwd_kernel<128, false, true><<<grid, kThreads, Cfg<128, false, true>::kSmemBytes, s>>>(P);
+    else if (d == 64 && !packed)
         fa_fwd_kernel<64, false><<<grid, kThreads, Cfg<64, false>::kSmemBytes, s>>>(P);
     else if (d == 64)
         fa_fwd_kernel<64, true><<<grid, kThreads, Cfg<64, true>::kSmemBytes, s>>>(P);
@@ -1189,6 +1235,29 @@ extern "C" int fa_fwd_splitkv(const void* q, const void* k, const void* v, void*
     else
         fa_combine_kernel<128><<<grid, 256, 0, s>>>(o_part, lse_part, static_cast<uint16_t*>(o), lse, rows, num_splits);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+extern "C" int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                          int N, int d, float scale, int causal, float q_scale, float k_scale, float v_scale,
+                          void* stream) {
+    if (B < 0 || N < 0 || Hq < 1) return FA_ERR_SHAPE;
+    if (d != 128) return FA_ERR_HEADDIM;
+    if (Hkv < 1 || Hq % Hkv != 0) return FA_ERR_GQA;
+    if (!(q_scale > 0.f) || !(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(q_scale) ||
+        !std::isfinite(k_scale) || !std::isfinite(v_scale))
+        return FA_ERR_SHAPE;
+    if (B == 0 || N == 0) return FA_OK;
+    if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+        return FA_ERR_ALIGN;
+    if ((long long)B * Hq * N > (1ll << 30)) return FA_ERR_SHAPE;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_LAUNCH;
+    DeviceState* ds = nullptr;
+    const int st = init_device(dev, &ds);
+    if (st != FA_OK) return st;
+    return launch_fwd(q, k, v, o, lse, B, Hq, Hkv, N, N, 0, d, scale, causal, nullptr, static_cast<cudaStream_t>(stream),
+                      ds->status, ds->num_sms, 0, 1, nullptr, nullptr, true, q_scale * k_scale, v_scale);
 }
 
 extern "C" int fa_selftest_watchdog(int timeout_ms, void* stream) {

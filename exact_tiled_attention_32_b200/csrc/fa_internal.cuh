@@ -20,8 +20,9 @@ constexpr int kMaxDevices = 64;
 // the forward kernels' shared-memory limits); returns FA_OK or the error.
 int init_device(int dev, DeviceState** out);
 
-// 4-D bf16 tensor map with the given box, 128-byte swizzle.
+// 4-D tensor map with the given box, 128-byte swizzle; bf16 elements, or
+// bytes (FP8) when `bytes` is set.
 bool encode_map(CUtensorMap* m, const void* base, const uint64_t dims[4], const uint64_t strides[3],
-                const uint32_t box[4]);
+                const uint32_t box[4], bool bytes = false);
 
 }  // namespace fa_sm100

@@ -105,6 +105,29 @@ int fa_fwd_kvcache(const void* q, const void* k, const void* v, void* o, float* 
                    void* stream);
 
 /*
+ * fa_fwd_fp8 -- the forward with FP8 inputs (dense batches, d = 128),
+ * asynchronous on `stream`.  "FlashAttention and Chunked Prefill Mechanics"
+ * (section 1) names FlashAttention-3's FP8 support; the same tiled algorithm
+ * runs on E4M3 operands with fp32 accumulation:
+ *
+ *   q, k, v        FP8 E4M3 codes (1 byte each, OCP E4M3: 4 exponent bits with
+ *                  bias 7, 3 mantissa bits), dense layouts of fa_fwd.  The
+ *                  values are code * q_scale, code * k_scale, code * v_scale
+ *                  (per-tensor scales, finite and > 0).
+ *   o, lse         bf16 output and fp32 logsumexp, as fa_fwd.
+ *
+ * S = Q K^T is computed exactly from the codes (E4M3 products are exact in
+ * fp32) and scaled by scale * q_scale * k_scale; the exponentials are rounded
+ * to E4M3 for the P V product (relative error <= 2^-4 for P >= 2^-6), O is
+ * divided by the fp32 row sum and multiplied by v_scale.  Errors: as fa_fwd;
+ * FA_ERR_HEADDIM for d != 128, FA_ERR_SHAPE for a scale that is not finite
+ * and positive.
+ */
+int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+               int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+               float q_scale, float k_scale, float v_scale, void* stream);
+
+/*
  * fa_fwd_splitkv -- fa_fwd_kvcache for decode-shaped problems (a few query
  * rows against a long KV cache), asynchronous on `stream`.  Same arguments,
  * layouts, masks and result as fa_fwd_kvcache, plus:

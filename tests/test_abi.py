@@ -126,6 +126,19 @@ def test_bwd_argument_errors_and_workspace_bytes():
     assert call(B=0, ptrs=(0,) * 9, ws=0, wb=0) == fa.FA_OK
 
 
+def test_fp8_argument_errors_found_on_the_host():
+    from exact_tiled_attention_32_b200 import binding as fa
+    p = 1 << 20
+    call = lambda d=128, qs=1.0, Hkv=2, ptrs=(p,) * 5, B=1: fa.fa_fwd_fp8(*ptrs, B, 4, Hkv, 256, d, 0.1, 1, qs, 1.0, 1.0)
+    assert call(d=64) == fa.FA_ERR_HEADDIM
+    assert call(qs=0.0) == fa.FA_ERR_SHAPE
+    assert call(qs=float("nan")) == fa.FA_ERR_SHAPE
+    assert call(Hkv=3) == fa.FA_ERR_GQA
+    assert call(ptrs=(p, p, 0, p, p)) == fa.FA_ERR_NULL
+    assert call(ptrs=(p + 1, p, p, p, p)) == fa.FA_ERR_ALIGN
+    assert call(B=0, ptrs=(0,) * 5) == fa.FA_OK
+
+
 def test_no_device_means_launch_error():
     import torch
     if torch.cuda.is_available():

@@ -1,0 +1,108 @@
+"""fa_fwd_fp8 on B200: E4M3 Q, K, V with per-tensor scales, compared with the
+fp64 oracle of attention on the dequantised inputs.
+
+Tolerance (per output element, derived from the arithmetic): the forward's
+1e-2, plus one bf16 rounding of O (2^-7 |O|), plus the E4M3 rounding of P for
+the P V product.  The kernel computes P = 2^8 exp(s - m_run) <= 2^8 with the
+exact running maximum m_run, so every entry with exp(s - m) >= 2^-14 of the
+final row maximum m is a normal E4M3 number (relative error <= 2^-4), and an
+entry below that is off by at most 2^-18 (half the subnormal step, in units of
+the row maximum).  After the division by the row sum l = sum_j exp(s_j - m):
+|dO_c| <= 1e-2 + 2^-7 |O_c| + 2^-4 sum_j p_j |v_jc| + 2^-18 sum_{tiny j} |v_jc| / l.
+The weights p, l and the tiny set come from the exact scores of the
+dequantised inputs."""
+import numpy as np
+import pytest
+
+import oracle
+from exact_tiled_attention_32_b200 import synthetic as syn
+
+pytestmark = pytest.mark.gpu
+
+S = syn.FP8_SCALE
+
+
+def _dev(codes):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(codes)).cuda()
+
+
+def _run(w):
+    import torch
+    from exact_tiled_attention_32_b200 import binding as fa
+    o, lse = fa.attention_forward_fp8(_dev(w.q), _dev(w.k), _dev(w.v), S, S, S, causal=w.causal, scale=w.scale)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status() == 0
+    return o.float().cpu().numpy().astype(np.float64).reshape(-1, w.d), lse.cpu().numpy().astype(np.float64).reshape(-1)
+
+
+def _bound(w, rows, o_ref):
+    """Per-element tolerance of the rows (see the module docstring)."""
+    qf = oracle.e4m3_decode(w.q).reshape(-1, w.d) * S
+    kf = oracle.e4m3_decode(w.k).reshape(w.B, w.Hkv, w.N, w.d) * S
+    vf = oracle.e4m3_decode(w.v).reshape(w.B, w.Hkv, w.N, w.d) * S
+    g = w.Hq // w.Hkv
+    out = np.empty((len(rows), w.d))
+    for n, rid in enumerate(rows):
+        t = rid % w.N
+        bh = rid // w.N
+        b, h = divmod(bh, w.Hq)
+        keys = t + 1 if w.causal else w.N
+        K = kf[b, h // g, :keys]
+        V = np.abs(vf[b, h // g, :keys])
+        s = w.scale * (K @ qf[rid])
+        e = np.exp(s - s.max())
+        l = e.sum()
+        tiny = e < 2.0 ** -14
+        out[n] = 2.0 ** -4 * (e / l) @ V + 2.0 ** -18 * V[tiny].sum(axis=0) / l
+    return 1e-2 + 2.0 ** -7 * np.abs(o_ref) + out
+
+
+def _check(w, o, lse, rows, what):
+    o_ref, l_ref = oracle.attention_fp8(w.q, w.k, w.v, S, S, S, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal,
+                                        rows=rows)
+    got = o[rows]
+    assert not np.isnan(got).any(), f"{what}: NaN"
+    err = np.abs(got - o_ref)
+    excess = err - _bound(w, rows, o_ref)
+    assert excess.max() <= 0, f"{what}: O error {err.max():.3e} exceeds the E4M3 bound by {excess.max():.3e}"
+    assert err.mean() <= 1e-2, f"{what}: O mean error {err.mean():.3e}"
+    lerr = np.abs(lse[rows] - l_ref)
+    assert lerr.max() <= 1e-3, f"{what}: lse error {lerr.max():.3e}"
+
+
+CASES = [
+    # B, Hq, Hkv, N, causal
+    (1, 2, 2, 256, False),
+    (1, 2, 2, 256, True),
+    (1, 4, 2, 300, True),      # GQA, ragged last tile
+    (2, 2, 1, 1000, True),
+    (1, 3, 3, 129, False),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,causal", CASES)
+def test_fp8_all_rows(B, Hq, Hkv, N, causal):
+    w = syn.Workload("fp8", B, Hq, Hkv, N, 128, causal, 1100 + N, fp8=True).draw()
+    o, lse = _run(w)
+    _check(w, o, lse, np.arange(B * Hq * N), f"fp8 {B},{Hq},{Hkv},{N},{causal}")
+
+
+def test_fp8_argument_errors():
+    from exact_tiled_attention_32_b200 import binding as fa
+    p = 1 << 20
+    assert fa.fa_fwd_fp8(p, p, p, p, p, 1, 2, 2, 128, 64, 0.1, 1, 1, 1, 1) == fa.FA_ERR_HEADDIM
+    assert fa.fa_fwd_fp8(p, p, p, p, p, 1, 2, 2, 128, 128, 0.1, 1, 0, 1, 1) == fa.FA_ERR_SHAPE
+    assert fa.fa_fwd_fp8(p, p, p, p, p, 1, 2, 2, 128, 128, 0.1, 1, 1, float("inf"), 1) == fa.FA_ERR_SHAPE
+    assert fa.fa_fwd_fp8(p, p, p, p, p, 1, 4, 3, 128, 128, 0.1, 1, 1, 1, 1) == fa.FA_ERR_GQA
+    assert fa.fa_fwd_fp8(0, 0, 0, 0, 0, 0, 2, 2, 128, 128, 0.1, 1, 1, 1, 1) == fa.FA_OK
+
+
+def test_c3f8_sampled_rows():
+    """The FP8 workload the bench times (c3's shape in E4M3): sampled rows of
+    every head, tile boundaries included."""
+    from fa_util import sample_rows
+    w = syn.config("c3f8").draw()
+    o, lse = _run(w)
+    rows = sample_rows(w, early=4, tile_stride=16, n_random=4, seed=8)
+    _check(w, o, lse, rows, "c3f8")
