@@ -30,7 +30,7 @@ FA_ERR_SEQLENS = -9
 
 EXPORTED = ("fa_fwd", "fa_get_device_status", "fa_status_string", "fa_fwd_noalloc", "fa_fwd_kvcache",
             "fa_selftest_watchdog", "fa_fwd_splitkv", "fa_splitkv_num_splits", "fa_splitkv_workspace_bytes",
-            "fa_bwd", "fa_bwd_workspace_bytes", "fa_fwd_fp8")
+            "fa_bwd", "fa_bwd_workspace_bytes", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -69,6 +69,11 @@ _lib.fa_bwd_workspace_bytes.argtypes = [ctypes.c_int] * 4
 _lib.fa_fwd_fp8.restype = ctypes.c_int
 _lib.fa_fwd_fp8.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_int] + \
     [ctypes.c_float] * 3 + [ctypes.c_void_p]
+_lib.fa_fwd_partial.restype = ctypes.c_int
+_lib.fa_fwd_partial.argtypes = _lib.fa_fwd_kvcache.argtypes
+_lib.fa_merge_partials.restype = ctypes.c_int
+_lib.fa_merge_partials.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_int,
+                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
 _lib.fa_selftest_watchdog.restype = ctypes.c_int
 _lib.fa_selftest_watchdog.argtypes = [ctypes.c_int, ctypes.c_void_p]
 _lib.fa_get_device_status.restype = ctypes.c_int
@@ -282,6 +287,18 @@ def attention_forward_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: floa
     if rc != FA_OK:
         raise FAError(rc, "fa_fwd_fp8")
     return out, lse
+
+
+def fa_fwd_partial(q, k, v, o_part, lse_part, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream=None) -> int:
+    """The C entry point writing one key range's fp32 share (O / l, lse)."""
+    return _lib.fa_fwd_partial(_addr(q), _addr(k), _addr(v), _addr(o_part), _addr(lse_part), int(B), int(Hq),
+                               int(Hkv), int(Nq), int(Nk), int(d), float(scale), int(bool(causal)), _stream(stream))
+
+
+def fa_merge_partials(o_parts, lse_parts, nparts, rows, d, o, lse, stream=None) -> int:
+    """The C entry point merging shares of the same rows."""
+    return _lib.fa_merge_partials(_addr(o_parts), _addr(lse_parts), int(nparts), int(rows), int(d), _addr(o),
+                                  _addr(lse), _stream(stream))
 
 
 def fa_selftest_watchdog(timeout_ms: int, stream=None) -> int:

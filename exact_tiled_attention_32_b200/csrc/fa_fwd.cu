@@ -77,8 +77,8 @@ struct alignas(64) Params {
     int qmod;                  // dense: row r sits at position q_off + r % qmod (rows of several
                                // query heads packed into one sequence); 0: position q_off + r
     int splits;                // dense: key blocks of each tile are cut into this many splits
-    float* o_part;             // splits > 1: fp32 O / l of each split, [splits][B*Hq*N][d]
-    float* lse_part;           // splits > 1: logsumexp of each split, [splits][B*Hq*N]
+    float* o_part;             // dense, when set: fp32 O / l of each split, [splits][B*Hq*N][d]
+    float* lse_part;           // dense, when set: logsumexp of each split, [splits][B*Hq*N]
     int group;                 // Hq / Hkv
     int group_units;           // dense: (batch, head) units scheduled together
     int causal, packed;
@@ -469,7 +469,14 @@ __device__ void mma_role(const Params& p, Misc& ms, const SeqTables& tab, uint32
 #ifndef FA_POLY_PAIRS_PER8
 #define FA_POLY_PAIRS_PER8 0
 #endif
-constexpr int kPolyPairsPer8 = FA_POLY_PAIRS_PER8;   // column pairs (of every 8) on the polynomial
+#ifndef FA_POLY_PAIRS_PER8_F8
+#define FA_POLY_PAIRS_PER8_F8 1
+#endif
+// column pairs (of every 8) on the polynomial: none for bf16 (measured on B200:
+// slower), one for FP8, whose tensor work per block is half as long while the
+// exponentials are as many (measured: +2.4 %)
+constexpr int kPolyPairsPer8 = FA_POLY_PAIRS_PER8;
+constexpr int kPolyPairsPer8F8 = FA_POLY_PAIRS_PER8_F8;
 __device__ __forceinline__ uint64_t f2_const(uint32_t bits) {
     return (static_cast<uint64_t>(bits) << 32) | bits;
 }
@@ -512,7 +519,7 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
         const int row = it.q0 + t * kBlockM + r;
         if (n == 0) {
             // a split that holds no key block of this tile contributes nothing
-            if (!PK && p.splits > 1 && row < it.len)
+            if (!PK && p.o_part != nullptr && row < it.len)
                 p.lse_part[static_cast<size_t>(it.split) * p.B * p.Hq * p.N +
                            (static_cast<size_t>(it.seq) * p.Hq + it.h) * p.N + row] = -INFINITY;
             continue;
@@ -598,7 +605,7 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
                     const uint64_t x = f2_fma(f2_pack(__uint_as_float(s[2 * gi]), __uint_as_float(s[2 * gi + 1])),
                                               sl2x2, nm2);
                     uint64_t e;
-                    if ((gi % 8) < kPolyPairsPer8) {
+                    if ((gi % 8) < (F8 ? kPolyPairsPer8F8 : kPolyPairsPer8)) {
                         e = exp2_poly2(x);
                     } else {
                         float x0, x1;
@@ -662,7 +669,7 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
         float* lrow;
         if constexpr (!PK) {
             const size_t rid = (static_cast<size_t>(it.seq) * p.Hq + it.h) * p.N + row;
-            if (p.splits > 1) {
+            if (p.o_part != nullptr) {
                 // this split's O / l in fp32 and its logsumexp; a combine pass
                 // merges the splits
                 const size_t prid = static_cast<size_t>(it.split) * p.B * p.Hq * p.N + rid;
@@ -1258,6 +1265,48 @@ extern "C" int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, 
     if (st != FA_OK) return st;
     return launch_fwd(q, k, v, o, lse, B, Hq, Hkv, N, N, 0, d, scale, causal, nullptr, static_cast<cudaStream_t>(stream),
                       ds->status, ds->num_sms, 0, 1, nullptr, nullptr, true, q_scale * k_scale, v_scale);
+}
+
+extern "C" int fa_fwd_partial(const void* q, const void* k, const void* v, float* o_part, float* lse_part, int B,
+                              int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, void* stream) {
+    if (B < 0 || Nq < 0 || Nk < 0 || Hq < 1) return FA_ERR_SHAPE;
+    if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+    if (Hkv < 1 || Hq % Hkv != 0) return FA_ERR_GQA;
+    if (B == 0 || Nq == 0) return FA_OK;
+    if (Nk == 0 || (causal && Nk < Nq)) return FA_ERR_SHAPE;
+    if (!q || !k || !v || !o_part || !lse_part) return FA_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o_part, 16) || !aligned(lse_part, 4))
+        return FA_ERR_ALIGN;
+    if ((long long)B * Hq * Nq > (1ll << 30) || (long long)B * Hkv * Nk > (1ll << 31)) return FA_ERR_SHAPE;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_LAUNCH;
+    DeviceState* ds = nullptr;
+    const int st = init_device(dev, &ds);
+    if (st != FA_OK) return st;
+    return launch_fwd(q, k, v, nullptr, nullptr, B, Hq, Hkv, Nq, Nk, causal ? Nk - Nq : 0, d, scale, causal, nullptr,
+                      static_cast<cudaStream_t>(stream), ds->status, ds->num_sms, 0, 1, o_part, lse_part);
+}
+
+extern "C" int fa_merge_partials(const float* o_parts, const float* lse_parts, int nparts, long long rows, int d,
+                                 void* o, float* lse, void* stream) {
+    if (nparts < 1 || nparts > 4096 || rows < 0) return FA_ERR_SHAPE;
+    if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+    if (rows == 0) return FA_OK;
+    if (rows * nparts > (1ll << 40)) return FA_ERR_SHAPE;
+    if (!o_parts || !lse_parts || !o || !lse) return FA_ERR_NULL;
+    if (!aligned(o_parts, 16) || !aligned(lse_parts, 4) || !aligned(o, 16) || !aligned(lse, 4)) return FA_ERR_ALIGN;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_LAUNCH;
+    DeviceState* ds = nullptr;
+    const int st = init_device(dev, &ds);
+    if (st != FA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
+    if (d == 64)
+        fa_combine_kernel<64><<<grid, 256, 0, s>>>(o_parts, lse_parts, static_cast<uint16_t*>(o), lse, rows, nparts);
+    else
+        fa_combine_kernel<128><<<grid, 256, 0, s>>>(o_parts, lse_parts, static_cast<uint16_t*>(o), lse, rows, nparts);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
 extern "C" int fa_selftest_watchdog(int timeout_ms, void* stream) {

@@ -128,6 +128,36 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
                float q_scale, float k_scale, float v_scale, void* stream);
 
 /*
+ * fa_fwd_partial -- one key range's share of the forward, for merging later
+ * (ring attention, any split of the keys).  Same arguments, layouts and
+ * masks as fa_fwd_kvcache (query row i at key position Nk - Nq + i), but the
+ * results go, in fp32, to
+ *   o_part    [B, Hq, Nq, d]: O / l over this call's keys (0 for a row with
+ *             no allowed key),
+ *   lse_part  [B, Hq, Nq]: the logsumexp over this call's keys (-inf for a
+ *             row with no allowed key).
+ * fa_merge_partials combines such shares of the same rows (the online-softmax
+ * rescale of "Flash Attention", Online Softmax, Theorem 2, applied to whole
+ * key ranges).  Errors as fa_fwd_kvcache.
+ */
+int fa_fwd_partial(const void* q, const void* k, const void* v, float* o_part, float* lse_part,
+                   int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                   void* stream);
+
+/*
+ * fa_merge_partials -- merges nparts shares of the same `rows` query rows:
+ * o_parts [nparts][rows][d] and lse_parts [nparts][rows] (fp32, device) as
+ * fa_fwd_partial writes them, into bf16 o [rows][d] and fp32 lse [rows]:
+ *   lse = ln sum_s exp(lse_s),  O = sum_s exp(lse_s - lse) O_s.
+ * A share with lse_s = -inf carries weight 0; a row without any allowed key
+ * gets O = 0, lse = -inf.  d is 64 or 128; 1 <= nparts <= 4096.  Asynchronous
+ * on `stream`.  Errors: FA_ERR_SHAPE, FA_ERR_HEADDIM, FA_ERR_NULL,
+ * FA_ERR_ALIGN (o 16-byte aligned), FA_ERR_LAUNCH.
+ */
+int fa_merge_partials(const float* o_parts, const float* lse_parts, int nparts, long long rows, int d,
+                      void* o, float* lse, void* stream);
+
+/*
  * fa_fwd_splitkv -- fa_fwd_kvcache for decode-shaped problems (a few query
  * rows against a long KV cache), asynchronous on `stream`.  Same arguments,
  * layouts, masks and result as fa_fwd_kvcache, plus:
