@@ -579,14 +579,14 @@ def run_bwd(args, w, rank, world, dev):
     do_bits = bwd_dout(w)
     q, k, v, do = dev_bits(w.q), dev_bits(w.k), dev_bits(w.v), dev_bits(do_bits)
     o, lse = fa.attention_forward(q, k, v, causal=w.causal, scale=w.scale)
-    ws_bytes = fa.fa_bwd_workspace_bytes(w.B, w.Hq, w.N, w.d)
+    ws_bytes = fa.fa_bwd_workspace_bytes(w.B, w.Hq, w.N, w.d, False)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     stream = torch.cuda.current_stream(dev)
     flops = BWD_FLOP_FACTOR * w.flops()
 
     def step():
-        rc = fa.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal, ws,
+        rc = fa.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal, None, ws,
                        ws_bytes, stream)
         if rc != 0:
             raise fa.FAError(rc, "fa_bwd")

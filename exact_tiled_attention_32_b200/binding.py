@@ -62,10 +62,10 @@ _lib.fa_splitkv_workspace_bytes.restype = ctypes.c_size_t
 _lib.fa_splitkv_workspace_bytes.argtypes = [ctypes.c_int] * 5
 _lib.fa_bwd.restype = ctypes.c_int
 _lib.fa_bwd.argtypes = [ctypes.c_void_p] * 9 + [ctypes.c_int] * 5 + [
-    ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+    ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
 ]
 _lib.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
-_lib.fa_bwd_workspace_bytes.argtypes = [ctypes.c_int] * 4
+_lib.fa_bwd_workspace_bytes.argtypes = [ctypes.c_int] * 5
 _lib.fa_fwd_fp8.restype = ctypes.c_int
 _lib.fa_fwd_fp8.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_int] + \
     [ctypes.c_float] * 3 + [ctypes.c_void_p]
@@ -209,24 +209,25 @@ def attention_forward_splitkv(q, k, v, *, causal: bool = False, scale: float | N
     return out, lse
 
 
-def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, workspace, workspace_bytes,
-           stream=None) -> int:
+def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, cu_seqlens, workspace,
+           workspace_bytes, stream=None) -> int:
     """The C entry point of the backward pass; returns the status."""
     return _lib.fa_bwd(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), _addr(dout), _addr(dq), _addr(dk),
                        _addr(dv), int(B), int(Hq), int(Hkv), int(N), int(d), float(scale), int(bool(causal)),
-                       _addr(workspace), int(workspace_bytes), _stream(stream))
+                       _addr(cu_seqlens), _addr(workspace), int(workspace_bytes), _stream(stream))
 
 
-def fa_bwd_workspace_bytes(B, Hq, N, d) -> int:
+def fa_bwd_workspace_bytes(B, Hq, N, d, packed=False) -> int:
     """Workspace bytes fa_bwd needs (0 for bad arguments)."""
-    return int(_lib.fa_bwd_workspace_bytes(int(B), int(Hq), int(N), int(d)))
+    return int(_lib.fa_bwd_workspace_bytes(int(B), int(Hq), int(N), int(d), int(bool(packed))))
 
 
 def attention_backward(q, k, v, o, lse, dout, *, causal: bool = False, scale: float | None = None,
-                       workspace=None):
-    """dq, dk, dv for the dense forward O, lse = attention_forward(q, k, v)
+                       cu_seqlens=None, workspace=None):
+    """dq, dk, dv for the forward O, lse = attention_forward(q, k, v, ...)
     and the upstream gradient ``dout`` (bf16 CUDA tensors, layouts of the
-    dense forward).  The workspace is allocated with torch unless given."""
+    forward: dense, or packed with ``cu_seqlens``).  The workspace is
+    allocated with torch unless given."""
     import torch
 
     for t in (q, k, v, o, dout):
@@ -235,19 +236,30 @@ def attention_backward(q, k, v, o, lse, dout, *, causal: bool = False, scale: fl
     if lse.dtype != torch.float32:
         raise TypeError("lse must be float32")
     q, k, v, o, dout, lse = (t.contiguous() for t in (q, k, v, o, dout, lse))
-    if q.dim() != 4 or k.shape != v.shape or o.shape != q.shape or dout.shape != q.shape:
-        raise ValueError("dense layout: q, o, dout [B,Hq,N,d], k/v [B,Hkv,N,d]")
-    B, Hq, N, d = q.shape
-    Hkv = k.shape[1]
+    if k.shape != v.shape or o.shape != q.shape or dout.shape != q.shape:
+        raise ValueError("o, dout must have q's shape and v k's")
+    if cu_seqlens is None:
+        if q.dim() != 4:
+            raise ValueError("dense layout: q, o, dout [B,Hq,N,d], k/v [B,Hkv,N,d]")
+        B, Hq, N, d = q.shape
+        Hkv = k.shape[1]
+    else:
+        if q.dim() != 3:
+            raise ValueError("packed layout: q, o, dout [N,Hq,d], k/v [N,Hkv,d]")
+        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda:
+            raise ValueError("cu_seqlens must be an int32 CUDA tensor")
+        N, Hq, d = q.shape
+        Hkv = k.shape[1]
+        B = cu_seqlens.numel() - 1
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    need = fa_bwd_workspace_bytes(B, Hq, N, d)
+    need = fa_bwd_workspace_bytes(B, Hq, N, d, cu_seqlens is not None)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     dq = torch.empty_like(q)
     dk = torch.empty_like(k)
     dv = torch.empty_like(v)
-    rc = fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, workspace,
+    rc = fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, cu_seqlens, workspace,
                 workspace.numel() * workspace.element_size(), torch.cuda.current_stream(q.device))
     if rc != FA_OK:
         raise FAError(rc, "fa_bwd")

@@ -73,6 +73,7 @@ __device__ unsigned long long* g_btrace = nullptr;
 #endif
 
 constexpr int kBlock = 128;            // keys per item, queries per step
+constexpr int kMaxSeqsBwd = 1024;      // packed batches: sequences (one CTA builds the tables)
 constexpr int kThreads = 512;
 constexpr int kDqWarp0 = 8;            // warps 8-11: dQ warpgroup
 constexpr int kAllocWarp = 12;
@@ -94,13 +95,18 @@ enum WaitSite : int {
 
 struct alignas(64) Params {
     CUtensorMap tm_q, tm_k, tm_v, tm_do;
-    const float* lse2;      // [B, Hq, Npad]: lse * log2(e); +inf on padding rows
-    const float* Dvec;      // [B, Hq, Npad]: rowsum(dO * O); 0 on padding rows
-    float* dq_acc;          // [B, Hq, Npad, d] fp32, cleared by the prep kernel
-    uint16_t* dk;           // [B, Hkv, N, d] bf16
+    // Per-row vectors and the dQ accumulator live on padded rows: dense,
+    // [B, Hq, Npad] with Npad = N rounded up to 128; packed, [Hq, Npad] with
+    // sequence s at rows pad_off[s] .. (128-aligned; Npad bounds the total).
+    const float* lse2;      // lse * log2(e); +inf on padding rows
+    const float* Dvec;      // rowsum(dO * O); 0 on padding rows
+    float* dq_acc;          // [.., d] fp32, cleared by the prep kernel
+    const int32_t* cu;      // packed: cu_seqlens (B+1 offsets); dense: NULL
+    const int* tab;         // packed: work-unit starts [B+1], order [B], pad_off [B+1], total units
+    uint16_t* dk;           // dense [B, Hkv, N, d]; packed [N, Hkv, d]; bf16
     uint16_t* dv;           // [B, Hkv, N, d] bf16
     int* status;
-    int B, Hq, Hkv, N, Npad, group, causal;
+    int B, Hq, Hkv, N, Npad, group, causal, packed;
     float scale_log2, scale;
     unsigned long long timeout_ns;
 };
@@ -132,13 +138,24 @@ struct Cfg {
     static constexpr int kSmemBytes = kLayoutBytes + 1024 <= 232448 ? kLayoutBytes + 1024 : 232448;
 };
 
-// One work item: key block j of one (batch, kv head).
+// One work item: key block j of one (batch or sequence, kv head).
 struct Item {
     int b, hk, j;
     int i0;       // first query block (causal: j)
     int nq;       // query blocks per head
     int niter;    // group * (nq - i0)
+    int len;      // tokens of the sequence
+    int tok0;     // packed: first token of the sequence
+    int padoff;   // packed: first padded row of the sequence
 };
+
+// Padded row of the per-row vectors and of the dQ accumulator for query head
+// h, query block i of the item (dense: [B, Hq, Npad]; packed: [Hq, Npad]).
+__device__ __forceinline__ size_t vrow(const Item& it, const Params& p, int h, int i) {
+    const size_t base = p.packed ? static_cast<size_t>(h) * p.Npad + it.padoff
+                                 : (static_cast<size_t>(it.b) * p.Hq + h) * p.Npad;
+    return base + static_cast<size_t>(i) * kBlock;
+}
 
 __device__ __forceinline__ int item_of_round(int r) {
     const int G = gridDim.x;
@@ -151,6 +168,7 @@ __device__ __forceinline__ int item_of_round(int r) {
 // alone).  Units are numbered (batch, kv head)-major, so the CTAs running at
 // the same time share few heads and those heads' dQ accumulators stay in L2.
 __device__ __forceinline__ int num_work_units(const Params& p) {
+    if (p.packed) return p.tab[3 * p.B + 2];
     const int nk = (p.N + kBlock - 1) / kBlock;
     return ((nk + 1) / 2) * p.B * p.Hkv;
 }
@@ -161,14 +179,40 @@ __device__ __forceinline__ int num_work_units(const Params& p) {
 __device__ __forceinline__ int next_item(int r, const Params& p, int total_wu, Item& it) {
     const int w = item_of_round(r >> 1);
     if (w >= total_wu) return 0;
-    const int nk = (p.N + kBlock - 1) / kBlock;
-    const int npairs = (nk + 1) / 2;
-    const int u = w / npairs;
-    const int pr = w - u * npairs;
+    int nk, pr;
+    if (!p.packed) {
+        nk = (p.N + kBlock - 1) / kBlock;
+        const int npairs = (nk + 1) / 2;
+        const int u = w / npairs;
+        pr = w - u * npairs;
+        it.b = u / p.Hkv;
+        it.hk = u - it.b * p.Hkv;
+        it.len = p.N;
+        it.tok0 = 0;
+        it.padoff = 0;
+    } else {
+        // packed: units of sequence order[k] start at wu[k] (longest first)
+        const int* wu = p.tab;
+        const int* order = p.tab + p.B + 1;
+        const int* pad = p.tab + 2 * p.B + 1;
+        int lo = 0, hi = p.B - 1;                  // largest k with wu[k] <= w
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (wu[mid] <= w) lo = mid; else hi = mid - 1;
+        }
+        const int sq = order[lo];
+        it.b = sq;
+        it.tok0 = p.cu[sq];
+        it.len = p.cu[sq + 1] - it.tok0;
+        it.padoff = pad[sq];
+        nk = (it.len + kBlock - 1) / kBlock;
+        const int npairs = (nk + 1) / 2;
+        const int rem = w - wu[lo];
+        it.hk = rem / npairs;
+        pr = rem - it.hk * npairs;
+    }
     const int j = (r & 1) ? nk - 1 - pr : pr;
     if ((r & 1) && j == pr) return 2;
-    it.b = u / p.Hkv;
-    it.hk = u - it.b * p.Hkv;
     it.j = j;
     it.nq = nk;
     it.i0 = p.causal ? j : 0;
@@ -240,10 +284,17 @@ __device__ void load_role(const Params& p, Misc& ms, uint8_t* smem, int total, i
             if (!(ok = wait_bar(smem_u32(&ms.kv_empty), (item_n & 1) ^ 1, p, ms, kSiteKvEmpty))) break;
             mbar_arrive_expect_tx(smem_u32(&ms.kv_full), 2 * C::kTileBytes);
             for (int bx = 0; bx < C::kBoxes; ++bx) {
-                tma_load_4d(s_k + bx * kBoxBytes, &p.tm_k, smem_u32(&ms.kv_full), bx * 64, it.j * kBlock, it.hk, it.b,
-                            pol_keep);
-                tma_load_4d(s_v + bx * kBoxBytes, &p.tm_v, smem_u32(&ms.kv_full), bx * 64, it.j * kBlock, it.hk, it.b,
-                            pol_keep);
+                if (!p.packed) {
+                    tma_load_4d(s_k + bx * kBoxBytes, &p.tm_k, smem_u32(&ms.kv_full), bx * 64, it.j * kBlock, it.hk,
+                                it.b, pol_keep);
+                    tma_load_4d(s_v + bx * kBoxBytes, &p.tm_v, smem_u32(&ms.kv_full), bx * 64, it.j * kBlock, it.hk,
+                                it.b, pol_keep);
+                } else {
+                    tma_load_4d(s_k + bx * kBoxBytes, &p.tm_k, smem_u32(&ms.kv_full), bx * 64, it.hk,
+                                it.tok0 + it.j * kBlock, 0, pol_keep);
+                    tma_load_4d(s_v + bx * kBoxBytes, &p.tm_v, smem_u32(&ms.kv_full), bx * 64, it.hk,
+                                it.tok0 + it.j * kBlock, 0, pol_keep);
+                }
             }
             ++item_n;
         }
@@ -258,10 +309,15 @@ __device__ void load_role(const Params& p, Misc& ms, uint8_t* smem, int total, i
                 BWD_TRACE(3, ng, 1);
                 const uint32_t qbar = smem_u32(&ms.q_full[slot]);
                 mbar_arrive_expect_tx(qbar, C::kTileBytes + 2 * kBlock * 4);
-                for (int bx = 0; bx < C::kBoxes; ++bx)
-                    tma_load_4d(s_q + slot * C::kTileBytes + bx * kBoxBytes, &p.tm_q, qbar, bx * 64, i * kBlock, h, it.b,
-                                pol_keep);
-                const size_t row0 = (static_cast<size_t>(it.b) * p.Hq + h) * p.Npad + static_cast<size_t>(i) * kBlock;
+                for (int bx = 0; bx < C::kBoxes; ++bx) {
+                    if (!p.packed)
+                        tma_load_4d(s_q + slot * C::kTileBytes + bx * kBoxBytes, &p.tm_q, qbar, bx * 64, i * kBlock, h,
+                                    it.b, pol_keep);
+                    else
+                        tma_load_4d(s_q + slot * C::kTileBytes + bx * kBoxBytes, &p.tm_q, qbar, bx * 64, h,
+                                    it.tok0 + i * kBlock, 0, pol_keep);
+                }
+                const size_t row0 = vrow(it, p, h, i);
                 bulk_load(s_vec + slot * kBlock * 4, p.lse2 + row0, kBlock * 4, qbar);
                 bulk_load(s_vec + (2 + slot) * kBlock * 4, p.Dvec + row0, kBlock * 4, qbar);
             } else {
@@ -270,8 +326,12 @@ __device__ void load_role(const Params& p, Misc& ms, uint8_t* smem, int total, i
                 BWD_TRACE(3, ng, 2);
                 const uint32_t dbar = smem_u32(&ms.do_full);
                 mbar_arrive_expect_tx(dbar, C::kTileBytes);
-                for (int bx = 0; bx < C::kBoxes; ++bx)
-                    tma_load_4d(s_do + bx * kBoxBytes, &p.tm_do, dbar, bx * 64, i * kBlock, h, it.b, pol_keep);
+                for (int bx = 0; bx < C::kBoxes; ++bx) {
+                    if (!p.packed)
+                        tma_load_4d(s_do + bx * kBoxBytes, &p.tm_do, dbar, bx * 64, i * kBlock, h, it.b, pol_keep);
+                    else
+                        tma_load_4d(s_do + bx * kBoxBytes, &p.tm_do, dbar, bx * 64, h, it.tok0 + i * kBlock, 0, pol_keep);
+                }
             }
         }
     }
@@ -416,7 +476,7 @@ __device__ void pds_role(const Params& p, Misc& ms, uint8_t* smem, uint32_t tmem
         const int st = next_item(rr, p, total, it);
         if (st == 0) break;
         if (st == 2) continue;
-        const bool key_valid = it.j * kBlock + r < p.N;
+        const bool key_valid = it.j * kBlock + r < it.len;
         for (int n = 0; n < it.niter; ++n, ++ng) {
             int h, i;
             iter_of(it, n, p, h, i);
@@ -533,7 +593,7 @@ __device__ void dq_role(const Params& p, Misc& ms, uint8_t* smem, uint32_t tmem,
             tc_fence_after();
             // row r of the block's dQ share: into registers first, so that Y can
             // take the next dP before the reductions go out
-            float* dst = p.dq_acc + ((static_cast<size_t>(it.b) * p.Hq + h) * p.Npad + static_cast<size_t>(i) * kBlock + r) * D;
+            float* dst = p.dq_acc + (vrow(it, p, h, i) + r) * D;
             uint32_t v[D];
             if constexpr (D == 128) {
                 tmem_ld128_sync(ty, v);
@@ -574,7 +634,8 @@ __device__ void dq_role(const Params& p, Misc& ms, uint8_t* smem, uint32_t tmem,
         ++item_n;
         tc_fence_after();
         const int key = it.j * kBlock + r;
-        const size_t row = (static_cast<size_t>(it.b) * p.Hkv + it.hk) * p.N + key;
+        const size_t row = p.packed ? static_cast<size_t>(it.tok0 + key) * p.Hkv + it.hk
+                                    : (static_cast<size_t>(it.b) * p.Hkv + it.hk) * p.N + key;
 #pragma unroll
         for (int which = 0; which < 2; ++which) {
             const float mul = which == 0 ? 1.f : p.scale;
@@ -588,7 +649,7 @@ __device__ void dq_role(const Params& p, Misc& ms, uint8_t* smem, uint32_t tmem,
 #pragma unroll
                 for (int t = 0; t < 16; ++t)
                     pk[t] = pack_bf16x2(__uint_as_float(v[2 * t]) * mul, __uint_as_float(v[2 * t + 1]) * mul);
-                if (key < p.N) {
+                if (key < it.len) {
                     uint4* o4 = reinterpret_cast<uint4*>(out + 32 * c);
 #pragma unroll
                     for (int t = 0; t < 4; ++t) o4[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
@@ -683,13 +744,65 @@ __global__ void __launch_bounds__(kThreads, 1) fa_bwd_kernel(const __grid_consta
     }
 }
 
-// D_i = sum_c dO_ic O_ic (fp32 from bf16), lse_i * log2(e), on rows padded to
-// a multiple of 128 (padding: D = 0, lse2 = +inf so that P = 0 there); and
-// the dQ accumulator cleared.  One warp per padded row.
+// Packed batches: checks cu_seqlens and builds the schedule tables (one CTA
+// of 1024 threads, B <= 1024): the sequences ordered by key-block count
+// (longest first), the first work unit of each in that order, and the first
+// padded row of each sequence (rows rounded up to 128 per sequence).  Bad
+// offsets record FA_ERR_SEQLENS and leave no work.
+__global__ void __launch_bounds__(1024) fa_bwd_tables_kernel(const int32_t* __restrict__ cu, int B, int N, int Hkv,
+                                                             int* tab, int* status) {
+    __shared__ int nk[1024];
+    __shared__ int bad;
+    const int tid = threadIdx.x;
+    if (tid == 0) bad = (cu[0] != 0 || cu[B] != N) ? 1 : 0;
+    __syncthreads();
+    if (tid < B) {
+        const int L = cu[tid + 1] - cu[tid];
+        if (L < 0) atomicOr(&bad, 1);
+        nk[tid] = L > 0 ? (L + kBlock - 1) / kBlock : 0;
+    }
+    __syncthreads();
+    int* wu = tab;
+    int* order = tab + B + 1;
+    int* pad = tab + 2 * B + 1;
+    if (tid < B) {
+        int rank = 0;
+        for (int u = 0; u < B; ++u) rank += (nk[u] > nk[tid]) || (nk[u] == nk[tid] && u < tid);
+        order[rank] = tid;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        wu[0] = 0;
+        for (int k = 0; k < B; ++k) wu[k + 1] = wu[k] + ((nk[order[k]] + 1) / 2) * Hkv;
+        pad[0] = 0;
+        for (int q = 0; q < B; ++q) pad[q + 1] = pad[q] + nk[q] * kBlock;
+        tab[3 * B + 2] = bad ? 0 : wu[B];
+        tab[3 * B + 3] = bad ? -1 : pad[B];       // -1: offsets rejected
+        if (bad) atomicCAS(status, 0, FA_ERR_SEQLENS);
+    }
+}
+
+// Largest s in [0, n) with a[s] <= x (a non-decreasing, a[0] <= x).
+__device__ __forceinline__ int last_le(const int* a, int n, long long x) {
+    int lo = 0, hi = n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (a[mid] <= x) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// D_i = sum_c dO_ic O_ic (fp32 from bf16), lse_i * log2(e), on the padded
+// rows (padding: D = 0, lse2 = +inf so that P = 0 there); and the dQ
+// accumulator cleared.  One warp per padded row.  Dense: rows [B, Hq, Npad],
+// O / dO [B, Hq, N, d], lse [B, Hq, N].  Packed: rows [Hq, Npad], O / dO
+// [N, Hq, d], lse [Hq, N].
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
                                                           const float* __restrict__ lse, float* lse2, float* Dvec,
-                                                          float* dq_acc, int N, int Npad, long long rows_pad) {
+                                                          float* dq_acc, int N, int Npad, long long rows_pad,
+                                                          const int32_t* __restrict__ cu, const int* __restrict__ tab,
+                                                          int B, int Hq) {
     const long long row = static_cast<long long>(blockIdx.x) * 8 + threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     if (row >= rows_pad) return;
@@ -697,9 +810,24 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const uint16_t* __rest
     const int t = static_cast<int>(row - bh * Npad);
     float* acc = dq_acc + row * D;
     for (int c = lane * 4; c < D; c += 128) *reinterpret_cast<float4*>(acc + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+    bool valid;
+    size_t src, lrow;
+    if (!cu) {
+        valid = t < N;
+        src = (static_cast<size_t>(bh) * N + t) * D;
+        lrow = static_cast<size_t>(bh) * N + t;
+    } else {
+        const int* pad = tab + 2 * B + 1;
+        const int sq = last_le(pad, B, t);
+        const int tt = t - pad[sq];
+        const int len = cu[sq + 1] - cu[sq];
+        valid = tab[3 * B + 3] >= 0 && t < pad[B] && tt >= 0 && tt < len;
+        const size_t token = static_cast<size_t>(cu[sq]) + tt;
+        src = (token * Hq + bh) * D;                 // bh is the head here
+        lrow = static_cast<size_t>(bh) * N + token;
+    }
     float dsum = 0.f;
-    if (t < N) {
-        const size_t src = (static_cast<size_t>(bh) * N + t) * D;
+    if (valid) {
         for (int c = lane * 2; c < D; c += 64) {
             const uint32_t ov = *reinterpret_cast<const uint32_t*>(o + src + c);
             const uint32_t dv = *reinterpret_cast<const uint32_t*>(dout + src + c);
@@ -711,27 +839,40 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const uint16_t* __rest
     for (int off = 16; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
     if (lane == 0) {
         float l2 = INFINITY;
-        if (t < N) {
-            const float l = lse[static_cast<size_t>(bh) * N + t];
+        if (valid) {
+            const float l = lse[lrow];
             l2 = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
         }
         lse2[row] = l2;
-        Dvec[row] = t < N ? dsum : 0.f;
+        Dvec[row] = valid ? dsum : 0.f;
     }
 }
 
-// dQ = scale * accumulator -> bf16, rows < N.  One thread per 4 values.
+// dQ = scale * accumulator -> bf16.  One thread per 4 values of dq (dense
+// [B, Hq, N, d]; packed [N, Hq, d]).
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float* __restrict__ dq_acc, uint16_t* dq, float scale,
-                                                        int N, int Npad, long long total4) {
+                                                        int N, int Npad, long long total4, const int32_t* __restrict__ cu,
+                                                        const int* __restrict__ tab, int B, int Hq) {
     const long long e4 = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
     if (e4 >= total4) return;
     const long long e = e4 * 4;
-    const long long row = e / D;               // row of [B*Hq, N]
+    const long long row = e / D;
     const int c = static_cast<int>(e - row * D);
-    const long long bh = row / N;
-    const long long t = row - bh * N;
-    const float4 v = *reinterpret_cast<const float4*>(dq_acc + (bh * Npad + t) * D + c);
+    size_t arow;
+    if (!cu) {
+        const long long bh = row / N;              // row of [B*Hq, N]
+        const long long t = row - bh * N;
+        arow = static_cast<size_t>(bh) * Npad + t;
+    } else {
+        if (tab[3 * B + 3] < 0) return;            // offsets rejected: dq is left unwritten
+        const long long token = row / Hq;          // row of [N, Hq]
+        const int h = static_cast<int>(row - token * Hq);
+        const int sq = last_le(cu, B, token);
+        const int* pad = tab + 2 * B + 1;
+        arow = static_cast<size_t>(h) * Npad + pad[sq] + (token - cu[sq]);
+    }
+    const float4 v = *reinterpret_cast<const float4*>(dq_acc + arow * D + c);
     *reinterpret_cast<uint2*>(dq + e) = make_uint2(pack_bf16x2(v.x * scale, v.y * scale), pack_bf16x2(v.z * scale, v.w * scale));
 }
 
@@ -750,9 +891,18 @@ static int bwd_setup(int dev) {
     return FA_OK;
 }
 
-static size_t workspace_bytes(int B, int Hq, int N, int d) {
-    const size_t npad = (static_cast<size_t>(N) + kBlock - 1) / kBlock * kBlock;
-    return static_cast<size_t>(B) * Hq * npad * (d + 2) * sizeof(float);
+// Padded rows per head: dense, N rounded up to 128; packed, a bound on the
+// sum over sequences of their lengths rounded up to 128.
+static size_t padded_rows(int B, int N, bool packed) {
+    const size_t n = packed ? static_cast<size_t>(N) + static_cast<size_t>(kBlock) * B : static_cast<size_t>(N);
+    return (n + kBlock - 1) / kBlock * kBlock;
+}
+
+static size_t workspace_bytes(int B, int Hq, int N, int d, bool packed) {
+    const size_t rows = (packed ? 1 : static_cast<size_t>(B)) * Hq * padded_rows(B, N, packed);
+    size_t bytes = rows * (d + 2) * sizeof(float);
+    if (packed) bytes += (static_cast<size_t>(3) * B + 4) * sizeof(int);
+    return bytes;
 }
 
 static bool aligned(const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) == 0; }
@@ -769,27 +919,33 @@ extern "C" int fa_bwd_trace_set(void* ptr) {
 }
 #endif
 
-extern "C" size_t fa_bwd_workspace_bytes(int B, int Hq, int N, int d) {
+extern "C" size_t fa_bwd_workspace_bytes(int B, int Hq, int N, int d, int packed) {
     if (B < 0 || Hq < 1 || N < 0 || (d != 64 && d != 128)) return 0;
-    return bwd::workspace_bytes(B, Hq, N, d);
+    if (packed && B > bwd::kMaxSeqsBwd) return 0;
+    return bwd::workspace_bytes(B, Hq, N, d, packed != 0);
 }
 
 extern "C" int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                       void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, float scale, int causal,
-                      void* workspace, size_t workspace_bytes, void* stream) {
+                      const int32_t* cu_seqlens, void* workspace, size_t workspace_bytes, void* stream) {
     using namespace bwd;
+    const bool packed = cu_seqlens != nullptr;
     if (B < 0 || N < 0 || Hq < 1) return FA_ERR_SHAPE;
     if (d != 64 && d != 128) return FA_ERR_HEADDIM;
     if (Hkv < 1 || Hq % Hkv != 0) return FA_ERR_GQA;
     if (B == 0 || N == 0) return FA_OK;
+    if (packed && B > kMaxSeqsBwd) return FA_ERR_SHAPE;
     if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return FA_ERR_NULL;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
-        !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) || !aligned(workspace, 16))
+        !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) || !aligned(workspace, 16) ||
+        (packed && !aligned(cu_seqlens, 4)))
         return FA_ERR_ALIGN;
-    const long long npad = (static_cast<long long>(N) + kBlock - 1) / kBlock * kBlock;
-    if ((long long)B * Hq * npad > (1ll << 30) || (long long)B * Hkv * ((N + kBlock - 1) / kBlock) > (1ll << 30))
+    const long long npad = (long long)padded_rows(B, N, packed);
+    const long long rows_pad = (packed ? 1ll : (long long)B) * Hq * npad;
+    if (rows_pad > (1ll << 30) || (long long)B * Hkv * ((N + kBlock - 1) / kBlock) > (1ll << 30) ||
+        (long long)Hq * N > (1ll << 30))
         return FA_ERR_SHAPE;
-    if (workspace_bytes < bwd::workspace_bytes(B, Hq, N, d)) return FA_ERR_SHAPE;
+    if (workspace_bytes < bwd::workspace_bytes(B, Hq, N, d, packed)) return FA_ERR_SHAPE;
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_LAUNCH;
@@ -799,27 +955,41 @@ extern "C" int fa_bwd(const void* q, const void* k, const void* v, const void* o
     if ((st = bwd_setup(dev)) != FA_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-    const long long rows_pad = (long long)B * Hq * npad;
     float* dq_acc = static_cast<float*>(workspace);
     float* lse2 = dq_acc + rows_pad * d;
     float* Dvec = lse2 + rows_pad;
+    int* tab = packed ? reinterpret_cast<int*>(Dvec + rows_pad) : nullptr;
 
     Params P;
     std::memset(&P, 0, sizeof(P));
     {
         const uint64_t e = 2;
-        const uint32_t box[4] = {64, (uint32_t)kBlock, 1, 1};
-        const uint64_t dq_[4] = {(uint64_t)d, (uint64_t)N, (uint64_t)Hq, (uint64_t)B};
-        const uint64_t sq[3] = {d * e, (uint64_t)N * d * e, (uint64_t)Hq * N * d * e};
-        const uint64_t dk_[4] = {(uint64_t)d, (uint64_t)N, (uint64_t)Hkv, (uint64_t)B};
-        const uint64_t sk[3] = {d * e, (uint64_t)N * d * e, (uint64_t)Hkv * N * d * e};
-        if (!encode_map(&P.tm_q, q, dq_, sq, box) || !encode_map(&P.tm_do, dout, dq_, sq, box) ||
-            !encode_map(&P.tm_k, k, dk_, sk, box) || !encode_map(&P.tm_v, v, dk_, sk, box))
-            return FA_ERR_LAUNCH;
+        bool good;
+        if (!packed) {
+            const uint32_t box[4] = {64, (uint32_t)kBlock, 1, 1};
+            const uint64_t dq_[4] = {(uint64_t)d, (uint64_t)N, (uint64_t)Hq, (uint64_t)B};
+            const uint64_t sq[3] = {d * e, (uint64_t)N * d * e, (uint64_t)Hq * N * d * e};
+            const uint64_t dk_[4] = {(uint64_t)d, (uint64_t)N, (uint64_t)Hkv, (uint64_t)B};
+            const uint64_t sk[3] = {d * e, (uint64_t)N * d * e, (uint64_t)Hkv * N * d * e};
+            good = encode_map(&P.tm_q, q, dq_, sq, box) && encode_map(&P.tm_do, dout, dq_, sq, box) &&
+                   encode_map(&P.tm_k, k, dk_, sk, box) && encode_map(&P.tm_v, v, dk_, sk, box);
+        } else {
+            // token-major [N, H, d]: 128 tokens of one head per box
+            const uint32_t box[4] = {64, 1, (uint32_t)kBlock, 1};
+            const uint64_t dq_[4] = {(uint64_t)d, (uint64_t)Hq, (uint64_t)N, 1};
+            const uint64_t sq[3] = {d * e, (uint64_t)Hq * d * e, (uint64_t)N * Hq * d * e};
+            const uint64_t dk_[4] = {(uint64_t)d, (uint64_t)Hkv, (uint64_t)N, 1};
+            const uint64_t sk[3] = {d * e, (uint64_t)Hkv * d * e, (uint64_t)N * Hkv * d * e};
+            good = encode_map(&P.tm_q, q, dq_, sq, box) && encode_map(&P.tm_do, dout, dq_, sq, box) &&
+                   encode_map(&P.tm_k, k, dk_, sk, box) && encode_map(&P.tm_v, v, dk_, sk, box);
+        }
+        if (!good) return FA_ERR_LAUNCH;
     }
     P.lse2 = lse2;
     P.Dvec = Dvec;
     P.dq_acc = dq_acc;
+    P.cu = cu_seqlens;
+    P.tab = tab;
     P.dk = static_cast<uint16_t*>(dk);
     P.dv = static_cast<uint16_t*>(dv);
     P.status = ds->status;
@@ -830,28 +1000,33 @@ extern "C" int fa_bwd(const void* q, const void* k, const void* v, const void* o
     P.Npad = (int)npad;
     P.group = Hq / Hkv;
     P.causal = causal ? 1 : 0;
+    P.packed = packed ? 1 : 0;
     P.scale = scale;
     P.scale_log2 = scale * 1.4426950408889634f;
     P.timeout_ns = 2000000000ull;
 
+    if (packed) fa_bwd_tables_kernel<<<1, 1024, 0, s>>>(cu_seqlens, B, N, Hkv, tab, ds->status);
     const unsigned prep_grid = static_cast<unsigned>((rows_pad + 7) / 8);
-    const long long units = (long long)B * Hkv * (((N + kBlock - 1) / kBlock + 1) / 2);
+    // dense: the exact number of work units; packed: one CTA per SM (the count is on the device)
+    const long long units = packed ? (long long)ds->num_sms
+                                   : (long long)B * Hkv * (((N + kBlock - 1) / kBlock + 1) / 2);
     const int grid = (int)std::min<long long>(units, ds->num_sms);
-    const long long total4 = (long long)B * Hq * N * d / 4;
+    const long long total4 = (packed ? (long long)N * Hq : (long long)B * Hq * N) * d / 4;
     const unsigned post_grid = static_cast<unsigned>((total4 + 255) / 256);
+    const uint16_t* o16 = static_cast<const uint16_t*>(o);
+    const uint16_t* do16 = static_cast<const uint16_t*>(dout);
     if (d == 64) {
-        fa_bwd_prep_kernel<64><<<prep_grid, 256, 0, s>>>(static_cast<const uint16_t*>(o),
-                                                          static_cast<const uint16_t*>(dout), lse, lse2, Dvec, dq_acc,
-                                                          N, (int)npad, rows_pad);
+        fa_bwd_prep_kernel<64><<<prep_grid, 256, 0, s>>>(o16, do16, lse, lse2, Dvec, dq_acc, N, (int)npad, rows_pad,
+                                                          cu_seqlens, tab, B, Hq);
         fa_bwd_kernel<64><<<grid, kThreads, Cfg<64>::kSmemBytes, s>>>(P);
-        fa_bwd_dq_kernel<64><<<post_grid, 256, 0, s>>>(dq_acc, static_cast<uint16_t*>(dq), scale, N, (int)npad, total4);
+        fa_bwd_dq_kernel<64><<<post_grid, 256, 0, s>>>(dq_acc, static_cast<uint16_t*>(dq), scale, N, (int)npad, total4,
+                                                        cu_seqlens, tab, B, Hq);
     } else {
-        fa_bwd_prep_kernel<128><<<prep_grid, 256, 0, s>>>(static_cast<const uint16_t*>(o),
-                                                           static_cast<const uint16_t*>(dout), lse, lse2, Dvec, dq_acc,
-                                                           N, (int)npad, rows_pad);
+        fa_bwd_prep_kernel<128><<<prep_grid, 256, 0, s>>>(o16, do16, lse, lse2, Dvec, dq_acc, N, (int)npad, rows_pad,
+                                                           cu_seqlens, tab, B, Hq);
         fa_bwd_kernel<128><<<grid, kThreads, Cfg<128>::kSmemBytes, s>>>(P);
         fa_bwd_dq_kernel<128><<<post_grid, 256, 0, s>>>(dq_acc, static_cast<uint16_t*>(dq), scale, N, (int)npad,
-                                                        total4);
+                                                         total4, cu_seqlens, tab, B, Hq);
     }
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }

@@ -204,9 +204,9 @@ int fa_splitkv_num_splits(int B, int Hq, int Hkv, int Nq, int Nk, int d);
 size_t fa_splitkv_workspace_bytes(int B, int Hq, int Nq, int d, int num_splits);
 
 /*
- * fa_bwd -- gradients of fa_fwd (dense batches), asynchronous on `stream`.
- * The backward pass recomputes the scores block by block from Q and K and the
- * logsumexp that fa_fwd saved, instead of storing them ("Flash Attention",
+ * fa_bwd -- gradients of fa_fwd, asynchronous on `stream`.  The backward
+ * pass recomputes the scores block by block from Q and K and the logsumexp
+ * that fa_fwd saved, instead of storing them ("Flash Attention",
  * 14cs17.netlify.app, "Common Pitfalls", Pitfall 3; fromzero2ai.dev, "Core
  * Mechanisms of FlashAttention", item 3).  The gradients are those of the
  * forward's definition: with P = softmax(scale Q K^T) (masked) and the
@@ -220,38 +220,46 @@ size_t fa_splitkv_workspace_bytes(int B, int Hq, int Nq, int d, int num_splits);
  *   dout              bf16 upstream gradient, same layout as o.
  *   dq                bf16 output, layout of q.
  *   dk, dv            bf16 outputs, layout of k (written, not accumulated).
+ *   B, Hq, Hkv, N, d, scale, causal, cu_seqlens
+ *                     as fa_fwd: dense (cu_seqlens NULL) q, o, dout, dq
+ *                     [B, Hq, N, d], k, v, dk, dv [B, Hkv, N, d], lse
+ *                     [B, Hq, N]; packed (cu_seqlens: B+1 device offsets,
+ *                     at most 1024 sequences) q, o, dout, dq [N, Hq, d],
+ *                     k, v, dk, dv [N, Hkv, d], lse [Hq, N].
  *   workspace         device memory, 16-byte aligned, at least
- *                     fa_bwd_workspace_bytes(B, Hq, N, d) bytes: an fp32 dQ
- *                     accumulator and two per-row fp32 vectors, on rows padded
- *                     to a multiple of 128.  Nothing in it needs initialising;
- *                     it must not be used by anything else until the call's
- *                     kernels have finished on `stream`.
- *   B, Hq, Hkv, N, d, scale, causal   as fa_fwd (dense layout only:
- *                     q, o, dout, dq [B, Hq, N, d]; k, v, dk, dv
- *                     [B, Hkv, N, d]; lse [B, Hq, N]).
+ *                     fa_bwd_workspace_bytes(B, Hq, N, d, packed) bytes: an
+ *                     fp32 dQ accumulator and two per-row fp32 vectors on rows
+ *                     padded to 128 per sequence (packed: and the schedule
+ *                     tables).  Nothing in it needs initialising; it must not
+ *                     be used by anything else until the call's kernels have
+ *                     finished on `stream`.
  *
- * Three kernels run on `stream`: a pass computing D and clearing the
- * accumulator, the main kernel (one 128-key block of one (batch, kv head)
- * per work item, dK and dV kept in tensor memory, each block's dQ share
- * added into the accumulator with fp32 reductions), and the dQ conversion.
- * The order of the fp32 reductions varies from run to run, so dQ may differ
- * in its last bits between runs; dK and dV do not.
+ * Kernels on `stream`: (packed) a table pass that checks cu_seqlens and
+ * orders the sequences longest first, a pass computing D and clearing the
+ * accumulator, the main kernel (one 128-key block of one (sequence, kv head)
+ * per work item, dK and dV kept in tensor memory, each block's dQ share added
+ * into the accumulator with fp32 reductions), and the dQ conversion.  The
+ * order of the fp32 reductions varies from run to run, so dQ may differ in
+ * its last bits between runs; dK and dV do not.
  *
  * Errors as fa_fwd (FA_ERR_NULL also for a missing workspace, FA_ERR_ALIGN for
- * a misaligned one, FA_ERR_SHAPE for one that is too small).  B == 0 or N == 0
- * is an empty problem (FA_OK, nothing launched).
+ * a misaligned one, FA_ERR_SHAPE for one that is too small or more than 1024
+ * sequences; inconsistent cu_seqlens are reported on the device as
+ * FA_ERR_SEQLENS and leave the outputs unwritten).  B == 0 or N == 0 is an
+ * empty problem (FA_OK, nothing launched).
  */
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
            const void* dout, void* dq, void* dk, void* dv,
            int B, int Hq, int Hkv, int N, int d, float scale, int causal,
-           void* workspace, size_t workspace_bytes, void* stream);
+           const int32_t* cu_seqlens, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * fa_bwd_workspace_bytes -- workspace fa_bwd needs:
- * B * Hq * Npad * (d + 2) * 4 bytes with Npad = N rounded up to 128; 0 for
- * invalid arguments.  Needs no device.
+ * fa_bwd_workspace_bytes -- workspace fa_bwd needs.  Dense (packed == 0):
+ * B * Hq * Npad * (d + 2) * 4 bytes with Npad = N rounded up to 128.
+ * Packed: Hq * Npad * (d + 2) * 4 + (3 B + 4) * 4 bytes with Npad = N + 128 B
+ * rounded up to 128.  0 for invalid arguments.  Needs no device.
  */
-size_t fa_bwd_workspace_bytes(int B, int Hq, int N, int d);
+size_t fa_bwd_workspace_bytes(int B, int Hq, int N, int d, int packed);
 
 /*
  * fa_get_device_status -- reads and clears the status word of the current

@@ -111,9 +111,12 @@ def test_bwd_argument_errors_and_workspace_bytes():
     assert fa.fa_bwd_workspace_bytes(2, 4, 300, 128) == 2 * 4 * 384 * 130 * 4
     assert fa.fa_bwd_workspace_bytes(1, 1, 128, 64) == 128 * 66 * 4
     assert fa.fa_bwd_workspace_bytes(1, 1, 128, 96) == 0
+    # packed: Hq * Npad * (d + 2) * 4 + (3 B + 4) * 4 with Npad = N + 128 B rounded up to 128
+    assert fa.fa_bwd_workspace_bytes(3, 4, 300, 128, True) == 4 * 768 * 130 * 4 + (3 * 3 + 4) * 4
+    assert fa.fa_bwd_workspace_bytes(1025, 4, 300, 128, True) == 0
 
-    def call(ptrs=(p,) * 9, ws=p, wb=1 << 30, B=1, Hq=4, Hkv=2, N=100, d=128):
-        return fa.fa_bwd(*ptrs, B, Hq, Hkv, N, d, 0.1, 1, ws, wb)
+    def call(ptrs=(p,) * 9, ws=p, wb=1 << 30, B=1, Hq=4, Hkv=2, N=100, d=128, cu=None):
+        return fa.fa_bwd(*ptrs, B, Hq, Hkv, N, d, 0.1, 1, cu, ws, wb)
 
     assert call(d=96) == fa.FA_ERR_HEADDIM
     assert call(Hkv=3) == fa.FA_ERR_GQA
@@ -124,6 +127,9 @@ def test_bwd_argument_errors_and_workspace_bytes():
     assert call(ptrs=(p + 2,) + (p,) * 8) == fa.FA_ERR_ALIGN
     assert call(wb=fa.fa_bwd_workspace_bytes(1, 4, 100, 128) - 16) == fa.FA_ERR_SHAPE
     assert call(B=0, ptrs=(0,) * 9, ws=0, wb=0) == fa.FA_OK
+    assert call(B=1025, cu=p) == fa.FA_ERR_SHAPE
+    assert call(cu=p + 2) == fa.FA_ERR_ALIGN
+    assert call(B=3, cu=p, wb=fa.fa_bwd_workspace_bytes(3, 4, 100, 128, True) - 4) == fa.FA_ERR_SHAPE
 
 
 def test_fp8_argument_errors_found_on_the_host():
