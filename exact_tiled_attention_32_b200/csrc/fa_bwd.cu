@@ -90,7 +90,7 @@ constexpr uint32_t kColX = 0, kColY = 128, kColDV = 256, kColDK = 384;
 
 enum WaitSite : int {
     kSiteKvEmpty = 11, kSiteKvFull, kSiteQEmpty, kSiteQFull, kSiteDoEmpty, kSiteDoFull, kSiteS, kSiteP, kSiteDp,
-    kSiteDs, kSiteDsFree, kSiteDq, kSiteYFree, kSiteAccDone, kSiteAccFree, kSiteAlign, kSiteStage
+    kSiteDs, kSiteDsFree, kSiteDq, kSiteYFree, kSiteAccDone, kSiteAccFree, kSiteAlign
 };
 
 struct alignas(64) Params {
