@@ -255,6 +255,10 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Pa
         }
     }
 }
+// wait_bar on every lane of a warp, with one verdict for the whole warp
+__device__ __forceinline__ bool wait_all(uint32_t bar, uint32_t parity, const Params& p, Misc& ms, int site) {
+    return __all_sync(0xffffffffu, wait_bar(bar, parity, p, ms, site));
+}
 __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, const Params& p) {
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(bar, parity)) {
@@ -357,6 +361,8 @@ __device__ __forceinline__ void mma_qk(uint32_t d_tmem, uint64_t a, uint64_t b) 
         umma_ss_k64_x4(d_tmem, a, b, idesc);
 }
 
+// The MMA issuer: all 32 lanes of the warp run the loop (waits included); one
+// elected lane issues each batch of MMAs and commits.
 template <int D>
 __device__ void mma_role(const Params& p, Misc& ms, uint8_t* smem, uint32_t tmem, int total) {
     using C = Cfg<D>;
@@ -382,71 +388,91 @@ __device__ void mma_role(const Params& p, Misc& ms, uint8_t* smem, uint32_t tmem
         const int st = next_item(r, p, total, it);
         if (st == 0) break;
         if (st == 2) continue;
-        if (!(ok = wait_bar(smem_u32(&ms.kv_full), item_n & 1, p, ms, kSiteKvFull))) break;
+        if (!(ok = wait_all(smem_u32(&ms.kv_full), item_n & 1, p, ms, kSiteKvFull))) break;
         tc_fence_after();
         for (int n = 0; n < it.niter && ok; ++n, ++ng) {
             const uint32_t slot = ng & 1;
             if (n == 0) {          // S^T of the item's first block
-                if (!(ok = wait_bar(smem_u32(&ms.q_full[slot]), (ng >> 1) & 1, p, ms, kSiteQFull))) break;
+                if (!(ok = wait_all(smem_u32(&ms.q_full[slot]), (ng >> 1) & 1, p, ms, kSiteQFull))) break;
                 tc_fence_after();
-                mma_qk<D>(tmem + kColX, dk_k, dq_k0 + slot * kTileStep);
-                umma_commit(smem_u32(&ms.s_full));
+                if (elect_one()) {
+                    mma_qk<D>(tmem + kColX, dk_k, dq_k0 + slot * kTileStep);
+                    umma_commit(smem_u32(&ms.s_full));
+                }
+                __syncwarp();
             }
             // dP^T = V_j dO_i^T (once the previous dQ share has left Y) and
             // dV_j += P^T dO_i (once P^T is in TMEM), whichever is ready first
             BWD_TRACE(0, ng, 0);
-            if (!(ok = wait_bar(smem_u32(&ms.do_full), ng & 1, p, ms, kSiteDoFull))) break;
+            if (!(ok = wait_all(smem_u32(&ms.do_full), ng & 1, p, ms, kSiteDoFull))) break;
             BWD_TRACE(0, ng, 1);
             const uint64_t ddo_k = ddo_k0, ddo_mn = ddo_mn0;
             bool dp_issued = false;
-            if (mbar_try_wait(smem_u32(&ms.y_free), (ng & 1) ^ 1)) {
+            if (__all_sync(0xffffffffu, mbar_try_wait(smem_u32(&ms.y_free), (ng & 1) ^ 1))) {
                 tc_fence_after();
-                mma_qk<D>(tmem + kColY, dv_k, ddo_k);
-                umma_commit(smem_u32(&ms.dp_full));
+                if (elect_one()) {
+                    mma_qk<D>(tmem + kColY, dv_k, ddo_k);
+                    umma_commit(smem_u32(&ms.dp_full));
+                }
+                __syncwarp();
                 dp_issued = true;
             }
-            if (!(ok = wait_bar(smem_u32(&ms.p_full), ng & 1, p, ms, kSiteP))) break;
+            if (!(ok = wait_all(smem_u32(&ms.p_full), ng & 1, p, ms, kSiteP))) break;
             BWD_TRACE(0, ng, 2);
-            if (n == 0 && !(ok = wait_bar(smem_u32(&ms.acc_free), (item_n & 1) ^ 1, p, ms, kSiteAccFree))) break;
+            if (n == 0 && !(ok = wait_all(smem_u32(&ms.acc_free), (item_n & 1) ^ 1, p, ms, kSiteAccFree))) break;
             tc_fence_after();
-            umma_ts_kv128_x8(tmem + kColDV, tmem + kColX, ddo_mn, id_dv, n > 0 ? 1u : 0u);
+            if (elect_one()) umma_ts_kv128_x8(tmem + kColDV, tmem + kColX, ddo_mn, id_dv, n > 0 ? 1u : 0u);
+            __syncwarp();
             if (!dp_issued) {
-                if (!(ok = wait_bar(smem_u32(&ms.y_free), (ng & 1) ^ 1, p, ms, kSiteYFree))) break;
+                if (!(ok = wait_all(smem_u32(&ms.y_free), (ng & 1) ^ 1, p, ms, kSiteYFree))) break;
                 tc_fence_after();
-                mma_qk<D>(tmem + kColY, dv_k, ddo_k);
-                umma_commit(smem_u32(&ms.dp_full));
+                if (elect_one()) {
+                    mma_qk<D>(tmem + kColY, dv_k, ddo_k);
+                    umma_commit(smem_u32(&ms.dp_full));
+                }
+                __syncwarp();
             }
-            umma_commit(smem_u32(&ms.do_empty));
+            if (elect_one()) umma_commit(smem_u32(&ms.do_empty));
+            __syncwarp();
             BWD_TRACE(0, ng, 3);
             // S^T of the next block (X is free once dV has read P^T: in order)
             if (n + 1 < it.niter) {
                 const uint32_t ns = (ng + 1) & 1;
-                if (!(ok = wait_bar(smem_u32(&ms.q_full[ns]), ((ng + 1) >> 1) & 1, p, ms, kSiteQFull))) break;
+                if (!(ok = wait_all(smem_u32(&ms.q_full[ns]), ((ng + 1) >> 1) & 1, p, ms, kSiteQFull))) break;
                 tc_fence_after();
-                mma_qk<D>(tmem + kColX, dk_k, dq_k0 + ns * kTileStep);
-                umma_commit(smem_u32(&ms.s_full));
+                if (elect_one()) {
+                    mma_qk<D>(tmem + kColX, dk_k, dq_k0 + ns * kTileStep);
+                    umma_commit(smem_u32(&ms.s_full));
+                }
+                __syncwarp();
             }
             // dK_j += dS^T Q_i and dQ_i share = dS K_j, once dS is in shared memory
             BWD_TRACE(0, ng, 4);
-            if (!(ok = wait_bar(smem_u32(&ms.ds_full), ng & 1, p, ms, kSiteDs))) break;
+            if (!(ok = wait_all(smem_u32(&ms.ds_full), ng & 1, p, ms, kSiteDs))) break;
             BWD_TRACE(0, ng, 5);
             tc_fence_after();
             // dQ first: the dQ warpgroup can start reading Y while dK runs
-            umma_ss_mnA_mnB_k128_x8(tmem + kColY, dds_mn, dk_mn, id_dq);
-            umma_commit(smem_u32(&ms.dq_full));
-            umma_ss_kA_mnB_k128_x8(tmem + kColDK, dds_k, dq_mn0 + slot * kTileStep, id_dk, n > 0 ? 1u : 0u);
-            umma_commit(smem_u32(&ms.ds_free));
-            umma_commit(smem_u32(&ms.q_empty[slot]));
+            if (elect_one()) {
+                umma_ss_mnA_mnB_k128_x8(tmem + kColY, dds_mn, dk_mn, id_dq);
+                umma_commit(smem_u32(&ms.dq_full));
+                umma_ss_kA_mnB_k128_x8(tmem + kColDK, dds_k, dq_mn0 + slot * kTileStep, id_dk, n > 0 ? 1u : 0u);
+                umma_commit(smem_u32(&ms.ds_free));
+                umma_commit(smem_u32(&ms.q_empty[slot]));
+            }
+            __syncwarp();
             BWD_TRACE(0, ng, 6);
             if (dp_issued) BWD_TRACE(0, ng, 7);
-            if (n == it.niter - 1) {
+            if (n == it.niter - 1 && elect_one()) {
                 umma_commit(smem_u32(&ms.acc_done));
                 umma_commit(smem_u32(&ms.kv_empty));
             }
+            __syncwarp();
         }
         ++item_n;
     }
-    umma_commit(smem_u32(&ms.drain));
+    __syncwarp();
+    if (elect_one()) umma_commit(smem_u32(&ms.drain));
+    __syncwarp();
     drain_bar(smem_u32(&ms.drain), 0, p);
 }
 
@@ -726,7 +752,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_bwd_kernel(const __grid_consta
     } else {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
         if (warp == kMmaWarp) {
-            if (lane == 0) mma_role<D>(p, ms, smem, tmem, total);
+            mma_role<D>(p, ms, smem, tmem, total);      // all 32 lanes
             __syncwarp();
         } else if (warp == kLoadWarp) {
             if (lane == 0) load_role<D>(p, ms, smem, total, 0);

@@ -90,7 +90,8 @@ struct alignas(64) Params {
 
 // Optional pipeline timeline (compile with -DFA_TRACE): CTA 0 records clock64
 // stamps per role and iteration into Params::trace, laid out as
-// [role][iteration][event], kTraceIters iterations and 8 events per role.
+// [role][iteration][event], kTraceIters iterations and 8 events per role
+// (roles 0, 1: the softmax warpgroups; 2, 3: the MMA issuer).
 [[maybe_unused]] constexpr int kTraceIters = 1024;
 #ifdef FA_TRACE
 #define FA_TRACE_EV(role, it, ev)                                                              \
@@ -279,6 +280,10 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Pa
         }
     }
 }
+// wait_bar on every lane of a warp, with one verdict for the whole warp
+__device__ __forceinline__ bool wait_all(uint32_t bar, uint32_t parity, const Params& p, Misc& ms, int site) {
+    return __all_sync(0xffffffffu, wait_bar(bar, parity, p, ms, site));
+}
 // Teardown wait: ignores the abort flag, still bounded.
 __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, const Params& p) {
     const uint64_t t0 = globaltimer_ns();
@@ -383,6 +388,8 @@ __device__ __forceinline__ void issue_pv_half(uint32_t tmem_o, uint32_t tmem_p, 
 // block count of the two tiles): O_t += P_t V_{j-1} for each tile that had
 // block j-1, then S_t = Q_t K_j^T for each tile that has block j, tile 0
 // before tile 1 -- the order that keeps the two softmax warpgroups out of phase.
+// All 32 lanes of the warp run the loop (waits included); one elected lane
+// issues each batch of MMAs and commits.
 template <int D, bool PK, bool F8 = false>
 __device__ void mma_role(const Params& p, Misc& ms, const SeqTables& tab, uint32_t tmem, uint32_t smem_q,
                          uint32_t smem_kv, int total) {
@@ -402,7 +409,7 @@ __device__ void mma_role(const Params& p, Misc& ms, const SeqTables& tab, uint32
         if (idx >= total) break;
         const Item it = decode_item<PK>(idx, p, ms, tab);
         if (max(it.n[0], it.n[1]) == 0) continue;      // a split with no key block
-        if (!(ok = wait_bar(smem_u32(&ms.bar_q_full), item_n & 1, p, ms, kSiteQFull))) break;
+        if (!(ok = wait_all(smem_u32(&ms.bar_q_full), item_n & 1, p, ms, kSiteQFull))) break;
         tc_fence_after();
         ++item_n;
         const int nmax = max(it.n[0], it.n[1]);
@@ -411,7 +418,7 @@ __device__ void mma_role(const Params& p, Misc& ms, const SeqTables& tab, uint32
             // V_{j-1} sits one ring position before K_j
             const uint32_t vst = kst == 0 ? C::kStages - 1 : kst - 1;
             const uint32_t vph = kst == 0 ? kph ^ 1u : kph;
-            if (j > 0 && !(ok = wait_bar(smem_u32(&ms.bar_kv_full[vst]), vph, p, ms, kSiteKvFull))) break;
+            if (j > 0 && !(ok = wait_all(smem_u32(&ms.bar_kv_full[vst]), vph, p, ms, kSiteKvFull))) break;
             bool k_ready = false;
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
@@ -419,31 +426,41 @@ __device__ void mma_role(const Params& p, Misc& ms, const SeqTables& tab, uint32
                 if (j > 0 && j - 1 < it.n[t]) {          // O_t += P_t V_{j-1}, in two key halves
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        if (!(ok = wait_bar(smem_u32(&ms.bar_p_half[t][h]), pc[t] & 1, p, ms, kSitePFull))) break;
+                        if (!(ok = wait_all(smem_u32(&ms.bar_p_half[t][h]), pc[t] & 1, p, ms, kSitePFull))) break;
                         tc_fence_after();
+                        FA_TRACE_EV(3, (item_n == 1 ? j : kTraceIters), 2 * t + h);
                         if (h == 0) FA_TRACE_EV(2, (item_n == 1 ? j : kTraceIters), 2 + 2 * t);
-                        issue_pv_half<D, F8>(tmem + 256 + t * 128, tmem + t * 128, dv0 + vst * kTileStep, h,
-                                             h > 0 || j - 1 > 0);
+                        if (elect_one())
+                            issue_pv_half<D, F8>(tmem + 256 + t * 128, tmem + t * 128, dv0 + vst * kTileStep, h,
+                                                 h > 0 || j - 1 > 0);
+                        __syncwarp();
                     }
                     if (!ok) break;
                     ++pc[t];
-                    if (j - 1 == it.n[t] - 1) umma_commit(smem_u32(&ms.bar_o_final[t]));
+                    if (j - 1 == it.n[t] - 1 && elect_one()) umma_commit(smem_u32(&ms.bar_o_final[t]));
+                    __syncwarp();
                 }
                 if (j < it.n[t]) {                       // S_t = Q_t K_j^T
                     if (!k_ready) {
-                        if (!(ok = wait_bar(smem_u32(&ms.bar_kv_full[kst]), kph, p, ms, kSiteKvFull))) break;
+                        if (!(ok = wait_all(smem_u32(&ms.bar_kv_full[kst]), kph, p, ms, kSiteKvFull))) break;
                         tc_fence_after();
                         k_ready = true;
                     }
-                    issue_qk<D, F8>(tmem + t * 128, dq0 + t * kTileStep, dk0 + kst * kTileStep);
-                    umma_commit(smem_u32(&ms.bar_s_full[t]));
+                    if (elect_one()) {
+                        issue_qk<D, F8>(tmem + t * 128, dq0 + t * kTileStep, dk0 + kst * kTileStep);
+                        umma_commit(smem_u32(&ms.bar_s_full[t]));
+                    }
+                    __syncwarp();
                     FA_TRACE_EV(2, (item_n == 1 ? j : kTraceIters), 3 + 2 * t);
                 }
             }
             if (!ok) break;
-            if (k_ready) umma_commit(smem_u32(&ms.bar_kv_empty[kst]));
-            if (j > 0) umma_commit(smem_u32(&ms.bar_kv_empty[vst]));
-            if (j == nmax - 1) umma_commit(smem_u32(&ms.bar_q_empty));
+            if (elect_one()) {
+                if (k_ready) umma_commit(smem_u32(&ms.bar_kv_empty[kst]));
+                if (j > 0) umma_commit(smem_u32(&ms.bar_kv_empty[vst]));
+                if (j == nmax - 1) umma_commit(smem_u32(&ms.bar_q_empty));
+            }
+            __syncwarp();
             if (j < nmax) {                               // next K tile: two positions on
                 kst += 2;
                 if (kst >= (uint32_t)C::kStages) {
@@ -454,7 +471,9 @@ __device__ void mma_role(const Params& p, Misc& ms, const SeqTables& tab, uint32
         }
     }
     // every MMA issued so far must be finished before TMEM and smem go away
-    umma_commit(smem_u32(&ms.bar_drain));
+    __syncwarp();
+    if (elect_one()) umma_commit(smem_u32(&ms.bar_drain));
+    __syncwarp();
     drain_bar(smem_u32(&ms.bar_drain), 0, p);
 }
 
@@ -831,7 +850,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     } else {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
         if (warp == kMmaWarp) {
-            if (lane == 0) mma_role<D, PK, F8>(p, ms, tab, tmem, smem_q, smem_kv, total);
+            mma_role<D, PK, F8>(p, ms, tab, tmem, smem_q, smem_kv, total);   // all 32 lanes
             __syncwarp();
         } else if (warp == kLoadWarp) {
             if (lane == 0) load_role<D, PK, F8>(p, ms, tab, smem_q, smem_kv, total);

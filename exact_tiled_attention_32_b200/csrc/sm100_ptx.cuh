@@ -291,6 +291,18 @@ __device__ __forceinline__ void umma_f8_ts_kv64_x2(uint32_t d_tmem, uint32_t a_t
 }
 
 // arrive once on `bar` when every tcgen05 op issued so far by this thread is done
+// true in exactly one lane of the (converged) warp.  The MMA issuers run
+// their whole loop on all 32 lanes and issue through this: measured on B200,
+// a tcgen05.mma issued this way costs 32-44 clocks of issue against 44-58
+// from a lone lane, and the issue rate of one thread is what bounds a
+// pipeline of 64-clock MMAs once other warps share its sub-partition.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b32 r;\n\telect.sync r|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                      bar)
