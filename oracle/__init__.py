@@ -35,7 +35,7 @@ of one, torch's fp64 scaled-dot-product attention as an independent library
 routine, brute force on tiny shapes with no max shift, closed forms (causal row
 0, all-zero queries, one dominant key) and the tiled == untiled identity.
 The GQA head mapping, the packed-sequence layout and the lse definition rest on
-readings of the pages (listed in the design doc) and are pinned only through the
+readings of the pages (stated in oracle.c) and are pinned only through the
 library routine and brute force that encode the same reading.
 """
 from __future__ import annotations

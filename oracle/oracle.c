@@ -18,7 +18,7 @@
  * are widened exactly.  The pages call the tiled method exact, so this plain
  * definition is the result the GPU path must reach up to rounding.
  *
- * Readings of points the pages leave open (each is also listed in the design doc):
+ * Readings of points the pages leave open:
  *   - scale is a parameter (the pages write softmax(QK^T) with no scale);
  *   - causal means key j is allowed for query i iff j <= i, positions counted
  *     inside the row's own sequence;
