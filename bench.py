@@ -365,6 +365,32 @@ def whole_job_tflops(flops_per_step: float, world: int, steps: int, ms: float) -
     return flops_per_step * world * steps / (ms / 1e3) / 1e12
 
 
+def step_percentiles(per_step_ms):
+    """Median, p10 and p90 of the per-step device times (milliseconds), taken
+    from one CUDA event recorded after each step inside the timed region."""
+    import numpy as np
+    a = np.asarray(per_step_ms, dtype=np.float64)
+    if a.size == 0:
+        return None
+    return {"median": float(np.median(a)), "p10": float(np.percentile(a, 10)),
+            "p90": float(np.percentile(a, 90)), "n": int(a.size)}
+
+
+def timed_steps(step, steps, stream):
+    """Runs ``steps`` steps between CUDA events on ``stream``: one event
+    before the first step and one after every step.  Returns the total device
+    time (first to last event) and the per-step times, in milliseconds."""
+    import torch
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    evs[0].record(stream)
+    for i in range(steps):
+        step()
+        evs[i + 1].record(stream)
+    evs[-1].synchronize()
+    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(steps)]
+    return evs[0].elapsed_time(evs[-1]), per
+
+
 # ------------------------------------------------------------- GPU path
 def main():
     args = parse_args()
@@ -445,17 +471,10 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
     t_host0 = time.time()
-    ev0.record(stream)
-    for _ in range(args.steps):
-        step()
-    ev1.record(stream)
-    ev1.synchronize()
+    ms, per_step = timed_steps(step, args.steps, stream)
     torch.cuda.synchronize(dev)
     t_host1 = time.time()
-    ms = ev0.elapsed_time(ev1)
     if world > 1:
         dist.barrier()
     ms = max_over_ranks(ms, world, dev)
@@ -560,6 +579,7 @@ def main():
         "e2e": e2e,
         "gpu_launches": args.steps * launches_per_step,
         "clocks": clocks,
+        "step_ms": step_percentiles(per_step),
     }
     print(json.dumps(line), flush=True)
 
@@ -605,17 +625,11 @@ def run_bwd(args, w, rank, world, dev):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
     t_host0 = time.time()
-    ev0.record(stream)
-    for _ in range(args.steps):
-        step()
-    ev1.record(stream)
-    ev1.synchronize()
+    ms, per_step = timed_steps(step, args.steps, stream)
     torch.cuda.synchronize(dev)
     t_host1 = time.time()
-    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+    ms = max_over_ranks(ms, world, dev)
     sampler.stop()
     status = fa.fa_get_device_status(stream)
     if status != 0:
@@ -681,6 +695,7 @@ def run_bwd(args, w, rank, world, dev):
         "e2e": e2e,
         "gpu_launches": 3 * args.steps,
         "clocks": sampler.summary(t_host0, t_host1),
+        "step_ms": step_percentiles(per_step),
     }
     print(json.dumps(line), flush=True)
 
