@@ -19,6 +19,12 @@ Every kernel is in libfa.so; this module only schedules them and moves the
 key/value shards with torch.distributed point-to-point operations (NCCL on
 GPUs), which run on the communication stream while the step's kernel runs on
 the compute stream.
+
+With contiguous shards the causal work is uneven: rank r has r + 1 non-empty
+steps.  The zig-zag assignment (``ring_attention_forward_zigzag``) cuts the
+sequence into 2 world chunks of C positions and gives rank r chunks r and
+2 world - 1 - r; at every step each rank then has the same work (two full
+C x C blocks, or at step 0 two diagonal blocks and one full one).
 """
 from __future__ import annotations
 
@@ -181,3 +187,161 @@ def emulate_ring_forward(q, k, v, world: int, *, causal: bool = False, scale: fl
         o[:, :, rank * L:(rank + 1) * L] = os_
         lse[:, :, rank * L:(rank + 1) * L] = ls_
     return o, lse
+
+
+# ---------------------------------------------------------------- zig-zag
+def zigzag_chunks(rank: int, world: int) -> tuple[int, int]:
+    """The two chunks (of 2 world equal chunks of the sequence) that ``rank``
+    holds, in the order of its local shard."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("need 0 <= rank < world")
+    return rank, 2 * world - 1 - rank
+
+
+def zigzag_schedule(rank: int, world: int, causal: bool) -> list[tuple[int, list[tuple[int, int, str]]]]:
+    """Per step t: (source rank, [(query half, key half, mode), ...]) for the
+    four chunk pairs of the rank's two query chunks and the two key chunks it
+    holds at that step (those of rank (rank - t) mod world).  Mode as
+    ``ring_schedule``: a key chunk below the query chunk is FULL, the same
+    chunk DIAG, a later one SKIP."""
+    qa = zigzag_chunks(rank, world)
+    out = []
+    for t in range(world):
+        src = (rank - t) % world
+        kb = zigzag_chunks(src, world)
+        pairs = []
+        for qi, a in enumerate(qa):
+            for ki, b in enumerate(kb):
+                mode = FULL if (not causal or b < a) else DIAG if b == a else SKIP
+                pairs.append((qi, ki, mode))
+        out.append((src, pairs))
+    return out
+
+
+def zigzag_shard(x, rank: int, world: int):
+    """The zig-zag local shard of a full-sequence tensor x [B, H, N, d]
+    (N = 2 world C): chunks rank and 2 world - 1 - rank, concatenated along
+    the sequence, contiguous [B, H, 2C, d]."""
+    import torch
+    N = x.shape[2]
+    if N % (2 * world):
+        raise ValueError("N must be a multiple of 2 * world")
+    C = N // (2 * world)
+    a, b = zigzag_chunks(rank, world)
+    return torch.cat([x[:, :, a * C:(a + 1) * C], x[:, :, b * C:(b + 1) * C]], dim=2).contiguous()
+
+
+def zigzag_unshard(shards, world: int):
+    """Inverse of ``zigzag_shard``: the full-sequence tensor from the local
+    shards of ranks 0 .. world - 1 (each [B, H, 2C, ...])."""
+    import torch
+    C = shards[0].shape[2] // 2
+    chunks = [None] * (2 * world)
+    for r, x in enumerate(shards):
+        a, b = zigzag_chunks(r, world)
+        chunks[a], chunks[b] = x[:, :, :C], x[:, :, C:]
+    return torch.cat(chunks, dim=2)
+
+
+def _halves(x):
+    C = x.shape[2] // 2
+    return x[:, :, :C].contiguous(), x[:, :, C:].contiguous()
+
+
+def _zigzag_step(fa, qh, kh, vh, pairs, t, o_parts, lse_parts, B, Hq, Hkv, C, d, scale, stream):
+    """The four chunk pairs of one step: each query half's share of each key
+    half goes to part 2 t + key half of that query half."""
+    for qi, ki, mode in pairs:
+        slot = 2 * t + ki
+        if mode == SKIP:
+            lse_parts[qi][slot].fill_(-math.inf)
+            continue
+        rc = fa.fa_fwd_partial(qh[qi], kh[ki], vh[ki], o_parts[qi][slot], lse_parts[qi][slot], B, Hq, Hkv, C, C, d,
+                               scale, mode == DIAG, stream)
+        if rc != fa.FA_OK:
+            raise fa.FAError(rc, "fa_fwd_partial")
+
+
+def _zigzag_merge(fa, o_parts, lse_parts, world, B, Hq, C, d, device, stream):
+    import torch
+    rows = B * Hq * C
+    outs, lses = [], []
+    for qi in range(2):
+        o = torch.empty((B, Hq, C, d), dtype=torch.bfloat16, device=device)
+        lse = torch.empty((B, Hq, C), dtype=torch.float32, device=device)
+        rc = fa.fa_merge_partials(o_parts[qi], lse_parts[qi], 2 * world, rows, d, o, lse, stream)
+        if rc != fa.FA_OK:
+            raise fa.FAError(rc, "fa_merge_partials")
+        outs.append(o)
+        lses.append(lse)
+    return torch.cat(outs, dim=2), torch.cat(lses, dim=2)
+
+
+def ring_attention_forward_zigzag(q, k, v, *, causal: bool = False, scale: float | None = None, group=None):
+    """Ring attention with the zig-zag assignment.  q [B, Hq, 2C, d], k/v
+    [B, Hkv, 2C, d]: bf16 CUDA tensors, this rank's zig-zag shard (chunks
+    rank and 2 world - 1 - rank of the sequence, see ``zigzag_shard``).
+    Returns O [B, Hq, 2C, d] (bf16) and lse [B, Hq, 2C] (fp32) in the same
+    local layout."""
+    import torch
+    from . import binding as fa
+
+    B, Hq, Hkv, L, d = _shapes(q, k, v)
+    if L % 2:
+        raise ValueError("a zig-zag shard holds two chunks of equal length")
+    C = L // 2
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    ex = DistExchange(group)
+    world, rank = ex.world, ex.rank
+    rows = B * Hq * C
+    qh = _halves(q)
+    o_parts = [torch.empty((2 * world, rows, d), dtype=torch.float32, device=q.device) for _ in range(2)]
+    lse_parts = [torch.empty((2 * world, rows), dtype=torch.float32, device=q.device) for _ in range(2)]
+    stream = torch.cuda.current_stream(q.device)
+    k0, k1 = _halves(k)
+    v0, v1 = _halves(v)
+    bufs = [(k0, k1, v0, v1), tuple(torch.empty_like(x) for x in (k0, k1, v0, v1))]
+    cur = 0
+    for t, (src, pairs) in enumerate(zigzag_schedule(rank, world, causal)):
+        reqs = None
+        if t + 1 < world:
+            reqs = ex.start(list(bufs[cur]), list(bufs[1 - cur]))
+        kc0, kc1, vc0, vc1 = bufs[cur]
+        _zigzag_step(fa, qh, (kc0, kc1), (vc0, vc1), pairs, t, o_parts, lse_parts, B, Hq, Hkv, C, d, scale, stream)
+        if reqs is not None:
+            ex.wait(reqs)
+            cur = 1 - cur
+    return _zigzag_merge(fa, o_parts, lse_parts, world, B, Hq, C, d, q.device, stream)
+
+
+def emulate_zigzag_forward(q, k, v, world: int, *, causal: bool = False, scale: float | None = None):
+    """Every rank of a ``world``-rank zig-zag ring run one after the other on
+    this device, each step's chunks taken directly from the full tensors (no
+    communication).  q [B, Hq, N, d], k/v [B, Hkv, N, d] with N = 2 world C.
+    Returns the full O and lse."""
+    import torch
+    from . import binding as fa
+
+    B, Hq, Hkv, N, d = _shapes(q, k, v)
+    if N % (2 * world):
+        raise ValueError("N must be a multiple of 2 * world")
+    C = N // (2 * world)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    stream = torch.cuda.current_stream(q.device)
+    rows = B * Hq * C
+    o_shards, lse_shards = [], []
+    for rank in range(world):
+        qh = _halves(zigzag_shard(q, rank, world))
+        o_parts = [torch.empty((2 * world, rows, d), dtype=torch.float32, device=q.device) for _ in range(2)]
+        lse_parts = [torch.empty((2 * world, rows), dtype=torch.float32, device=q.device) for _ in range(2)]
+        for t, (src, pairs) in enumerate(zigzag_schedule(rank, world, causal)):
+            kh = _halves(zigzag_shard(k, src, world))
+            vh = _halves(zigzag_shard(v, src, world))
+            _zigzag_step(fa, qh, kh, vh, pairs, t, o_parts, lse_parts, B, Hq, Hkv, C, d, scale, stream)
+        o, lse = _zigzag_merge(fa, o_parts, lse_parts, world, B, Hq, C, d, q.device, stream)
+        o_shards.append(o)
+        lse_shards.append(lse.unsqueeze(-1))
+    return zigzag_unshard(o_shards, world), zigzag_unshard(lse_shards, world).squeeze(-1)
+

@@ -95,3 +95,50 @@ def test_ring_forward_on_one_rank():
                       lse.cpu().numpy().astype(np.float64).reshape(-1), oo, lo, "ring world 1")
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,B,Hq,Hkv,N,d,causal", [
+    (1, 1, 2, 2, 256, 128, True),
+    (2, 1, 4, 2, 512, 128, True),     # chunks of 128
+    (4, 2, 2, 2, 1024, 64, True),
+    (3, 1, 2, 1, 900, 128, True),     # chunks of 150: ragged tiles in every chunk
+    (4, 1, 2, 2, 1024, 128, False),
+])
+def test_emulated_zigzag_ring_matches_oracle(world, B, Hq, Hkv, N, d, causal):
+    """The zig-zag assignment (rank r holds chunks r and 2 world - 1 - r):
+    every rank's four chunk pairs per step, run one after the other, merged,
+    and put back in sequence order."""
+    import torch
+    from exact_tiled_attention_32_b200 import binding as fa
+    from exact_tiled_attention_32_b200.ring import emulate_zigzag_forward
+    w = syn.Workload("zigzag", B, Hq, Hkv, N, d, causal, 1270 + N + world).draw()
+    o, lse = emulate_zigzag_forward(to_device(w.q), to_device(w.k), to_device(w.v), world, causal=causal,
+                                    scale=w.scale)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status() == 0
+    oo, lo = oracle.attention(w.q, w.k, w.v, B, Hq, Hkv, N, d, w.scale, causal)
+    assert_parity(o.float().cpu().numpy().astype(np.float64).reshape(-1, d),
+                  lse.cpu().numpy().astype(np.float64).reshape(-1), oo, lo, f"zigzag {world} {N} {causal}")
+
+
+def test_zigzag_ring_forward_on_one_rank():
+    """The distributed zig-zag driver (one NCCL rank: its shard is chunks 0
+    and 1, the whole sequence in order)."""
+    import socket
+
+    import torch
+    import torch.distributed as dist
+    from exact_tiled_attention_32_b200.ring import ring_attention_forward_zigzag
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1)
+    try:
+        w = syn.Workload("zz1", 1, 2, 2, 384, 128, True, 1280).draw()
+        o, lse = ring_attention_forward_zigzag(to_device(w.q), to_device(w.k), to_device(w.v), causal=True)
+        torch.cuda.synchronize()
+        oo, lo = oracle.attention(w.q, w.k, w.v, 1, 2, 2, 384, 128, w.scale, True)
+        assert_parity(o.float().cpu().numpy().astype(np.float64).reshape(-1, 128),
+                      lse.cpu().numpy().astype(np.float64).reshape(-1), oo, lo, "zigzag world 1")
+    finally:
+        dist.destroy_process_group()
