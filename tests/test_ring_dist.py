@@ -217,3 +217,71 @@ def test_ring_driver_host_logic(world, causal, zigzag, monkeypatch):
     oo, lo = oracle.attention(w.q, w.k, w.v, B, Hq, Hkv, N, d, w.scale, causal)
     assert np.abs(o.double().numpy().reshape(-1, d) - oo).max() < 1e-2      # bf16 output rounding
     assert np.abs(lse.double().numpy().reshape(-1) - lo).max() < 1e-5
+
+
+def _driver_worker(rank, world, port, zigzag, causal, out):
+    """One rank of the distributed drivers over gloo, with the torch
+    stand-ins for the kernels: returns this rank's O and lse."""
+    import sys
+
+    import numpy as np
+
+    import exact_tiled_attention_32_b200 as pkg
+    from exact_tiled_attention_32_b200 import ring
+    from exact_tiled_attention_32_b200 import synthetic as syn
+    sys.modules["exact_tiled_attention_32_b200.binding"] = _TorchKernels
+    pkg.binding = _TorchKernels
+    torch.cuda.current_stream = lambda *a, **k: None
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        B, Hq, Hkv, d = 1, 4, 2, 16
+        N = 2 * world * 6
+        w = syn.Workload("zzd", B, Hq, Hkv, N, d, causal, 1400 + N).draw()
+        t = lambda a: torch.from_numpy(a.view(np.int16).astype(np.int32) << 16).view(torch.float32)
+        q, k, v = t(w.q), t(w.k), t(w.v)
+        if zigzag:
+            o, lse = ring.ring_attention_forward_zigzag(ring.zigzag_shard(q, rank, world), ring.zigzag_shard(k, rank, world),
+                                                        ring.zigzag_shard(v, rank, world), causal=causal, scale=w.scale)
+        else:
+            L = N // world
+            sl = slice(rank * L, (rank + 1) * L)
+            o, lse = ring.ring_attention_forward(q[:, :, sl].contiguous(), k[:, :, sl].contiguous(),
+                                                 v[:, :, sl].contiguous(), causal=causal, scale=w.scale)
+        out[rank] = (o.double().numpy(), lse.double().numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("zigzag", [False, True])
+@pytest.mark.parametrize("world,causal", [(2, True), (3, True), (2, False)])
+def test_distributed_ring_drivers(world, causal, zigzag):
+    """ring_attention_forward and ring_attention_forward_zigzag over gloo
+    ranks, the kernels replaced by torch stand-ins: every rank's rows match
+    the oracle's attention of the whole sequence."""
+    import numpy as np
+
+    import oracle
+    from exact_tiled_attention_32_b200 import ring
+    from exact_tiled_attention_32_b200 import synthetic as syn
+    ctx = mp.get_context("spawn")
+    out = ctx.Manager().dict()
+    mp.start_processes(_driver_worker, args=(world, _free_port(), zigzag, causal, out), nprocs=world, join=True,
+                       start_method="spawn")
+    B, Hq, Hkv, d = 1, 4, 2, 16
+    N = 2 * world * 6
+    w = syn.Workload("zzd", B, Hq, Hkv, N, d, causal, 1400 + N).draw()
+    oo, lo = oracle.attention(w.q, w.k, w.v, B, Hq, Hkv, N, d, w.scale, causal)
+    oo = torch.from_numpy(oo.reshape(B, Hq, N, d))
+    lo = torch.from_numpy(lo.reshape(B, Hq, N))
+    if zigzag:
+        want = [(ring.zigzag_shard(oo, r, world), ring.zigzag_shard(lo.unsqueeze(-1), r, world).squeeze(-1))
+                for r in range(world)]
+    else:
+        L = N // world
+        want = [(oo[:, :, r * L:(r + 1) * L], lo[:, :, r * L:(r + 1) * L]) for r in range(world)]
+    for r in range(world):
+        o, lse = out[r]
+        assert np.abs(o - want[r][0].numpy()).max() < 1e-2
+        assert np.abs(lse - want[r][1].numpy()).max() < 1e-5
