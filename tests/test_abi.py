@@ -67,6 +67,48 @@ def test_argument_errors_found_on_the_host():
     assert call(N=0, ptrs=(0, 0, 0, 0, 0)) == fa.FA_OK
 
 
+def test_chunk_partial_merge_noalloc_argument_errors_found_on_the_host():
+    """fa_fwd_kvcache, fa_fwd_partial, fa_merge_partials and fa_fwd_noalloc
+    reject bad arguments before touching a device."""
+    from exact_tiled_attention_32_b200 import binding as fa
+    p = 1 << 20
+    P5 = (p, p, p, p, p)
+    for fn in (fa.fa_fwd_kvcache, fa.fa_fwd_partial):
+        def call(B=1, Hq=4, Hkv=2, Nq=64, Nk=256, d=128, causal=1, ptrs=P5):
+            return fn(*ptrs, B, Hq, Hkv, Nq, Nk, d, 0.1, causal)
+        assert call(d=80) == fa.FA_ERR_HEADDIM
+        assert call(Hkv=3) == fa.FA_ERR_GQA
+        assert call(Nq=-1) == fa.FA_ERR_SHAPE
+        assert call(Nk=0) == fa.FA_ERR_SHAPE
+        assert call(Nq=300, Nk=256, causal=1) == fa.FA_ERR_SHAPE      # causal needs Nk >= Nq
+        assert call(ptrs=(p, p, 0, p, p)) == fa.FA_ERR_NULL
+        assert call(ptrs=(p, p, p, p + 4, p)) == fa.FA_ERR_ALIGN
+        assert call(ptrs=(p, p, p, p, p + 2)) == fa.FA_ERR_ALIGN
+        assert call(Nq=0, ptrs=(0, 0, 0, 0, 0)) == fa.FA_OK
+        assert call(B=0, ptrs=(0, 0, 0, 0, 0)) == fa.FA_OK
+
+    def merge(nparts=2, rows=10, d=128, ptrs=(p, p, p, p)):
+        return fa.fa_merge_partials(ptrs[0], ptrs[1], nparts, rows, d, ptrs[2], ptrs[3])
+    assert merge(nparts=0) == fa.FA_ERR_SHAPE
+    assert merge(nparts=4097) == fa.FA_ERR_SHAPE
+    assert merge(rows=-1) == fa.FA_ERR_SHAPE
+    assert merge(d=32) == fa.FA_ERR_HEADDIM
+    assert merge(ptrs=(p, 0, p, p)) == fa.FA_ERR_NULL
+    assert merge(ptrs=(p + 4, p, p, p)) == fa.FA_ERR_ALIGN
+    assert merge(rows=0, ptrs=(0, 0, 0, 0)) == fa.FA_OK
+
+    def noalloc(B=1, Hq=4, Hkv=2, N=128, d=128, cu=None, ptrs=P5):
+        return fa.fa_fwd_noalloc(*ptrs, B, Hq, Hkv, N, d, 0.1, 1, cu)
+    assert noalloc(d=96) == fa.FA_ERR_HEADDIM
+    assert noalloc(Hkv=3) == fa.FA_ERR_GQA
+    assert noalloc(B=-1) == fa.FA_ERR_SHAPE
+    assert noalloc(ptrs=(0, p, p, p, p)) == fa.FA_ERR_NULL
+    assert noalloc(ptrs=(p, p, p, p + 2, p)) == fa.FA_ERR_ALIGN
+    assert noalloc(B=1025, cu=p) == fa.FA_ERR_SHAPE
+    assert noalloc(cu=p + 2) == fa.FA_ERR_ALIGN
+    assert noalloc(N=0, ptrs=(0, 0, 0, 0, 0)) == fa.FA_OK
+
+
 def test_splitkv_argument_errors_found_on_the_host():
     from exact_tiled_attention_32_b200 import binding as fa
     p = 1 << 20
