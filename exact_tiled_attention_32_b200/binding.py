@@ -30,7 +30,8 @@ FA_ERR_SEQLENS = -9
 
 EXPORTED = ("fa_fwd", "fa_get_device_status", "fa_status_string", "fa_fwd_noalloc", "fa_fwd_kvcache",
             "fa_selftest_watchdog", "fa_fwd_splitkv", "fa_splitkv_num_splits", "fa_splitkv_workspace_bytes",
-            "fa_bwd", "fa_bwd_workspace_bytes", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials")
+            "fa_bwd", "fa_bwd_workspace_bytes", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials",
+            "fa_get_noalloc_status")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -78,6 +79,8 @@ _lib.fa_selftest_watchdog.restype = ctypes.c_int
 _lib.fa_selftest_watchdog.argtypes = [ctypes.c_int, ctypes.c_void_p]
 _lib.fa_get_device_status.restype = ctypes.c_int
 _lib.fa_get_device_status.argtypes = [ctypes.c_void_p]
+_lib.fa_get_noalloc_status.restype = ctypes.c_int
+_lib.fa_get_noalloc_status.argtypes = [ctypes.c_void_p]
 _lib.fa_status_string.restype = ctypes.c_char_p
 _lib.fa_status_string.argtypes = [ctypes.c_int]
 
@@ -320,6 +323,12 @@ def fa_selftest_watchdog(timeout_ms: int, stream=None) -> int:
 
 def fa_get_device_status(stream=None) -> int:
     return _lib.fa_get_device_status(_stream(stream))
+
+
+def fa_get_noalloc_status(stream=None) -> int:
+    """Reads and clears the device-side status of fa_fwd_noalloc (kept in the
+    library's fixed array); allocates no device memory."""
+    return _lib.fa_get_noalloc_status(_stream(stream))
 
 
 def fa_status_string(code: int) -> str:

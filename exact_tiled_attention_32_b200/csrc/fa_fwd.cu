@@ -60,9 +60,58 @@ constexpr int kMaxStages = 10;
 constexpr int kBoxBytes = kBlockM * 64 * 2;   // one 128-row x 64-column bf16 TMA box
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only past 2^8
 
+// TMEM layouts (512 columns), per path:
+//  kAlias   S0/P0 [0,128), S1/P1 [128,256), O0 [256,384), O1 [384,512):
+//           P_t is written over S_t, so S_t(j+1) can only be computed after
+//           P_t(j) V_j has read P_t(j): each tile's chain is softmax(j) ->
+//           P V(j) -> S(j+1) -> softmax(j+1).
+//  kSepP    (d = 64) S0 [0,128), S1 [128,256), P0 [256,320), P1 [320,384),
+//           O0 [384,448), O1 [448,512): S_t(j+1) is computed as soon as the
+//           softmax warps have loaded S_t(j) into registers.
+//  kSharedS (d = 128) S [0,128) shared by both tiles, P0 [128,192),
+//           P1 [192,256), O0 [256,384), O1 [384,512): the two tiles' scores
+//           pass through one buffer in turn (S_0(j), S_1(j), S_0(j+1), ...),
+//           each computed once the other tile's softmax warps have loaded
+//           theirs, with the P V products of the tiles in between.
+// In kSepP and kSharedS the softmax of block j+1 starts as soon as that of
+// block j ends; the tensor core runs the other tile's work meanwhile.
+enum TmemLayout : int { kAlias = 0, kSepP = 1, kSharedS = 2 };
+#ifndef FA_LAYOUT_D64
+#define FA_LAYOUT_D64 0
+#endif
+#ifndef FA_LAYOUT_D128
+#define FA_LAYOUT_D128 0
+#endif
+#ifndef FA_LAYOUT_F8
+#define FA_LAYOUT_F8 0
+#endif
+template <int D, bool F8>
+__host__ __device__ constexpr int tmem_layout() {
+    return F8 ? FA_LAYOUT_F8 : (D == 64 ? FA_LAYOUT_D64 : FA_LAYOUT_D128);
+}
+template <int D, bool F8>
+__host__ __device__ constexpr bool sep_p() {
+    return tmem_layout<D, F8>() != kAlias;
+}
+template <int D, bool F8>
+__host__ __device__ constexpr uint32_t tmem_s_col(int t) {
+    return tmem_layout<D, F8>() == kSharedS ? 0u : 128u * t;
+}
+template <int D, bool F8>
+__host__ __device__ constexpr uint32_t tmem_p_col(int t) {
+    return tmem_layout<D, F8>() == kSepP ? 256u + 64u * t
+                                         : (tmem_layout<D, F8>() == kSharedS ? 128u + 64u * t : 128u * t);
+}
+template <int D, bool F8>
+__host__ __device__ constexpr uint32_t tmem_o_col(int t) {
+    return tmem_layout<D, F8>() == kSepP ? 384u + 64u * t : 256u + 128u * t;
+}
+static_assert(tmem_o_col<64, false>(1) + 64 <= 512 && tmem_o_col<128, false>(1) + 128 <= 512, "TMEM columns");
+
 // where a wait gave up (reported in status[1])
 enum WaitSite : int {
-    kSiteQEmpty = 1, kSiteKvEmpty, kSiteQFull, kSiteKvFull, kSitePFull, kSiteSFull, kSiteOFinal
+    kSiteQEmpty = 1, kSiteKvEmpty, kSiteQFull, kSiteKvFull, kSitePFull, kSiteSFull, kSiteOFinal, kSiteSFree,
+    kSitePvDone
 };
 
 struct alignas(64) Params {
@@ -110,6 +159,8 @@ struct Misc {
     uint64_t bar_kv_full[kMaxStages], bar_kv_empty[kMaxStages];
     uint64_t bar_s_full[2], bar_o_final[2], bar_drain;
     uint64_t bar_p_half[2][2];     // P_t keys 0-63 / 64-127 are in TMEM
+    uint64_t bar_s_free[2];        // separate-P layout: the softmax warps have read S_t
+    uint64_t bar_pv_done[2];       // separate-P layout: O_t += P_t V_j has completed
     uint32_t tmem_base;
     int abort_flag;
     int bad;
@@ -477,6 +528,115 @@ __device__ void mma_role(const Params& p, Misc& ms, const SeqTables& tab, uint32
     drain_bar(smem_u32(&ms.bar_drain), 0, p);
 }
 
+// The MMA issuer of the kSepP and kSharedS layouts (P in its own TMEM
+// columns).  Per key block j it issues S_0(j), then S_1(j), each once the
+// softmax warps have loaded the previous scores held in that S buffer
+// (bar_s_free: per tile with kSepP, one for the shared buffer with kSharedS),
+// and O_t += P_t(j-1) V_{j-1} for each tile once P_t(j-1) is written (two
+// 64-key halves), each followed by a commit to bar_pv_done[t]: the softmax
+// waits for it before it overwrites P_t or rescales O_t, and before its
+// epilogue.  Order: kSepP  S_0(j) S_1(j) PV_0(j-1) PV_1(j-1);
+//                   kSharedS S_0(j) PV_0(j-1) S_1(j) PV_1(j-1), so that a
+// P V product runs while the shared scores are being read out.  K_j is
+// released after the last S that reads it, V_{j-1} after the last P V, Q after
+// the item's last S.
+template <int D, bool PK, bool F8>
+__device__ void mma_role_sep_p(const Params& p, Misc& ms, const SeqTables& tab, uint32_t tmem, uint32_t smem_q,
+                               uint32_t smem_kv, int total) {
+    using C = Cfg<D, PK, F8>;
+    constexpr bool kShared = tmem_layout<D, F8>() == kSharedS;
+    const uint64_t dq0 = smem_desc_sw128(smem_q, 16, 1024);
+    const uint64_t dk0 = smem_desc_sw128(smem_kv, 16, 1024);              // K-major (K tiles)
+    const uint64_t dv0 = smem_desc_sw128(smem_kv, kBoxBytes, 1024);       // MN-major (V tiles)
+    constexpr uint64_t kTileStep = C::kTileBytes >> 4;
+    uint32_t kst = 0, kph = 0, item_n = 0;
+    uint32_t pc[2] = {0, 0};      // P_t blocks consumed (phase parity of bar_p_half[t][*])
+    uint32_t sn[2] = {0, 0};      // S issued into buffer 0 / 1: every S but the first waits for bar_s_free
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+        const int idx = item_of_round(r);
+        if (idx >= total) break;
+        const Item it = decode_item<PK>(idx, p, ms, tab);
+        if (max(it.n[0], it.n[1]) == 0) continue;      // a split with no key block
+        if (!(ok = wait_all(smem_u32(&ms.bar_q_full), item_n & 1, p, ms, kSiteQFull))) break;
+        tc_fence_after();
+        ++item_n;
+        const int nmax = max(it.n[0], it.n[1]);
+        for (int j = 0; j <= nmax && ok; ++j) {
+            // V_{j-1} sits one ring position before K_j
+            const uint32_t vst = kst == 0 ? C::kStages - 1 : kst - 1;
+            const uint32_t vph = kst == 0 ? kph ^ 1u : kph;
+            bool k_ready = false, v_ready = false;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                if (j < it.n[t]) {                        // S_t = Q_t K_j^T
+                    const int b = kShared ? 0 : t;        // S buffer
+                    if (sn[b] > 0 &&
+                        !(ok = wait_all(smem_u32(&ms.bar_s_free[b]), (sn[b] - 1) & 1, p, ms, kSiteSFree)))
+                        break;
+                    if (!k_ready) {
+                        if (!(ok = wait_all(smem_u32(&ms.bar_kv_full[kst]), kph, p, ms, kSiteKvFull))) break;
+                        k_ready = true;
+                    }
+                    tc_fence_after();
+                    if (elect_one()) {
+                        issue_qk<D, F8>(tmem + tmem_s_col<D, F8>(t), dq0 + t * kTileStep, dk0 + kst * kTileStep);
+                        umma_commit(smem_u32(&ms.bar_s_full[t]));
+                        // the last S that reads K_j (and, at the item's end, Q)
+                        if (t == 1 || j >= it.n[1]) {
+                            umma_commit(smem_u32(&ms.bar_kv_empty[kst]));
+                            if (j == nmax - 1) umma_commit(smem_u32(&ms.bar_q_empty));
+                        }
+                    }
+                    __syncwarp();
+                    ++sn[b];
+                }
+                // O_u += P_u V_{j-1}: tile u = t right after its S with the
+                // shared buffer, both tiles after S_1 with separate buffers
+#pragma unroll
+                for (int u = kShared ? t : 0; u <= t; ++u) {
+                    if (!kShared && t == 0) break;
+                    if (j == 0 || j - 1 >= it.n[u]) continue;
+                    if (!v_ready) {
+                        if (!(ok = wait_all(smem_u32(&ms.bar_kv_full[vst]), vph, p, ms, kSiteKvFull))) break;
+                        v_ready = true;
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        if (!(ok = wait_all(smem_u32(&ms.bar_p_half[u][h]), pc[u] & 1, p, ms, kSitePFull))) break;
+                        tc_fence_after();
+                        if (elect_one())
+                            issue_pv_half<D, F8>(tmem + tmem_o_col<D, F8>(u), tmem + tmem_p_col<D, F8>(u),
+                                             dv0 + vst * kTileStep, h, h > 0 || j - 1 > 0);
+                        __syncwarp();
+                    }
+                    if (!ok) break;
+                    ++pc[u];
+                    if (elect_one()) {
+                        umma_commit(smem_u32(&ms.bar_pv_done[u]));
+                        if (u == 1 || j - 1 >= it.n[1]) umma_commit(smem_u32(&ms.bar_kv_empty[vst]));
+                    }
+                    __syncwarp();
+                }
+                if (!ok) break;
+            }
+            if (!ok) break;
+            if (j < nmax) {                               // next K tile: two positions on
+                kst += 2;
+                if (kst >= (uint32_t)C::kStages) {
+                    kst -= C::kStages;
+                    kph ^= 1u;
+                }
+            }
+        }
+    }
+    // every MMA issued so far must be finished before TMEM and smem go away
+    __syncwarp();
+    if (elect_one()) umma_commit(smem_u32(&ms.bar_drain));
+    __syncwarp();
+    drain_bar(smem_u32(&ms.bar_drain), 0, p);
+}
+
 // ---------------------------------------------------------------- softmax
 // exp2 of a pair of floats on the FMA pipe instead of the MUFU unit:
 // 2^x = 2^j * 2^f with j = round(x), f = x - j in [-0.5, 0.5]; 2^f is a
@@ -491,11 +651,23 @@ __device__ void mma_role(const Params& p, Misc& ms, const SeqTables& tab, uint32
 #ifndef FA_POLY_PAIRS_PER8_F8
 #define FA_POLY_PAIRS_PER8_F8 1
 #endif
-// column pairs (of every 8) on the polynomial: none for bf16 (measured on B200:
-// slower), one for FP8, whose tensor work per block is half as long while the
-// exponentials are as many (measured: +2.4 %)
-constexpr int kPolyPairsPer8 = FA_POLY_PAIRS_PER8;
-constexpr int kPolyPairsPer8F8 = FA_POLY_PAIRS_PER8_F8;
+// column pairs (of every 8) on the polynomial, per path: FP8 (tensor work per
+// block half as long as bf16's, as many exponentials), bf16 d = 64 (the
+// exponentials cost twice the block's MMAs), bf16 d = 128 (equal costs)
+#ifndef FA_POLY_PAIRS_PER8_D64
+#define FA_POLY_PAIRS_PER8_D64 0
+#endif
+template <int D, bool F8>
+__host__ __device__ constexpr int poly_pairs_per8() {
+    return F8 ? FA_POLY_PAIRS_PER8_F8 : (D == 64 ? FA_POLY_PAIRS_PER8_D64 : FA_POLY_PAIRS_PER8);
+}
+// The row maximum may be formed alongside the first half's exponentials,
+// taken against the current reference m_used (set after key block 0); the
+// half is redone only when the block's maximum exceeds m_used by more than
+// the rescale threshold (bf16 paths; FP8 keeps the exact running maximum).
+#ifndef FA_SPEC_MAX
+#define FA_SPEC_MAX 0
+#endif
 __device__ __forceinline__ uint64_t f2_const(uint32_t bits) {
     return (static_cast<uint64_t>(bits) << 32) | bits;
 }
@@ -517,6 +689,57 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
     return f2_pack(q0, q1);
 }
 
+// Row maximum of the 128 scores: four independent chains of 3-input max.
+__device__ __forceinline__ float row_max128(const uint32_t (&s)[128]) {
+    float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 128; c += 8) {
+        m0 = fmax3(m0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+        m1 = fmax3(m1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+        m2 = fmax3(m2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
+        m3 = fmax3(m3, __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
+    }
+    return fmax3(fmaxf(m0, m1), m2, m3);
+}
+
+// Exponentials of key half HALF (columns 64*HALF .. +63) of a score row:
+// p = 2^(s * scale_log2 - msub) with nm2 = (-msub, -msub), packed into pk
+// (bf16 pairs; FP8: four E4M3 per word in pk[0..15]), their fp32 sums added
+// pairwise into acc.  NPOLY column pairs of every 8 take the FMA-pipe
+// polynomial, the rest ex2 on MUFU.
+template <bool F8, int HALF, int NPOLY>
+__device__ __forceinline__ void exp_half(const uint32_t (&s)[128], uint64_t sl2x2, uint64_t nm2, uint32_t (&pk)[32],
+                                         uint64_t (&acc)[4]) {
+    float e_prev = 0.f, e_prev1 = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const int gi = 32 * HALF + i;       // pair of columns 2gi, 2gi+1
+        const uint64_t x = f2_fma(f2_pack(__uint_as_float(s[2 * gi]), __uint_as_float(s[2 * gi + 1])), sl2x2, nm2);
+        uint64_t e;
+        if ((gi % 8) < NPOLY) {
+            e = exp2_poly2(x);
+        } else {
+            float x0, x1;
+            f2_unpack(x, x0, x1);
+            e = f2_pack(ex2_approx(x0), ex2_approx(x1));
+        }
+        acc[i & 3] = f2_add(acc[i & 3], e);
+        float e0, e1;
+        f2_unpack(e, e0, e1);
+        if constexpr (F8) {
+            // P <= 2^8 fits E4M3's range (448)
+            if (i & 1)
+                pk[i >> 1] = pack_e4m3x4(e_prev, e_prev1, e0, e1);
+            else {
+                e_prev = e0;
+                e_prev1 = e1;
+            }
+        } else {
+            pk[i] = pack_bf16x2(e0, e1);
+        }
+    }
+}
+
 template <int D, bool PK, bool F8 = false>
 __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, uint32_t tmem, int warp, int lane,
                              int total) {
@@ -524,11 +747,14 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
     const int wq = warp % 4;                         // TMEM lane quarter
     const int r = wq * 32 + lane;                    // row inside the tile
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t taddr_s = tmem + lane_off + t * 128;
-    const uint32_t taddr_o = tmem + lane_off + 256 + t * 128;
+    constexpr bool SP = sep_p<D, F8>();
+    const uint32_t taddr_s = tmem + lane_off + tmem_s_col<D, F8>(t);
+    const uint32_t taddr_p = tmem + lane_off + tmem_p_col<D, F8>(t);
+    const int sfree = tmem_layout<D, F8>() == kSharedS ? 0 : t;     // barrier of this tile's S buffer
+    const uint32_t taddr_o = tmem + lane_off + tmem_o_col<D, F8>(t);
     const float sl2 = p.scale_log2;
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
-    uint32_t sc = 0, oc = 0;
+    uint32_t sc = 0, oc = 0, pw = 0;     // S blocks, O finals, P V completions waited for
     bool ok = true;
     for (int rr = 0; ok; ++rr) {
         const int idx = item_of_round(rr);
@@ -556,35 +782,64 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
             if (lane == 0 && wq == 0) FA_TRACE_EV(t, sc - 1, 1);
             uint32_t s[128];
             tmem_ld128_sync(taddr_s, s);
+            if constexpr (SP) {
+                // the scores are in registers: S_t may take the next block
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&ms.bar_s_free[sfree]));
+            }
             if (lane == 0 && wq == 0) FA_TRACE_EV(t, sc - 1, 2);
+            // separate P: P_t and O_t may be written once P_t V_{j-1} is done
+            bool pv_free = !SP || j == 0;
             if ((it.j0 + j) * kBlockN + kBlockN > limit) {      // diagonal or tail block
                 const int lim = limit - (it.j0 + j) * kBlockN;
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
                     if (c >= lim) s[c] = __float_as_uint(-INFINITY);
             }
-            // row max: four independent chains of 3-input max
-            float mx;
-            {
-                float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
-#pragma unroll
-                for (int c = 0; c < 128; c += 8) {
-                    m0 = fmax3(m0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
-                    m1 = fmax3(m1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
-                    m2 = fmax3(m2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
-                    m3 = fmax3(m3, __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
-                }
-                mx = fmax3(fmaxf(m0, m1), m2, m3);
-            }
-            const float m_new = fmaxf(m_used, mx * sl2);
-            if (lane == 0 && wq == 0) FA_TRACE_EV(t, sc - 1, 3);
+            constexpr int kPoly = poly_pairs_per8<D, F8>();
             // FP8: exact running maximum (threshold 0), so that P <= 1 before the
             // 2^8 shift below; bf16: lazy rescale
             constexpr float kThr = F8 ? 0.f : kRescaleThreshold;
+            // FP8: P is computed as 2^8 * exp2(x - m) in (0, 256], so that E4M3
+            // holds every entry above 2^-14 of the row maximum as a normal
+            // number (relative rounding error <= 2^-4); l carries the same
+            // factor, and lse takes it back out
+            constexpr float kPShift = F8 ? 8.f : 0.f;
+            uint64_t acc[4] = {0, 0, 0, 0};      // packed row sums (+0.0f pairs)
+            uint32_t pk[32];
+            // speculative half 0 against the current reference (every row of
+            // the warp has one after its first key block)
+            const bool spec = FA_SPEC_MAX && !F8 && j > 0 && __all_sync(0xffffffffu, m_used != -INFINITY);
+            if (spec) {
+                // stored at once (over scores already in registers), so that
+                // pk is free while the maximum is formed; not yet signalled
+                exp_half<F8, 0, kPoly>(s, sl2x2, f2_pack(-m_used, -m_used), pk, acc);
+                if (!pv_free) {
+                    ok = wait_bar(smem_u32(&ms.bar_pv_done[t]), pw & 1, p, ms, kSitePvDone);
+                    if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                    ++pw;
+                    pv_free = true;
+                    tc_fence_after();
+                }
+                tmem_st32(taddr_p, pk);
+            }
+            const float mx = row_max128(s);
+            const float m_new = fmaxf(m_used, mx * sl2);
+            if (lane == 0 && wq == 0) FA_TRACE_EV(t, sc - 1, 3);
             const bool need = m_new > m_used + kThr;
-            if (j > 0 && __any_sync(0xffffffffu, need)) {
+            const bool any_need = __any_sync(0xffffffffu, need);
+            if (j > 0 && any_need) {
                 // Theorem 2: rescale the partial output when the max grows.
-                // S_t(j) was issued after O_t += P_t V_{j-1}, so O_t is final here.
+                // Shared S/P: S_t(j) was issued after O_t += P_t V_{j-1}, so O_t
+                // is final here; separate P: wait for that product first.
+                if (!pv_free) {
+                    ok = wait_bar(smem_u32(&ms.bar_pv_done[t]), pw & 1, p, ms, kSitePvDone);
+                    if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                    ++pw;
+                    pv_free = true;
+                    tc_fence_after();
+                }
                 const float f = need ? ex2_approx(m_used - m_new) : 1.f;
                 const uint64_t f2 = f2_pack(f, f);
 #pragma unroll
@@ -606,67 +861,38 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
                 l *= (m_used == -INFINITY) ? 0.f : ex2_approx(m_used - m_new);
                 m_used = m_new;
             }
-            // FP8: P is computed as 2^8 * exp2(x - m) in (0, 256], so that E4M3
-            // holds every entry above 2^-14 of the row maximum as a normal
-            // number (relative rounding error <= 2^-4); l carries the same
-            // factor, and lse takes it back out
-            constexpr float kPShift = F8 ? 8.f : 0.f;
             const float msub = ((m_used == -INFINITY) ? 0.f : m_used) - kPShift;
             const uint64_t nm2 = f2_pack(-msub, -msub);
-            uint64_t acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0;   // packed row sums (+0.0f pairs)
+            if (!spec || any_need) {
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t pk[32];             // bf16: 32 pairs; FP8: pk[0..15], four per word
-                float e_prev = 0.f, e_prev1 = 0.f;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int gi = 32 * half + i;       // pair of columns 2gi, 2gi+1
-                    const uint64_t x = f2_fma(f2_pack(__uint_as_float(s[2 * gi]), __uint_as_float(s[2 * gi + 1])),
-                                              sl2x2, nm2);
-                    uint64_t e;
-                    if ((gi % 8) < (F8 ? kPolyPairsPer8F8 : kPolyPairsPer8)) {
-                        e = exp2_poly2(x);
-                    } else {
-                        float x0, x1;
-                        f2_unpack(x, x0, x1);
-                        e = f2_pack(ex2_approx(x0), ex2_approx(x1));
-                    }
-                    switch (i & 3) {
-                        case 0: acc0 = f2_add(acc0, e); break;
-                        case 1: acc1 = f2_add(acc1, e); break;
-                        case 2: acc2 = f2_add(acc2, e); break;
-                        default: acc3 = f2_add(acc3, e); break;
-                    }
-                    float e0, e1;
-                    f2_unpack(e, e0, e1);
-                    if constexpr (F8) {
-                        // P <= 2^8 fits E4M3's range (448)
-                        if (i & 1)
-                            pk[i >> 1] = pack_e4m3x4(e_prev, e_prev1, e0, e1);
-                        else {
-                            e_prev = e0;
-                            e_prev1 = e1;
-                        }
-                    } else {
-                        pk[i] = pack_bf16x2(e0, e1);
-                    }
+                for (int i = 0; i < 4; ++i) acc[i] = 0;
+                exp_half<F8, 0, kPoly>(s, sl2x2, nm2, pk, acc);
+                if (!pv_free) {
+                    ok = wait_bar(smem_u32(&ms.bar_pv_done[t]), pw & 1, p, ms, kSitePvDone);
+                    if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                    ++pw;
+                    pv_free = true;
+                    tc_fence_after();
                 }
-                if constexpr (F8) {
-                    tmem_st16(taddr_s + half * 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
-                } else {
-                    tmem_st32(taddr_s + half * 32, pk);
-                }
-                if (half == 0) {
-                    // keys 0-63 of P are ready: the tensor core can start on them
-                    tmem_wait_st();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_u32(&ms.bar_p_half[t][0]));
-                }
+                if constexpr (F8)
+                    tmem_st16(taddr_p, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
+                else
+                    tmem_st32(taddr_p, pk);
             }
+            // keys 0-63 of P are ready: the tensor core can start on them
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ms.bar_p_half[t][0]));
+            uint32_t pk1[32];
+            exp_half<F8, 1, kPoly>(s, sl2x2, nm2, pk1, acc);
+            if constexpr (F8)
+                tmem_st16(taddr_p + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk1[0]));
+            else
+                tmem_st32(taddr_p + 32, pk1);
             {
                 float a, b;
-                f2_unpack(f2_add(f2_add(acc0, acc1), f2_add(acc2, acc3)), a, b);
+                f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a, b);
                 l += a + b;
             }
             tmem_wait_st();
@@ -677,9 +903,15 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
         }
         if (!ok) break;
         // epilogue: O / l -> bf16 -> HBM, and the logsumexp
-        ok = wait_bar(smem_u32(&ms.bar_o_final[t]), oc & 1, p, ms, kSiteOFinal);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        ++oc;
+        if constexpr (SP) {
+            ok = wait_bar(smem_u32(&ms.bar_pv_done[t]), pw & 1, p, ms, kSitePvDone);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            ++pw;
+        } else {
+            ok = wait_bar(smem_u32(&ms.bar_o_final[t]), oc & 1, p, ms, kSiteOFinal);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            ++oc;
+        }
         tc_fence_after();
         const bool valid = row < it.len;
         float inv = l > 0.f ? 1.f / l : 0.f;
@@ -771,6 +1003,8 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             mbar_init(smem_u32(&ms.bar_p_half[t][0]), 4); // one arrival per warp
             mbar_init(smem_u32(&ms.bar_p_half[t][1]), 4);
             mbar_init(smem_u32(&ms.bar_o_final[t]), 1);
+            mbar_init(smem_u32(&ms.bar_s_free[t]), 4);     // one arrival per warp
+            mbar_init(smem_u32(&ms.bar_pv_done[t]), 1);
         }
         ms.abort_flag = 0;
         ms.bad = 0;
@@ -850,7 +1084,10 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     } else {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
         if (warp == kMmaWarp) {
-            mma_role<D, PK, F8>(p, ms, tab, tmem, smem_q, smem_kv, total);   // all 32 lanes
+            if constexpr (sep_p<D, F8>())
+                mma_role_sep_p<D, PK, F8>(p, ms, tab, tmem, smem_q, smem_kv, total);   // all 32 lanes
+            else
+                mma_role<D, PK, F8>(p, ms, tab, tmem, smem_q, smem_kv, total);   // all 32 lanes
             __syncwarp();
         } else if (warp == kLoadWarp) {
             if (lane == 0) load_role<D, PK, F8>(p, ms, tab, smem_q, smem_kv, total);
@@ -1312,6 +1549,7 @@ extern "C" int fa_merge_partials(const float* o_parts, const float* lse_parts, i
     if (d != 64 && d != 128) return FA_ERR_HEADDIM;
     if (rows == 0) return FA_OK;
     if (rows * nparts > (1ll << 40)) return FA_ERR_SHAPE;
+    if ((rows + 7) / 8 > 0x7fffffffll) return FA_ERR_SHAPE;     // grid x: 8 rows per block
     if (!o_parts || !lse_parts || !o || !lse) return FA_ERR_NULL;
     if (!aligned(o_parts, 16) || !aligned(lse_parts, 4) || !aligned(o, 16) || !aligned(lse, 4)) return FA_ERR_ALIGN;
     int dev = 0;
@@ -1477,4 +1715,20 @@ extern "C" int fa_fwd_noalloc(const void* q, const void* k, const void* v, void*
     if (cudaMemsetAsync(st->scratch, 0, kStatusBytes, s) != cudaSuccess) return FA_ERR_LAUNCH;
     return launch_fwd(q, k, v, o, lse, B, Hq, Hkv, N, N, 0, d, scale, causal, cu_seqlens, s, st->scratch,
                       st->num_sms);
+}
+
+extern "C" int fa_get_noalloc_status(void* stream) {
+    using namespace fa_sm100;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_LAUNCH;
+    NoAllocState* st = nullptr;
+    const int rc = noalloc_setup(dev, &st);
+    if (rc != FA_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int h[4] = {0, 0, 0, 0};
+    static_assert(sizeof(h) == kStatusBytes, "status words");
+    if (cudaMemcpyAsync(h, st->scratch, kStatusBytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return FA_ERR_LAUNCH;
+    if (cudaMemsetAsync(st->scratch, 0, kStatusBytes, s) != cudaSuccess) return FA_ERR_LAUNCH;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return FA_ERR_LAUNCH;
+    return h[0];
 }

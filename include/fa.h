@@ -150,8 +150,10 @@ int fa_fwd_partial(const void* q, const void* k, const void* v, float* o_part, f
  * fa_fwd_partial writes them, into bf16 o [rows][d] and fp32 lse [rows]:
  *   lse = ln sum_s exp(lse_s),  O = sum_s exp(lse_s - lse) O_s.
  * A share with lse_s = -inf carries weight 0; a row without any allowed key
- * gets O = 0, lse = -inf.  d is 64 or 128; 1 <= nparts <= 4096.  Asynchronous
- * on `stream`.  Errors: FA_ERR_SHAPE, FA_ERR_HEADDIM, FA_ERR_NULL,
+ * gets O = 0, lse = -inf.  d is 64 or 128; 1 <= nparts <= 4096;
+ * rows * nparts <= 2^40 and rows <= 8 * (2^31 - 1) (one block per 8 rows),
+ * else FA_ERR_SHAPE.  Asynchronous on `stream`.  Errors: FA_ERR_SHAPE,
+ * FA_ERR_HEADDIM, FA_ERR_NULL,
  * FA_ERR_ALIGN (o 16-byte aligned), FA_ERR_LAUNCH.
  */
 int fa_merge_partials(const float* o_parts, const float* lse_parts, int nparts, long long rows, int d,
@@ -311,12 +313,33 @@ const char* fa_status_string(int status);
  * All calls share the array, which keeps the last call's contents; each call
  * clears the status words on its stream before its kernel starts.  Calls that
  * overlap on the GPU (different streams, or several host threads) race on the
- * status words.  Device-side errors of this entry point are written to that
- * array only; fa_get_device_status reports the word of fa_fwd, not this one.
+ * status words.  Device-side errors of this entry point (FA_ERR_DEVICE_TIMEOUT,
+ * FA_ERR_SEQLENS) are written to that array only: read them with
+ * fa_get_noalloc_status, not fa_get_device_status (which reports fa_fwd's
+ * word).
  */
 int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
                    int B, int Hq, int Hkv, int N, int d, float scale, int causal,
                    const int32_t* cu_seqlens, void* stream);
+
+/*
+ * fa_get_noalloc_status -- reads and clears the device-side status word of
+ * fa_fwd_noalloc on the current device.  (Part of the no-allocation addition;
+ * the pages have no counterpart.)
+ *
+ * Copies the status words out of the library's fixed array with
+ * cudaMemcpyAsync on `stream` into a host variable, zeroes them with
+ * cudaMemsetAsync on the same stream, and waits for `stream`; so it reports
+ * the last fa_fwd_noalloc call ordered before it on `stream`.  Allocates no
+ * device memory (on a device where fa_fwd_noalloc has not run yet it does that
+ * device's set-up first, which allocates nothing either).
+ *
+ * Returns FA_OK, the first device-side error recorded since the words were
+ * last cleared (FA_ERR_DEVICE_TIMEOUT, FA_ERR_SEQLENS), or a host-side error
+ * (FA_ERR_ARCH, FA_ERR_LAUNCH).  Shares the array's race: a fa_fwd_noalloc
+ * call running concurrently on another stream may be reported or cleared.
+ */
+int fa_get_noalloc_status(void* stream);
 
 #ifdef __cplusplus
 }

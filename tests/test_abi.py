@@ -96,6 +96,8 @@ def test_chunk_partial_merge_noalloc_argument_errors_found_on_the_host():
     assert merge(ptrs=(p, 0, p, p)) == fa.FA_ERR_NULL
     assert merge(ptrs=(p + 4, p, p, p)) == fa.FA_ERR_ALIGN
     assert merge(rows=0, ptrs=(0, 0, 0, 0)) == fa.FA_OK
+    # one block of the merge kernel per 8 rows: the grid's x limit bounds rows
+    assert merge(nparts=1, rows=8 * (2 ** 31 - 1) + 1) == fa.FA_ERR_SHAPE
 
     def noalloc(B=1, Hq=4, Hkv=2, N=128, d=128, cu=None, ptrs=P5):
         return fa.fa_fwd_noalloc(*ptrs, B, Hq, Hkv, N, d, 0.1, 1, cu)
@@ -195,6 +197,7 @@ def test_no_device_means_launch_error():
     p = 1 << 20
     assert fa.fa_fwd(p, p, p, p, p, 1, 1, 1, 128, 64, 0.1, 0) == fa.FA_ERR_LAUNCH
     assert fa.fa_get_device_status() == fa.FA_ERR_LAUNCH
+    assert fa.fa_get_noalloc_status() == fa.FA_ERR_LAUNCH
     assert fa.fa_splitkv_num_splits(1, 32, 8, 1, 32768, 128) == fa.FA_ERR_LAUNCH
 
 

@@ -10,7 +10,20 @@ entry below that is off by at most 2^-18 (half the subnormal step, in units of
 the row maximum).  After the division by the row sum l = sum_j exp(s_j - m):
 |dO_c| <= 1e-2 + 2^-7 |O_c| + 2^-4 sum_j p_j |v_jc| + 2^-18 sum_{tiny j} |v_jc| / l.
 The weights p, l and the tiny set come from the exact scores of the
-dequantised inputs."""
+dequantised inputs.
+
+Mean bound (over the compared elements): the worst case above adds every
+weight's rounding error with the same sign; the mean error is checked
+against the typical size instead.  Taking the E4M3 rounding errors d_j of
+the weights as independent and zero-mean, each at most 2^-4 relative and
+uniform within its rounding interval (E[d_j^2] <= 2^-8 / 3), the P V term
+of column c has the root-mean-square size
+    r_c = 2^-4 / sqrt(3) * sqrt(sum_j p_j^2 v_jc^2),
+which bounds its mean absolute value.  So
+    mean |dO| <= 1e-3 + mean(2^-8 |O| + 3 r + tiny term),
+the benchmark spec's mean-abs 1e-3, the worst case of the bf16 rounding of O
+(round to nearest: 2^-8 relative) and of the tiny weights, and three times
+the typical P V rounding error as the margin for a finite sample."""
 import numpy as np
 import pytest
 
@@ -37,12 +50,15 @@ def _run(w):
 
 
 def _bound(w, rows, o_ref):
-    """Per-element tolerance of the rows (see the module docstring)."""
+    """Per-element worst-case tolerance of the rows (see the module
+    docstring) and the per-element terms of the mean bound."""
     qf = oracle.e4m3_decode(w.q).reshape(-1, w.d) * S
     kf = oracle.e4m3_decode(w.k).reshape(w.B, w.Hkv, w.N, w.d) * S
     vf = oracle.e4m3_decode(w.v).reshape(w.B, w.Hkv, w.N, w.d) * S
     g = w.Hq // w.Hkv
     out = np.empty((len(rows), w.d))
+    rms = np.empty((len(rows), w.d))
+    tiny_t = np.empty((len(rows), w.d))
     for n, rid in enumerate(rows):
         t = rid % w.N
         bh = rid // w.N
@@ -54,8 +70,12 @@ def _bound(w, rows, o_ref):
         e = np.exp(s - s.max())
         l = e.sum()
         tiny = e < 2.0 ** -14
-        out[n] = 2.0 ** -4 * (e / l) @ V + 2.0 ** -18 * V[tiny].sum(axis=0) / l
-    return 1e-2 + 2.0 ** -7 * np.abs(o_ref) + out
+        tiny_t[n] = 2.0 ** -18 * V[tiny].sum(axis=0) / l
+        out[n] = 2.0 ** -4 * (e / l) @ V + tiny_t[n]
+        rms[n] = 2.0 ** -4 / np.sqrt(3.0) * np.sqrt(((e / l) ** 2) @ (V ** 2))
+    worst = 1e-2 + 2.0 ** -7 * np.abs(o_ref) + out
+    mean_terms = 2.0 ** -8 * np.abs(o_ref) + 3.0 * rms + tiny_t
+    return worst, mean_terms
 
 
 def _check(w, o, lse, rows, what):
@@ -64,9 +84,11 @@ def _check(w, o, lse, rows, what):
     got = o[rows]
     assert not np.isnan(got).any(), f"{what}: NaN"
     err = np.abs(got - o_ref)
-    excess = err - _bound(w, rows, o_ref)
+    worst, mean_terms = _bound(w, rows, o_ref)
+    excess = err - worst
     assert excess.max() <= 0, f"{what}: O error {err.max():.3e} exceeds the E4M3 bound by {excess.max():.3e}"
-    assert err.mean() <= 1e-2, f"{what}: O mean error {err.mean():.3e}"
+    mean_bound = 1e-3 + mean_terms.mean()
+    assert err.mean() <= mean_bound, f"{what}: O mean error {err.mean():.3e} > derived {mean_bound:.3e}"
     lerr = np.abs(lse[rows] - l_ref)
     assert lerr.max() <= 1e-3, f"{what}: lse error {lerr.max():.3e}"
 

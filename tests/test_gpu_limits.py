@@ -4,13 +4,13 @@ sequence at the forward's maximum of 262,144 tokens (sampled rows), and one
 token past it rejected on the device.  Tolerances as the other parity tests;
 the 1024 short causal sequences have rows with one or two keys, whose O is
 a V row (|O| up to ~4.5), so there the bf16-derived bound of the stress tests
-applies (one bf16 ulp of |O| is 2^-6 on [2, 4))."""
+applies (the rounding of O alone can reach 2^-8 |O| > 1e-2 there)."""
 import numpy as np
 import pytest
 
 import oracle
 from exact_tiled_attention_32_b200 import synthetic as syn
-from fa_util import assert_bf16_bound, assert_parity, gather, to_device
+from fa_util import assert_bf16_bound, assert_parity, gather, softmax_weighted_abs_v, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -30,8 +30,7 @@ def test_forward_1024_sequences():
     assert fa.fa_get_device_status() == 0
     og, lg = gather(w, o, lse)
     oo, lo = oracle.attention(w.q, w.k, w.v, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, True, w.cu_seqlens)
-    vmax = float(np.abs(syn.bf16_bits_to_float(w.v)).max())
-    assert_bf16_bound(og, lg, oo, lo, vmax, "1024 sequences")
+    assert_bf16_bound(og, lg, oo, lo, softmax_weighted_abs_v(w, w.scale, True, lo), "1024 sequences")
 
 
 def test_backward_1024_sequences():

@@ -12,7 +12,7 @@ import pytest
 
 import oracle
 from exact_tiled_attention_32_b200 import synthetic as syn
-from fa_util import assert_bf16_bound, assert_parity, gather, run_gpu, sample_rows, to_device
+from fa_util import assert_bf16_bound, assert_parity, gather, run_gpu, sample_rows, softmax_weighted_abs_v, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -90,8 +90,7 @@ def test_large_scores_exercise_rescale(d, causal):
     torch.cuda.synchronize()
     og, lg = gather(w, o, lse)
     oo, lo = oracle.attention(w.q, w.k, w.v, w.B, w.Hq, w.Hkv, w.N, d, w_scale, causal)
-    vmax = float(np.abs(syn.bf16_bits_to_float(w.v)).max())
-    assert_bf16_bound(og, lg, oo, lo, vmax, "large scores")
+    assert_bf16_bound(og, lg, oo, lo, softmax_weighted_abs_v(w, w_scale, causal, lo), "large scores")
 
 
 def test_increasing_scores_force_rescale_every_block():
@@ -113,8 +112,7 @@ def test_increasing_scores_force_rescale_every_block():
     torch.cuda.synchronize()
     og, lg = gather(w, o, lse)
     oo, lo = oracle.attention(w.q, w.k, w.v, 1, 1, 1, N, d, scale, False)
-    vmax = float(np.abs(syn.bf16_bits_to_float(w.v)).max())
-    assert_bf16_bound(og, lg, oo, lo, vmax, "ramp")
+    assert_bf16_bound(og, lg, oo, lo, softmax_weighted_abs_v(w, scale, False, lo), "ramp")
 
 
 def test_zero_queries_give_mean_of_values():
