@@ -80,7 +80,7 @@ enum TmemLayout : int { kAlias = 0, kSepP = 1, kSharedS = 2 };
 #define FA_LAYOUT_D64 0
 #endif
 #ifndef FA_LAYOUT_D128
-#define FA_LAYOUT_D128 0
+#define FA_LAYOUT_D128 2
 #endif
 #ifndef FA_LAYOUT_F8
 #define FA_LAYOUT_F8 0
@@ -314,9 +314,17 @@ constexpr uint32_t kSuspendNs = FA_SUSPEND_NS;
 
 // Bounded wait: gives up after timeout_ns (recording the site in the status
 // word and raising the CTA's abort flag) or as soon as another role aborted.
+#ifndef FA_SPIN
+#define FA_SPIN 0
+#endif
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Params& p, Misc& ms,
                                       int site) {
     if (mbar_try_wait(bar, parity)) return true;
+#if FA_SPIN > 0
+    // a short busy poll first: a phase that completes within it is seen at once
+    for (int i = 0; i < FA_SPIN; ++i)
+        if (mbar_test_wait(bar, parity)) return true;
+#endif
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
@@ -631,6 +639,160 @@ __device__ void mma_role_sep_p(const Params& p, Misc& ms, const SeqTables& tab, 
         }
     }
     // every MMA issued so far must be finished before TMEM and smem go away
+    __syncwarp();
+    if (elect_one()) umma_commit(smem_u32(&ms.bar_drain));
+    __syncwarp();
+    drain_bar(smem_u32(&ms.bar_drain), 0, p);
+}
+
+// Two issuers for the separate-P layouts: warp kMmaWarp issues the S
+// products (each as soon as its S buffer is free), warp kAllocWarp the P V
+// products (each as soon as its P is written), so that neither kind waits
+// behind the other's barriers.  They walk the same items and ring positions:
+// K_j at 2j, V_j at 2j + 1 from an item's first tile.
+#ifndef FA_SPLIT_ISSUE
+#define FA_SPLIT_ISSUE 1
+#endif
+template <int D, bool F8>
+__host__ __device__ constexpr bool split_issue() {
+    return sep_p<D, F8>() && FA_SPLIT_ISSUE;
+}
+
+#ifndef FA_PRE_DESC
+#define FA_PRE_DESC 1
+#endif
+template <int D, bool PK, bool F8, bool PV>
+__device__ void mma_role_split(const Params& p, Misc& ms, const SeqTables& tab, uint32_t tmem, uint32_t smem_q,
+                               uint32_t smem_kv, int total) {
+    using C = Cfg<D, PK, F8>;
+    constexpr bool kShared = tmem_layout<D, F8>() == kSharedS;
+    constexpr bool kPre = FA_PRE_DESC && !F8;
+    // descriptor start-address steps of the 16-element K steps (128-byte
+    // swizzle, K-major): +2 per step, +1024 for the second 64-column box;
+    // V (MN-major): +128 per 16 key rows
+    constexpr int kSteps = D / 16;
+    const uint64_t dq0 = smem_desc_sw128(smem_q, 16, 1024);
+    const uint64_t dk0 = smem_desc_sw128(smem_kv, 16, 1024);              // K-major (K tiles)
+    const uint64_t dv0 = smem_desc_sw128(smem_kv, kBoxBytes, 1024);       // MN-major (V tiles)
+    constexpr uint64_t kTileStep = C::kTileBytes >> 4;
+    uint32_t kst = 0, kph = 0, item_n = 0;    // ring position of the item's next K tile
+    uint32_t pc[2] = {0, 0};      // P_t blocks consumed (phase parity of bar_p_half[t][*])
+    uint32_t sn[2] = {0, 0};      // S issued into buffer 0 / 1: every S but the first waits for bar_s_free
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+        const int idx = item_of_round(r);
+        if (idx >= total) break;
+        const Item it = decode_item<PK>(idx, p, ms, tab);
+        if (max(it.n[0], it.n[1]) == 0) continue;      // a split with no key block
+        if constexpr (!PV) {
+            FA_TRACE_EV(2, kTraceIters - 32 + (item_n & 31), 6);
+            if (!(ok = wait_all(smem_u32(&ms.bar_q_full), item_n & 1, p, ms, kSiteQFull))) break;
+            tc_fence_after();
+            FA_TRACE_EV(2, kTraceIters - 32 + (item_n & 31), 7);
+        }
+        ++item_n;
+        const int nmax = max(it.n[0], it.n[1]);
+        for (int j = 0; j < nmax && ok; ++j) {
+            [[maybe_unused]] const int tj = item_n == 1 ? j : kTraceIters;     // timeline of the first item only
+            FA_TRACE_EV(PV ? 3 : 2, tj, 0);
+            if constexpr (!PV) {
+                bool k_ready = false;
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    if (j >= it.n[t]) continue;
+                    const int b = kShared ? 0 : t;
+                    if (sn[b] > 0 &&
+                        !(ok = wait_all(smem_u32(&ms.bar_s_free[b]), (sn[b] - 1) & 1, p, ms, kSiteSFree)))
+                        break;
+                    if (!k_ready) {
+                        if (!(ok = wait_all(smem_u32(&ms.bar_kv_full[kst]), kph, p, ms, kSiteKvFull))) break;
+                        k_ready = true;
+                    }
+                    tc_fence_after();
+                    FA_TRACE_EV(2, tj, 1 + 2 * t);
+                    if constexpr (kPre) {
+                        uint64_t ad[kSteps], bd[kSteps];
+#pragma unroll
+                        for (int i = 0; i < kSteps; ++i) {
+                            const uint64_t off = (i & 3) * 2 + (i >> 2) * 1024;
+                            ad[i] = dq0 + t * kTileStep + off;
+                            bd[i] = dk0 + kst * kTileStep + off;
+                        }
+                        if (elect_one()) {
+                            constexpr uint32_t idesc = idesc_bf16_f32(kBlockM, kBlockN, false);
+                            if constexpr (D == 128)
+                                umma_ss_x8_pre(tmem + tmem_s_col<D, F8>(t), ad, bd, idesc);
+                            else
+                                umma_ss_x4_pre(tmem + tmem_s_col<D, F8>(t), ad, bd, idesc);
+                            umma_commit(smem_u32(&ms.bar_s_full[t]));
+                            if (t == 1 || j >= it.n[1]) {
+                                umma_commit(smem_u32(&ms.bar_kv_empty[kst]));
+                                if (j == nmax - 1) umma_commit(smem_u32(&ms.bar_q_empty));
+                            }
+                        }
+                    } else if (elect_one()) {
+                        issue_qk<D, F8>(tmem + tmem_s_col<D, F8>(t), dq0 + t * kTileStep, dk0 + kst * kTileStep);
+                        umma_commit(smem_u32(&ms.bar_s_full[t]));
+                        if (t == 1 || j >= it.n[1]) {
+                            umma_commit(smem_u32(&ms.bar_kv_empty[kst]));
+                            if (j == nmax - 1) umma_commit(smem_u32(&ms.bar_q_empty));
+                        }
+                    }
+                    __syncwarp();
+                    FA_TRACE_EV(2, tj, 2 + 2 * t);
+                    ++sn[b];
+                }
+            } else {
+                // V_j sits one ring position after K_j
+                const uint32_t vst = kst + 1 == (uint32_t)C::kStages ? 0 : kst + 1;
+                const uint32_t vph = kst + 1 == (uint32_t)C::kStages ? kph ^ 1u : kph;
+                if (!(ok = wait_all(smem_u32(&ms.bar_kv_full[vst]), vph, p, ms, kSiteKvFull))) break;
+                FA_TRACE_EV(3, tj, 1);
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    if (j >= it.n[t]) continue;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        if (!(ok = wait_all(smem_u32(&ms.bar_p_half[t][h]), pc[t] & 1, p, ms, kSitePFull))) break;
+                        tc_fence_after();
+                        FA_TRACE_EV(3, tj, 2 + 3 * t + h);
+                        if constexpr (kPre) {
+                            uint32_t a[4];
+                            uint64_t b[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                a[i] = tmem + tmem_p_col<D, F8>(t) + 32 * h + 8 * i;
+                                b[i] = dv0 + vst * kTileStep + static_cast<uint64_t>(h * ((64 * 128) >> 4) + 128 * i);
+                            }
+                            if (elect_one())
+                                umma_ts_x4_pre(tmem + tmem_o_col<D, F8>(t), a, b, idesc_bf16_f32(kBlockM, D, true),
+                                               (h > 0 || j > 0) ? 1u : 0u);
+                        } else if (elect_one()) {
+                            issue_pv_half<D, F8>(tmem + tmem_o_col<D, F8>(t), tmem + tmem_p_col<D, F8>(t),
+                                                 dv0 + vst * kTileStep, h, h > 0 || j > 0);
+                        }
+                        __syncwarp();
+                    }
+                    if (!ok) break;
+                    ++pc[t];
+                    if (elect_one()) {
+                        umma_commit(smem_u32(&ms.bar_pv_done[t]));
+                        if (t == 1 || j >= it.n[1]) umma_commit(smem_u32(&ms.bar_kv_empty[vst]));
+                    }
+                    __syncwarp();
+                    FA_TRACE_EV(3, tj, 4 + 3 * t);
+                }
+            }
+            if (!ok) break;
+            kst += 2;                                     // next K tile: two positions on
+            if (kst >= (uint32_t)C::kStages) {
+                kst -= C::kStages;
+                kph ^= 1u;
+            }
+        }
+    }
+    // every MMA this warp issued must be finished before TMEM and smem go
+    // away (bar_drain takes one commit from each issuer)
     __syncwarp();
     if (elect_one()) umma_commit(smem_u32(&ms.bar_drain));
     __syncwarp();
@@ -993,7 +1155,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     if (tid == 0) {
         mbar_init(smem_u32(&ms.bar_q_full), 1);
         mbar_init(smem_u32(&ms.bar_q_empty), 1);
-        mbar_init(smem_u32(&ms.bar_drain), 1);
+        mbar_init(smem_u32(&ms.bar_drain), split_issue<D, F8>() ? 2 : 1);
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(smem_u32(&ms.bar_kv_full[s]), 1);
             mbar_init(smem_u32(&ms.bar_kv_empty[s]), 1);
@@ -1083,7 +1245,13 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         softmax_role<D, PK, F8>(p, ms, tab, tmem, warp, lane, total);
     } else {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
-        if (warp == kMmaWarp) {
+        if (split_issue<D, F8>() && (warp == kMmaWarp || warp == kAllocWarp)) {
+            if (warp == kMmaWarp)
+                mma_role_split<D, PK, F8, false>(p, ms, tab, tmem, smem_q, smem_kv, total);
+            else
+                mma_role_split<D, PK, F8, true>(p, ms, tab, tmem, smem_q, smem_kv, total);
+            __syncwarp();
+        } else if (warp == kMmaWarp) {
             if constexpr (sep_p<D, F8>())
                 mma_role_sep_p<D, PK, F8>(p, ms, tab, tmem, smem_q, smem_kv, total);   // all 32 lanes
             else

@@ -61,6 +61,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// true once the phase with the given parity has completed; never suspends
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // --------------------------------------------------------------------- TMA
 // 4-D tiled bulk-tensor load into this CTA's shared memory; completion is
 // signalled on `bar` as transaction bytes.  No multicast.
@@ -287,6 +300,54 @@ __device__ __forceinline__ void umma_f8_ts_kv64_x2(uint32_t d_tmem, uint32_t a_t
         "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [t1], b1, %3, pt;\n\t}"
         ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Eight / four MMAs with every descriptor given (computed before the issuing
+// thread's waits); the first MMA overwrites D, the rest accumulate.
+__device__ __forceinline__ void umma_ss_x8_pre(uint32_t d_tmem, const uint64_t (&a)[8], const uint64_t (&b)[8],
+                                               uint32_t idesc) {
+    asm volatile(
+        "{\n\t.reg .pred pf, pt;\n\t"
+        "setp.ne.b32 pf, %1, %1;\n\tsetp.eq.b32 pt, %1, %1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %10, %1, pf;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %11, %1, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %12, %1, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %13, %1, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %6, %14, %1, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %15, %1, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %8, %16, %1, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %9, %17, %1, pt;\n\t}"
+        ::"r"(d_tmem), "r"(idesc), "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(a[4]), "l"(a[5]), "l"(a[6]),
+        "l"(a[7]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "l"(b[4]), "l"(b[5]), "l"(b[6]), "l"(b[7])
+        : "memory");
+}
+__device__ __forceinline__ void umma_ss_x4_pre(uint32_t d_tmem, const uint64_t (&a)[4], const uint64_t (&b)[4],
+                                               uint32_t idesc) {
+    asm volatile(
+        "{\n\t.reg .pred pf, pt;\n\t"
+        "setp.ne.b32 pf, %1, %1;\n\tsetp.eq.b32 pt, %1, %1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %6, %1, pf;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %7, %1, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %1, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %9, %1, pt;\n\t}"
+        ::"r"(d_tmem), "r"(idesc), "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]),
+        "l"(b[3])
+        : "memory");
+}
+// Four TS MMAs (A from TMEM) with every address and descriptor given; the
+// first accumulates only if `accumulate` is nonzero.
+__device__ __forceinline__ void umma_ts_x4_pre(uint32_t d_tmem, const uint32_t (&a)[4], const uint64_t (&b)[4],
+                                               uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p0, pt;\n\t"
+        "setp.ne.b32 p0, %2, 0;\n\tsetp.eq.b32 pt, %1, %1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %7, %1, p0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %8, %1, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%5], %9, %1, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%6], %10, %1, pt;\n\t}"
+        ::"r"(d_tmem), "r"(idesc), "r"(accumulate), "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "l"(b[0]),
+        "l"(b[1]), "l"(b[2]), "l"(b[3])
         : "memory");
 }
 
