@@ -66,7 +66,9 @@ def workload_desc(w):
                 f"positions) against {w.Nk} keys, B={w.B} Hq={w.Hq} Hkv={w.Hkv} d={w.d}, bf16 N(0,1), "
                 "scale=1/sqrt(d)")
     if w.fp8:
-        return (f"{w.name}: {'causal' if w.causal else 'non-causal'} B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d}, "
+        shape = (f"packed {w.B} sequences (lengths {min(w.seqlens)}..{max(w.seqlens)}), H={w.Hq}" if w.packed
+                 else f"B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N}")
+        return (f"{w.name}: {'causal' if w.causal else 'non-causal'} {shape} d={w.d}, "
                 "Q/K/V E4M3 codes of N(0,1)*32 (per-tensor scale 1/32), scale=1/sqrt(d)")
     if w.packed:
         shape = f"packed {w.B} sequences (lengths {min(w.seqlens)}..{max(w.seqlens)}), H={w.Hq}"
@@ -261,7 +263,7 @@ def oracle_rows(w, rows):
         from exact_tiled_attention_32_b200 import synthetic as syn
         s = syn.FP8_SCALE
         return oracle.attention_fp8(w.q, w.k, w.v, s, s, s, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal,
-                                    rows=rows)
+                                    rows=rows, cu_seqlens=w.cu_seqlens)
     if w.chunk:
         return oracle.attention_kv(w.q, w.k, w.v, w.B, w.Hq, w.Hkv, w.N, w.Nk, w.d, w.scale, w.causal,
                                    rows=rows)
@@ -518,7 +520,10 @@ def main():
     fp8_scale = syn.FP8_SCALE
 
     def step():
-        if w.fp8:
+        if w.fp8 and w.packed:
+            rc = fa.fa_fwd_fp8_varlen(q, k, v, o, lse, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal, fp8_scale,
+                                      fp8_scale, fp8_scale, cu, stream)
+        elif w.fp8:
             rc = fa.fa_fwd_fp8(q, k, v, o, lse, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal, fp8_scale, fp8_scale,
                                fp8_scale, stream)
         elif w.decode:
@@ -582,7 +587,7 @@ def main():
             vd = vh.to(dev, non_blocking=True)
             if w.fp8:
                 od, ld = fa.attention_forward_fp8(qd, kd, vd, fp8_scale, fp8_scale, fp8_scale, causal=w.causal,
-                                                  scale=w.scale)
+                                                  scale=w.scale, cu_seqlens=cu)
             elif w.decode:
                 od, ld = fa.attention_forward_splitkv(qd, kd, vd, causal=w.causal, scale=w.scale,
                                                       num_splits=splits, workspace=ws)

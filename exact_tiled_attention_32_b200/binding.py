@@ -31,7 +31,7 @@ FA_ERR_SEQLENS = -9
 EXPORTED = ("fa_fwd", "fa_get_device_status", "fa_status_string", "fa_fwd_noalloc", "fa_fwd_kvcache",
             "fa_selftest_watchdog", "fa_fwd_splitkv", "fa_splitkv_num_splits", "fa_splitkv_workspace_bytes",
             "fa_bwd", "fa_bwd_workspace_bytes", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials",
-            "fa_get_noalloc_status")
+            "fa_get_noalloc_status", "fa_fwd_fp8_varlen", "fa_fwd_kvcache_varlen")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -53,6 +53,8 @@ _lib.fa_fwd_kvcache.argtypes = [
     ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
     ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
 ]
+_lib.fa_fwd_kvcache_varlen.restype = ctypes.c_int
+_lib.fa_fwd_kvcache_varlen.argtypes = _lib.fa_fwd_kvcache.argtypes[:-1] + [ctypes.c_void_p] * 3
 _lib.fa_fwd_splitkv.restype = ctypes.c_int
 _lib.fa_fwd_splitkv.argtypes = _lib.fa_fwd_kvcache.argtypes[:-1] + [
     ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
@@ -70,6 +72,8 @@ _lib.fa_bwd_workspace_bytes.argtypes = [ctypes.c_int] * 5
 _lib.fa_fwd_fp8.restype = ctypes.c_int
 _lib.fa_fwd_fp8.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_int] + \
     [ctypes.c_float] * 3 + [ctypes.c_void_p]
+_lib.fa_fwd_fp8_varlen.restype = ctypes.c_int
+_lib.fa_fwd_fp8_varlen.argtypes = _lib.fa_fwd_fp8.argtypes[:-1] + [ctypes.c_void_p, ctypes.c_void_p]
 _lib.fa_fwd_partial.restype = ctypes.c_int
 _lib.fa_fwd_partial.argtypes = _lib.fa_fwd_kvcache.argtypes
 _lib.fa_merge_partials.restype = ctypes.c_int
@@ -131,14 +135,49 @@ def fa_fwd_kvcache(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream
                                _stream(stream))
 
 
-def attention_forward_kvcache(q, k, v, *, causal: bool = False, scale: float | None = None):
+def fa_fwd_kvcache_varlen(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, cu_seqlens_q, cu_seqlens_k,
+                          stream=None) -> int:
+    """The C entry point for packed query chunks against packed keys."""
+    return _lib.fa_fwd_kvcache_varlen(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), int(B), int(Hq),
+                                      int(Hkv), int(Nq), int(Nk), int(d), float(scale), int(bool(causal)),
+                                      _addr(cu_seqlens_q), _addr(cu_seqlens_k), _stream(stream))
+
+
+def attention_forward_kvcache(q, k, v, *, causal: bool = False, scale: float | None = None,
+                              cu_seqlens_q=None, cu_seqlens_k=None):
     """O, lse for q [B, Hq, Nq, d] against k/v [B, Hkv, Nk, d] (bf16 CUDA
-    tensors); query row i sits at key position Nk - Nq + i."""
+    tensors); query row i sits at key position Nk - Nq + i.  Packed
+    (``cu_seqlens_q`` and ``cu_seqlens_k``, int32 [B+1] CUDA tensors): q
+    [Nq, Hq, d] against k/v [Nk, Hkv, d], sequence s's rows the last of its
+    key positions; returns O [Nq, Hq, d] and lse [Hq, Nq]."""
     import torch
 
     if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
         raise TypeError("q, k, v must be bfloat16")
     q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    if (cu_seqlens_q is None) != (cu_seqlens_k is None):
+        raise ValueError("give both cu_seqlens_q and cu_seqlens_k, or neither")
+    if cu_seqlens_q is not None:
+        for c in (cu_seqlens_q, cu_seqlens_k):
+            if c.dtype != torch.int32 or not c.is_cuda or c.dim() != 1:
+                raise ValueError("cu_seqlens: int32 CUDA tensors [B+1]")
+        if cu_seqlens_q.numel() != cu_seqlens_k.numel():
+            raise ValueError("cu_seqlens_q and cu_seqlens_k must have the same length")
+        if q.dim() != 3 or k.dim() != 3 or k.shape != v.shape:
+            raise ValueError("packed layout: q [Nq,Hq,d], k/v [Nk,Hkv,d]")
+        Nq, Hq, d = q.shape
+        Nk, Hkv = k.shape[0], k.shape[1]
+        if k.shape[2] != d:
+            raise ValueError("k/v shape does not match q")
+        if scale is None:
+            scale = 1.0 / math.sqrt(d)
+        out = torch.empty_like(q)
+        lse = torch.empty((Hq, Nq), dtype=torch.float32, device=q.device)
+        rc = fa_fwd_kvcache_varlen(q, k, v, out, lse, cu_seqlens_q.numel() - 1, Hq, Hkv, Nq, Nk, d, scale, causal,
+                                   cu_seqlens_q, cu_seqlens_k, torch.cuda.current_stream(q.device))
+        if rc != FA_OK:
+            raise FAError(rc, "fa_fwd_kvcache_varlen")
+        return out, lse
     if q.dim() != 4 or k.dim() != 4 or k.shape != v.shape:
         raise ValueError("q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d]")
     B, Hq, Nq, d = q.shape
@@ -276,17 +315,47 @@ def fa_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, q_scale, k_scal
                            _stream(stream))
 
 
+def fa_fwd_fp8_varlen(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, q_scale, k_scale, v_scale, cu_seqlens,
+                      stream=None) -> int:
+    """The C entry point of the FP8 (E4M3) forward on packed sequences."""
+    return _lib.fa_fwd_fp8_varlen(_addr(q), _addr(k), _addr(v), _addr(o), _addr(lse), int(B), int(Hq), int(Hkv),
+                                  int(N), int(d), float(scale), int(bool(causal)), float(q_scale), float(k_scale),
+                                  float(v_scale), _addr(cu_seqlens), _stream(stream))
+
+
 def attention_forward_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: float, *, causal: bool = False,
-                          scale: float | None = None):
-    """O (bf16), lse for E4M3 q [B, Hq, N, d], k/v [B, Hkv, N, d] (CUDA tensors
-    of dtype torch.float8_e4m3fn or uint8 holding E4M3 codes) with per-tensor
-    scales: the values are code * scale."""
+                          scale: float | None = None, cu_seqlens=None):
+    """O (bf16), lse for E4M3 q, k, v (CUDA tensors of dtype
+    torch.float8_e4m3fn or uint8 holding E4M3 codes) with per-tensor scales:
+    the values are code * scale.  Dense: q [B, Hq, N, d], k/v [B, Hkv, N, d];
+    packed (``cu_seqlens`` int32 [B+1] on the device): q [N, Hq, d], k/v
+    [N, Hkv, d], returning O [N, Hq, d] and lse [Hq, N]."""
     import torch
 
     for t in (q, k, v):
         if t.dtype not in (torch.uint8, getattr(torch, "float8_e4m3fn", torch.uint8)):
             raise TypeError("q, k, v must be float8_e4m3fn (or uint8 E4M3 codes)")
     q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    stream = torch.cuda.current_stream(q.device)
+    if cu_seqlens is not None:
+        if q.dim() != 3 or k.dim() != 3 or k.shape != v.shape:
+            raise ValueError("packed layout: q [N,Hq,d], k/v [N,Hkv,d]")
+        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or cu_seqlens.dim() != 1:
+            raise ValueError("cu_seqlens: int32 CUDA tensor [B+1]")
+        N, Hq, d = q.shape
+        Hkv = k.shape[1]
+        if k.shape[0] != N or k.shape[2] != d:
+            raise ValueError("k/v shape does not match q")
+        if scale is None:
+            scale = 1.0 / math.sqrt(d)
+        B = cu_seqlens.numel() - 1
+        out = torch.empty((N, Hq, d), dtype=torch.bfloat16, device=q.device)
+        lse = torch.empty((Hq, N), dtype=torch.float32, device=q.device)
+        rc = fa_fwd_fp8_varlen(q, k, v, out, lse, B, Hq, Hkv, N, d, scale, causal, q_scale, k_scale, v_scale,
+                               cu_seqlens, stream)
+        if rc != FA_OK:
+            raise FAError(rc, "fa_fwd_fp8_varlen")
+        return out, lse
     if q.dim() != 4 or k.dim() != 4 or k.shape != v.shape:
         raise ValueError("dense layout: q [B,Hq,N,d], k/v [B,Hkv,N,d]")
     B, Hq, N, d = q.shape
@@ -297,8 +366,7 @@ def attention_forward_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: floa
         scale = 1.0 / math.sqrt(d)
     out = torch.empty((B, Hq, N, d), dtype=torch.bfloat16, device=q.device)
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
-    rc = fa_fwd_fp8(q, k, v, out, lse, B, Hq, Hkv, N, d, scale, causal, q_scale, k_scale, v_scale,
-                    torch.cuda.current_stream(q.device))
+    rc = fa_fwd_fp8(q, k, v, out, lse, B, Hq, Hkv, N, d, scale, causal, q_scale, k_scale, v_scale, stream)
     if rc != FA_OK:
         raise FAError(rc, "fa_fwd_fp8")
     return out, lse

@@ -89,6 +89,13 @@ template <int D, bool F8>
 __host__ __device__ constexpr int tmem_layout() {
     return F8 ? FA_LAYOUT_F8 : (D == 64 ? FA_LAYOUT_D64 : FA_LAYOUT_D128);
 }
+// kSepP only: the two tiles' exponential phases take turns (tile 0, tile 1,
+// tile 0, ... over the key blocks both tiles of an item visit), so that one
+// tile loads its scores and forms its row maxima while the other keeps the
+// MUFU busy.
+#ifndef FA_TOKEN
+#define FA_TOKEN 0
+#endif
 template <int D, bool F8>
 __host__ __device__ constexpr bool sep_p() {
     return tmem_layout<D, F8>() != kAlias;
@@ -119,6 +126,7 @@ struct alignas(64) Params {
     void* o;
     float* lse;
     const int32_t* cu_seqlens;
+    const int32_t* cu_seqlens_k;   // packed query chunks: key offsets (NULL: the keys are the queries' tokens)
     int* status;
     int B, Hq, Hkv, N;         // N: query rows per sequence (dense) or total tokens (packed)
     int Nk;                    // dense: keys per sequence (== N except for a query chunk)
@@ -161,6 +169,7 @@ struct Misc {
     uint64_t bar_p_half[2][2];     // P_t keys 0-63 / 64-127 are in TMEM
     uint64_t bar_s_free[2];        // separate-P layout: the softmax warps have read S_t
     uint64_t bar_pv_done[2];       // separate-P layout: O_t += P_t V_j has completed
+    uint64_t bar_tok[2];           // kSepP with FA_TOKEN: the exponentials may start (tile t's turn)
     uint32_t tmem_base;
     int abort_flag;
     int bad;
@@ -171,6 +180,7 @@ struct Misc {
 // Packed batches only: the sequence offsets and the pair-level schedule.
 struct SeqTables {
     int seq_off[kMaxSeqs + 1];
+    int kseq_off[kMaxSeqs + 1];   // key offsets (equal to seq_off unless the queries are chunks)
     int order[kMaxSeqs];       // sequences by pair count, descending
     int pcnt[kMaxPairs];       // number of sequences with more than p pairs
     int pstart[kMaxPairs];     // first item index at pair level p
@@ -179,7 +189,7 @@ struct SeqTables {
 template <int D, bool PK, bool F8 = false>
 struct Cfg {
     static_assert(D == 64 || D == 128, "head dim");
-    static_assert(!F8 || (D == 128 && !PK), "FP8: dense batches, d = 128");
+    static_assert(!F8 || D == 128, "FP8: d = 128");
     static constexpr int kElem = F8 ? 1 : 2;                // bytes per element
     static constexpr int kTileBytes = kBlockM * D * kElem;  // one 128 x D tile
     static constexpr int kBoxes = D * kElem / 128;          // 128-byte-wide TMA boxes per tile row
@@ -204,6 +214,7 @@ struct Item {
     int klen;      // keys of the sequence
     int qoff;      // position of query row 0 among the keys
     int tok0;      // packed: first token of the sequence
+    int ktok0;     // packed: first key token of the sequence
     int split;     // split of the key blocks this item covers (0 without splits)
     int j0;        // first key block of the item
     int n[2];      // key blocks each tile visits from j0 on (0: none)
@@ -261,6 +272,7 @@ __device__ __forceinline__ Item decode_item(int idx, const Params& p, const Misc
         it.klen = p.Nk;
         it.qoff = p.q_off;
         it.tok0 = 0;
+        it.ktok0 = 0;
     } else {
         int lo = 0, hi = ms.pmax - 1;      // smallest level whose start <= idx
         while (lo < hi) {
@@ -274,8 +286,9 @@ __device__ __forceinline__ Item decode_item(int idx, const Params& p, const Misc
         it.seq = tab.order[k];
         it.tok0 = tab.seq_off[it.seq];
         it.len = tab.seq_off[it.seq + 1] - it.tok0;
-        it.klen = it.len;
-        it.qoff = 0;
+        it.ktok0 = tab.kseq_off[it.seq];
+        it.klen = tab.kseq_off[it.seq + 1] - it.ktok0;
+        it.qoff = p.causal ? it.klen - it.len : 0;     // a chunk's rows are the last positions
         it.split = 0;
     }
     it.q0 = pair * kRowsPerItem;
@@ -395,7 +408,7 @@ __device__ void load_role(const Params& p, Misc& ms, const SeqTables& tab, uint3
                     if constexpr (!PK)
                         tma_load_4d(dst, map, bar, b * C::kBoxCols, key0, kvh, it.seq, pol_kv);
                     else
-                        tma_load_4d(dst, map, bar, b * C::kBoxCols, kvh, it.tok0 + key0, 0, pol_kv);
+                        tma_load_4d(dst, map, bar, b * C::kBoxCols, kvh, it.ktok0 + key0, 0, pol_kv);
                 }
                 ++kv_it;
                 if (++st == (uint32_t)C::kStages) {
@@ -917,6 +930,8 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
     const float sl2 = p.scale_log2;
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
     uint32_t sc = 0, oc = 0, pw = 0;     // S blocks, O finals, P V completions waited for
+    constexpr bool kTok = FA_TOKEN && tmem_layout<D, F8>() == kSepP;
+    uint32_t tw = 0;                     // turns waited for (phase parity of bar_tok[t])
     bool ok = true;
     for (int rr = 0; ok; ++rr) {
         const int idx = item_of_round(rr);
@@ -935,6 +950,7 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
         const int limit = p.causal ? min(row_pos(row, it.qoff, PK ? 0 : p.qmod) + 1, it.klen) : it.klen;
         float m_used = -INFINITY;    // max the exponentials are taken against (log2 units)
         float l = 0.f;               // running sum of exp2(x - m_used)
+        const int n_common = min(it.n[0], it.n[1]);      // blocks both tiles visit: they take turns
         for (int j = 0; j < n; ++j) {
             if (lane == 0 && wq == 0) FA_TRACE_EV(t, sc, 0);
             ok = wait_bar(smem_u32(&ms.bar_s_full[t]), sc & 1, p, ms, kSiteSFull);
@@ -1025,6 +1041,11 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
             }
             const float msub = ((m_used == -INFINITY) ? 0.f : m_used) - kPShift;
             const uint64_t nm2 = f2_pack(-msub, -msub);
+            if (kTok && j < n_common && !(t == 0 && j == 0)) {
+                ok = wait_bar(smem_u32(&ms.bar_tok[t]), tw & 1, p, ms, kSitePFull);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                ++tw;
+            }
             if (!spec || any_need) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i) acc[i] = 0;
@@ -1062,6 +1083,8 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
             __syncwarp();
             if (lane == 0) FA_TRACE_EV(t, sc - 1, wq == 0 ? 4 : 4 + wq);
             if (lane == 0) mbar_arrive(smem_u32(&ms.bar_p_half[t][1]));
+            if (kTok && j < n_common && !(t == 1 && j == n_common - 1) && lane == 0)
+                mbar_arrive(smem_u32(&ms.bar_tok[1 - t]));            // the other tile's turn
         }
         if (!ok) break;
         // epilogue: O / l -> bf16 -> HBM, and the logsumexp
@@ -1167,6 +1190,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             mbar_init(smem_u32(&ms.bar_o_final[t]), 1);
             mbar_init(smem_u32(&ms.bar_s_free[t]), 4);     // one arrival per warp
             mbar_init(smem_u32(&ms.bar_pv_done[t]), 1);
+            mbar_init(smem_u32(&ms.bar_tok[t]), 4);        // one arrival per warp of the other tile
         }
         ms.abort_flag = 0;
         ms.bad = 0;
@@ -1181,13 +1205,20 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     int total;
     if constexpr (PK) {
         // stage the offsets, check them, and build the pair-level tables
-        for (int i = tid; i <= p.B; i += kThreads) tab.seq_off[i] = p.cu_seqlens[i];
+        for (int i = tid; i <= p.B; i += kThreads) {
+            tab.seq_off[i] = p.cu_seqlens[i];
+            tab.kseq_off[i] = p.cu_seqlens_k ? p.cu_seqlens_k[i] : p.cu_seqlens[i];
+        }
         __syncthreads();
         if (tid == 0) {
-            int bad = tab.seq_off[0] != 0 || tab.seq_off[p.B] != p.N;
+            int bad = tab.seq_off[0] != 0 || tab.seq_off[p.B] != p.N || tab.kseq_off[0] != 0 ||
+                      tab.kseq_off[p.B] != p.Nk;
             for (int s = 0; s < p.B && !bad; ++s) {
                 const int L = tab.seq_off[s + 1] - tab.seq_off[s];
-                if (L < 0 || L > kMaxPairs * kRowsPerItem) bad = 1;
+                const int Lk = tab.kseq_off[s + 1] - tab.kseq_off[s];
+                if (L < 0 || L > kMaxPairs * kRowsPerItem || Lk < 0) bad = 1;
+                if (p.causal && Lk < L) bad = 1;       // a chunk's rows are the last Lk positions
+                if (!p.causal && L > 0 && Lk == 0) bad = 1;
             }
             ms.bad = bad;
         }
@@ -1382,6 +1413,9 @@ int init_device(int dev, DeviceState** out) {
             good = good && cudaFuncSetAttribute(fa_fwd_kernel<128, false, true>,
                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 Cfg<128, false, true>::kSmemBytes) == cudaSuccess;
+            good = good && cudaFuncSetAttribute(fa_fwd_kernel<128, true, true>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                Cfg<128, true, true>::kSmemBytes) == cudaSuccess;
             ds.status_code = good ? FA_OK : FA_ERR_LAUNCH;
         }
     }
@@ -1414,11 +1448,11 @@ static bool make_maps(Params& P, const void* q, const void* k, const void* v, in
     }
     const uint64_t dq[4] = {(uint64_t)d, (uint64_t)Hq, (uint64_t)N, 1};
     const uint64_t sq[3] = {d * e, (uint64_t)Hq * d * e, (uint64_t)N * Hq * d * e};
-    const uint64_t dk[4] = {(uint64_t)d, (uint64_t)Hkv, (uint64_t)N, 1};
-    const uint64_t sk[3] = {d * e, (uint64_t)Hkv * d * e, (uint64_t)N * Hkv * d * e};
-    const uint32_t box[4] = {64, 1, (uint32_t)kBlockM, 1};
-    return encode_map(&P.tm_q, q, dq, sq, box, false) && encode_map(&P.tm_k, k, dk, sk, box, false) &&
-           encode_map(&P.tm_v, v, dk, sk, box, false);
+    const uint64_t dk[4] = {(uint64_t)d, (uint64_t)Hkv, (uint64_t)Nk, 1};
+    const uint64_t sk[3] = {d * e, (uint64_t)Hkv * d * e, (uint64_t)Nk * Hkv * d * e};
+    const uint32_t box[4] = {(uint32_t)(128 / e), 1, (uint32_t)kBlockM, 1};      // 128-byte box rows
+    return encode_map(&P.tm_q, q, dq, sq, box, fp8) && encode_map(&P.tm_k, k, dk, sk, box, fp8) &&
+           encode_map(&P.tm_v, v, dk, sk, box, fp8);
 }
 
 #ifndef FA_L2_GROUP_MIB
@@ -1440,7 +1474,7 @@ static int launch_fwd(const void* q, const void* k, const void* v, void* o, floa
                       int N, int Nk, int q_off, int d, float scale, int causal, const int32_t* cu_seqlens,
                       cudaStream_t s, int* status, int num_sms, int qmod = 0, int splits = 1,
                       float* o_part = nullptr, float* lse_part = nullptr, bool fp8 = false,
-                      float qk_scale = 1.f, float v_scale = 1.f) {
+                      float qk_scale = 1.f, float v_scale = 1.f, const int32_t* cu_seqlens_k = nullptr) {
     const bool packed = cu_seqlens != nullptr;
     Params P;
     std::memset(&P, 0, sizeof(P));
@@ -1448,6 +1482,7 @@ static int launch_fwd(const void* q, const void* k, const void* v, void* o, floa
     P.o = o;
     P.lse = lse;
     P.cu_seqlens = cu_seqlens;
+    P.cu_seqlens_k = cu_seqlens_k;
     P.status = status;
     P.B = B;
     P.Hq = Hq;
@@ -1483,7 +1518,9 @@ static int launch_fwd(const void* q, const void* k, const void* v, void* o, floa
         items = (long long)num_sms;    // exact count is known only on the device
     }
     const int grid = (int)std::min<long long>(items, num_sms);
-    if (fp8)
+    if (fp8 && packed)
+        fa_fwd_kernel<128, true, true><<<grid, kThreads, Cfg<128, true, true>::kSmemBytes, s>>>(P);
+    else if (fp8)
         fa_fwd_kernel<128, false, true><<<grid, kThreads, Cfg<128, false, true>::kSmemBytes, s>>>(P);
     else if (d == 64 && !packed)
         fa_fwd_kernel<64, false><<<grid, kThreads, Cfg<64, false>::kSmemBytes, s>>>(P);
@@ -1552,6 +1589,30 @@ extern "C" int fa_fwd_kvcache(const void* q, const void* k, const void* v, void*
     // the chunk's rows are the last Nq positions of the key sequence
     return launch_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, causal ? Nk - Nq : 0, d, scale, causal, nullptr,
                       static_cast<cudaStream_t>(stream), ds->status, ds->num_sms);
+}
+
+extern "C" int fa_fwd_kvcache_varlen(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                                     int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                                     const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, void* stream) {
+    if (B < 0 || Nq < 0 || Nk < 0 || Hq < 1) return FA_ERR_SHAPE;
+    if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+    if (Hkv < 1 || Hq % Hkv != 0) return FA_ERR_GQA;
+    if (B == 0 || Nq == 0) return FA_OK;
+    if (Nk == 0) return FA_ERR_SHAPE;
+    if (!q || !k || !v || !o || !lse || !cu_seqlens_q || !cu_seqlens_k) return FA_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+        !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4))
+        return FA_ERR_ALIGN;
+    if (B > kMaxSeqs) return FA_ERR_SHAPE;
+    if ((long long)Hq * Nq > (1ll << 30) || (long long)Hkv * Nk > (1ll << 31)) return FA_ERR_SHAPE;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_LAUNCH;
+    DeviceState* ds = nullptr;
+    const int st = init_device(dev, &ds);
+    if (st != FA_OK) return st;
+    return launch_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, 0, d, scale, causal, cu_seqlens_q,
+                      static_cast<cudaStream_t>(stream), ds->status, ds->num_sms, 0, 1, nullptr, nullptr, false, 1.f,
+                      1.f, cu_seqlens_k);
 }
 
 // ------------------------------------------------------------ split keys
@@ -1668,9 +1729,10 @@ extern "C" int fa_fwd_splitkv(const void* q, const void* k, const void* v, void*
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
-extern "C" int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
-                          int N, int d, float scale, int causal, float q_scale, float k_scale, float v_scale,
-                          void* stream) {
+static int fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+                   int d, float scale, int causal, float q_scale, float k_scale, float v_scale,
+                   const int32_t* cu_seqlens, void* stream) {
+    const bool packed = cu_seqlens != nullptr;
     if (B < 0 || N < 0 || Hq < 1) return FA_ERR_SHAPE;
     if (d != 128) return FA_ERR_HEADDIM;
     if (Hkv < 1 || Hq % Hkv != 0) return FA_ERR_GQA;
@@ -1681,14 +1743,29 @@ extern "C" int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, 
     if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
         return FA_ERR_ALIGN;
-    if ((long long)B * Hq * N > (1ll << 30)) return FA_ERR_SHAPE;
+    if (packed && (B > kMaxSeqs || !aligned(cu_seqlens, 4))) return B > kMaxSeqs ? FA_ERR_SHAPE : FA_ERR_ALIGN;
+    if ((packed ? (long long)Hq * N : (long long)B * Hq * N) > (1ll << 30)) return FA_ERR_SHAPE;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_LAUNCH;
     DeviceState* ds = nullptr;
     const int st = init_device(dev, &ds);
     if (st != FA_OK) return st;
-    return launch_fwd(q, k, v, o, lse, B, Hq, Hkv, N, N, 0, d, scale, causal, nullptr, static_cast<cudaStream_t>(stream),
-                      ds->status, ds->num_sms, 0, 1, nullptr, nullptr, true, q_scale * k_scale, v_scale);
+    return launch_fwd(q, k, v, o, lse, B, Hq, Hkv, N, N, 0, d, scale, causal, cu_seqlens,
+                      static_cast<cudaStream_t>(stream), ds->status, ds->num_sms, 0, 1, nullptr, nullptr, true,
+                      q_scale * k_scale, v_scale);
+}
+
+extern "C" int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                          int N, int d, float scale, int causal, float q_scale, float k_scale, float v_scale,
+                          void* stream) {
+    return fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, q_scale, k_scale, v_scale, nullptr, stream);
+}
+
+extern "C" int fa_fwd_fp8_varlen(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                                 int Hkv, int N, int d, float scale, int causal, float q_scale, float k_scale,
+                                 float v_scale, const int32_t* cu_seqlens, void* stream) {
+    if (!cu_seqlens && B > 0 && N > 0) return FA_ERR_NULL;
+    return fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, q_scale, k_scale, v_scale, cu_seqlens, stream);
 }
 
 extern "C" int fa_fwd_partial(const void* q, const void* k, const void* v, float* o_part, float* lse_part, int B,

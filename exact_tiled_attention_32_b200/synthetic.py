@@ -297,7 +297,7 @@ def packed_from_lengths(name, lens, H, d, causal, seed, Hkv=None) -> Workload:
 
 
 def config(name: str) -> Workload:
-    """The named workloads c1, c2nc, c2c, c3, c4, c5, p3, dec, c3f8 (inputs not yet drawn)."""
+    """The named workloads c1, c2nc, c2c, c3, c4, c5, p3, dec, c3f8, c5f8 (inputs not yet drawn)."""
     if name == "c1":
         return Workload("c1", 1, 1, 1, 256, 64, False, 1001)
     if name == "c2nc":
@@ -317,6 +317,11 @@ def config(name: str) -> Workload:
     if name == "c3f8":
         # c3 with Q, K, V in E4M3 (per-tensor scale 1/32)
         return Workload("c3f8", 1, 32, 32, 16384, 128, True, 1008, fp8=True)
+    if name == "c5f8":
+        # c5's packed batch (same lengths) with E4M3 inputs
+        w = packed_workload("c5f8", 16, 512, 8192, 16, 128, True, 1005)
+        w.fp8 = True
+        return w
     if name == "dec":
         # one new token per sequence of a batch of 8 against a 32768-token
         # cache, c4's grouped heads
@@ -324,4 +329,4 @@ def config(name: str) -> Workload:
     raise KeyError(name)
 
 
-CONFIGS = ("c1", "c2nc", "c2c", "c3", "c4", "c5", "p3", "dec", "c3f8")
+CONFIGS = ("c1", "c2nc", "c2c", "c3", "c4", "c5", "p3", "dec", "c3f8", "c5f8")

@@ -128,6 +128,45 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
                float q_scale, float k_scale, float v_scale, void* stream);
 
 /*
+ * fa_fwd_fp8_varlen -- fa_fwd_fp8 on a packed batch of variable-length
+ * sequences ("Flash Attention" page, "Flash Attention 2 Improvements":
+ * variable sequence lengths; "FlashAttention and Chunked Prefill Mechanics",
+ * section 1: FP8).  Layouts, masks and errors are those of fa_fwd with
+ * cu_seqlens != NULL (q, o [N_total, Hq, 128]; k, v [N_total, Hkv, 128];
+ * lse [Hq, N_total]; cu_seqlens int32 [B + 1] on the device with
+ * cu_seqlens[B] == N, checked on the device: FA_ERR_SEQLENS through
+ * fa_get_device_status), with E4M3 q, k, v codes and per-tensor scales as
+ * fa_fwd_fp8.  cu_seqlens must not be NULL (FA_ERR_NULL) unless B or N is 0.
+ */
+int fa_fwd_fp8_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                      int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                      float q_scale, float k_scale, float v_scale, const int32_t* cu_seqlens,
+                      void* stream);
+
+/*
+ * fa_fwd_kvcache_varlen -- fa_fwd_kvcache on a packed batch: B sequences, each
+ * with its own query chunk against its own keys ("FlashAttention and Chunked
+ * Prefill Mechanics", section 1: a prefill split into chunks, the chunks of
+ * several requests run together; "Flash Attention" page, "Flash Attention 2
+ * Improvements": variable sequence lengths).  Sequence s has query rows
+ * [cu_seqlens_q[s], cu_seqlens_q[s+1]) and keys [cu_seqlens_k[s],
+ * cu_seqlens_k[s+1]) (both int32 [B + 1] on the device); its Lq rows are the
+ * last Lq of its Lk positions, so with causal row i may attend keys
+ * 0 .. Lk - Lq + i (bottom-right alignment; Lk >= Lq is required).
+ *   q, o   [Nq, Hq, d] bf16 (Nq = cu_seqlens_q[B] query tokens in total)
+ *   k, v   [Nk, Hkv, d] bf16 (Nk = cu_seqlens_k[B] key tokens in total)
+ *   lse    [Hq, Nq] fp32
+ * The offsets are checked on the device (starts at 0, totals Nq and Nk, no
+ * negative lengths, Lk >= Lq when causal, Lk > 0 for a non-empty chunk when
+ * not causal): a failure writes nothing and reports FA_ERR_SEQLENS through
+ * fa_get_device_status.  Host errors: as fa_fwd; FA_ERR_NULL also for a NULL
+ * offset array, FA_ERR_SHAPE for B > 1024.  A sequence may have Lq = 0.
+ */
+int fa_fwd_kvcache_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                          const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, void* stream);
+
+/*
  * fa_fwd_partial -- one key range's share of the forward, for merging later
  * (ring attention, any split of the keys).  Same arguments, layouts and
  * masks as fa_fwd_kvcache (query row i at key position Nk - Nq + i), but the

@@ -268,18 +268,19 @@ def _exact_bf16_bits(x: np.ndarray) -> np.ndarray:
 
 
 def attention_fp8(q8, k8, v8, q_scale, k_scale, v_scale, B, Hq, Hkv, N, d, scale, causal, rows=None,
-                  nthreads=0, lib=None, abs_v=False) -> tuple[np.ndarray, np.ndarray]:
+                  nthreads=0, lib=None, abs_v=False, cu_seqlens=None) -> tuple[np.ndarray, np.ndarray]:
     """Standard attention, in fp64, of the dequantised E4M3 inputs
-    (value = e4m3_decode(code) * tensor scale).  Dense layouts as
-    ``attention``.  With power-of-two scales every dequantised value is exact
-    in bf16, so the fp64 materialised attention of ``oracle.c`` runs on them
-    unchanged.  ``abs_v``: use |V| (gives sum_j p_j |v_j| per row, the
-    weight the FP8 tolerance is stated in)."""
+    (value = e4m3_decode(code) * tensor scale).  Dense or packed
+    (``cu_seqlens``) layouts as ``attention``.  With power-of-two scales every
+    dequantised value is exact in bf16, so the fp64 materialised attention of
+    ``oracle.c`` runs on them unchanged.  ``abs_v``: use |V| (gives
+    sum_j p_j |v_j| per row, the weight the FP8 tolerance is stated in)."""
     qb = _exact_bf16_bits(e4m3_decode(q8) * q_scale)
     kb = _exact_bf16_bits(e4m3_decode(k8) * k_scale)
     vv = e4m3_decode(v8) * v_scale
     vb = _exact_bf16_bits(np.abs(vv) if abs_v else vv)
-    return attention(qb, kb, vb, B, Hq, Hkv, N, d, scale, causal, rows=rows, nthreads=nthreads, lib=lib)
+    return attention(qb, kb, vb, B, Hq, Hkv, N, d, scale, causal, cu_seqlens=cu_seqlens, rows=rows,
+                     nthreads=nthreads, lib=lib)
 
 
 def num_threads() -> int:

@@ -189,6 +189,35 @@ def test_fp8_argument_errors_found_on_the_host():
     assert call(B=0, ptrs=(0,) * 5) == fa.FA_OK
 
 
+def test_fp8_varlen_argument_errors_found_on_the_host():
+    from exact_tiled_attention_32_b200 import binding as fa
+    p = 1 << 20
+
+    def call(B=2, d=128, cu=p, ptrs=(p, p, p, p, p)):
+        return fa.fa_fwd_fp8_varlen(*ptrs, B, 2, 2, 128, d, 0.1, 1, 1, 1, 1, cu)
+    assert call(d=64) == fa.FA_ERR_HEADDIM
+    assert call(cu=0) == fa.FA_ERR_NULL
+    assert call(cu=p + 2) == fa.FA_ERR_ALIGN
+    assert call(B=1025) == fa.FA_ERR_SHAPE
+    assert call(ptrs=(p, p, p, p, p + 2)) == fa.FA_ERR_ALIGN
+    assert call(B=0, cu=0, ptrs=(0,) * 5) == fa.FA_OK
+
+
+def test_kvcache_varlen_argument_errors_found_on_the_host():
+    from exact_tiled_attention_32_b200 import binding as fa
+    p = 1 << 20
+
+    def call(B=2, Nq=64, Nk=256, d=128, cq=p, ck=p, ptrs=(p, p, p, p, p)):
+        return fa.fa_fwd_kvcache_varlen(*ptrs, B, 4, 2, Nq, Nk, d, 0.1, 1, cq, ck)
+    assert call(d=80) == fa.FA_ERR_HEADDIM
+    assert call(cq=0) == fa.FA_ERR_NULL
+    assert call(ck=0) == fa.FA_ERR_NULL
+    assert call(ck=p + 2) == fa.FA_ERR_ALIGN
+    assert call(B=1025) == fa.FA_ERR_SHAPE
+    assert call(Nk=0) == fa.FA_ERR_SHAPE
+    assert call(Nq=0, ptrs=(0,) * 5, cq=0, ck=0) == fa.FA_OK
+
+
 def test_no_device_means_launch_error():
     import torch
     if torch.cuda.is_available():

@@ -110,6 +110,56 @@ def test_fp8_all_rows(B, Hq, Hkv, N, causal):
     _check(w, o, lse, np.arange(B * Hq * N), f"fp8 {B},{Hq},{Hkv},{N},{causal}")
 
 
+PACKED = [
+    # lengths, Hq, Hkv, causal
+    ([300, 1, 129, 0, 513], 4, 2, True),
+    ([300, 1, 129, 0, 513], 4, 2, False),
+    ([128, 256, 77], 2, 1, True),
+]
+
+
+@pytest.mark.parametrize("lens,Hq,Hkv,causal", PACKED)
+def test_fp8_packed_every_sequence(lens, Hq, Hkv, causal):
+    """fa_fwd_fp8_varlen against the oracle, sequence by sequence: each
+    sequence's rows are compared with those of the dense problem of that
+    sequence alone, under the same per-element and mean bounds."""
+    import torch
+    from exact_tiled_attention_32_b200 import binding as fa
+    w = syn.packed_from_lengths("fp8p", lens, Hq, 128, causal, 1200 + sum(lens), Hkv=Hkv)
+    w.fp8 = True
+    w.draw()
+    cu = torch.from_numpy(w.cu_seqlens).cuda()
+    o, lse = fa.attention_forward_fp8(_dev(w.q), _dev(w.k), _dev(w.v), S, S, S, causal=causal, scale=w.scale,
+                                      cu_seqlens=cu)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status() == 0
+    o = o.float().cpu().numpy().astype(np.float64)          # [N, Hq, d]
+    lse = lse.cpu().numpy().astype(np.float64)               # [Hq, N]
+    for s_, L in enumerate(lens):
+        if L == 0:
+            continue
+        a = int(w.cu_seqlens[s_])
+        ws = syn.Workload("fp8seq", 1, Hq, Hkv, L, 128, causal, 0, fp8=True)
+        ws.q = np.ascontiguousarray(w.q[a:a + L].transpose(1, 0, 2)[None])
+        ws.k = np.ascontiguousarray(w.k[a:a + L].transpose(1, 0, 2)[None])
+        ws.v = np.ascontiguousarray(w.v[a:a + L].transpose(1, 0, 2)[None])
+        od = o[a:a + L].transpose(1, 0, 2).reshape(-1, 128)
+        ld = lse[:, a:a + L].reshape(-1)
+        _check(ws, od, ld, np.arange(Hq * L), f"fp8 packed {lens} seq {s_}")
+
+
+def test_fp8_varlen_argument_errors():
+    from exact_tiled_attention_32_b200 import binding as fa
+    p = 1 << 20
+    call = lambda B=2, d=128, cu=p, ptrs=(p, p, p, p, p): fa.fa_fwd_fp8_varlen(*ptrs, B, 2, 2, 128, d, 0.1, 1,
+                                                                               1, 1, 1, cu)
+    assert call(d=64) == fa.FA_ERR_HEADDIM
+    assert call(cu=0) == fa.FA_ERR_NULL
+    assert call(cu=p + 2) == fa.FA_ERR_ALIGN
+    assert call(B=1025) == fa.FA_ERR_SHAPE
+    assert call(B=0, cu=0, ptrs=(0,) * 5) == fa.FA_OK
+
+
 def test_fp8_argument_errors():
     from exact_tiled_attention_32_b200 import binding as fa
     p = 1 << 20

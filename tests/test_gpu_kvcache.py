@@ -67,6 +67,73 @@ def test_chunked_prefill_matches_whole_forward():
     assert mx <= 1e-2 and mean <= 1e-3 and lmx <= 1e-3
 
 
+PACKED = [
+    # (Lq, Lk) per sequence, Hq, Hkv, d, causal
+    ([(1, 1000), (130, 130), (0, 77), (200, 777), (257, 1024)], 4, 2, 128, True),
+    ([(5, 300), (128, 4096), (1, 1)], 2, 1, 64, True),
+    ([(100, 513), (7, 9), (0, 0), (300, 301)], 2, 2, 128, False),
+]
+
+
+@pytest.mark.parametrize("pairs,Hq,Hkv,d,causal", PACKED)
+def test_packed_chunks_every_sequence(pairs, Hq, Hkv, d, causal):
+    """fa_fwd_kvcache_varlen: each sequence's chunk against its own keys,
+    compared with the oracle of that sequence's dense chunk problem."""
+    import torch
+    from exact_tiled_attention_32_b200 import binding as fa
+    lq = [a for a, _ in pairs]
+    lk = [b for _, b in pairs]
+    Nq, Nk = sum(lq), sum(lk)
+    st = syn.Stream(900 + Nq + Nk)
+    qb = st.normal_bf16((Nq, Hq, d))
+    kb = st.normal_bf16((Nk, Hkv, d))
+    vb = st.normal_bf16((Nk, Hkv, d))
+    cq = np.concatenate([[0], np.cumsum(lq)]).astype(np.int32)
+    ck = np.concatenate([[0], np.cumsum(lk)]).astype(np.int32)
+    scale = 1.0 / np.sqrt(d)
+    o, lse = fa.attention_forward_kvcache(to_device(qb), to_device(kb), to_device(vb), causal=causal, scale=scale,
+                                          cu_seqlens_q=torch.from_numpy(cq).cuda(),
+                                          cu_seqlens_k=torch.from_numpy(ck).cuda())
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status() == 0
+    o = o.float().cpu().numpy().astype(np.float64)
+    lse = lse.cpu().numpy().astype(np.float64)
+    for s_, (Lq, Lk) in enumerate(pairs):
+        if Lq == 0:
+            continue
+        a, b = int(cq[s_]), int(ck[s_])
+        dense = lambda x, lo, n: np.ascontiguousarray(x[lo:lo + n].transpose(1, 0, 2)[None])
+        oo, lo = oracle.attention_kv(dense(qb, a, Lq), dense(kb, b, Lk), dense(vb, b, Lk), 1, Hq, Hkv, Lq, Lk, d,
+                                     scale, causal)
+        got_o = o[a:a + Lq].transpose(1, 0, 2).reshape(-1, d)
+        got_l = lse[:, a:a + Lq].reshape(-1)
+        assert_parity(got_o, got_l, oo, lo, f"packed chunk seq {s_} ({Lq} x {Lk})")
+
+
+def test_packed_chunks_bad_offsets_reported_by_device():
+    import torch
+    from exact_tiled_attention_32_b200 import binding as fa
+    H, d = 2, 64
+    q = torch.zeros((20, H, d), dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros((30, H, d), dtype=torch.bfloat16, device="cuda")
+    o = torch.full_like(q, 3.0)
+    lse = torch.zeros((H, 20), dtype=torch.float32, device="cuda")
+    s = torch.cuda.current_stream()
+    good_q = torch.tensor([0, 10, 20], dtype=torch.int32, device="cuda")
+    for cq, ck in (([0, 10, 20], [0, 5, 30]),     # causal: 10 rows against 5 keys
+                   ([0, 10, 20], [0, 15, 29]),    # keys do not total Nk
+                   ([0, 10, 20], [1, 15, 30]),    # keys do not start at 0
+                   ([0, 12, 20], [0, 25, 30])):   # causal: 8 rows against 5 keys
+        cqt = torch.tensor(cq, dtype=torch.int32, device="cuda")
+        ckt = torch.tensor(ck, dtype=torch.int32, device="cuda")
+        assert fa.fa_fwd_kvcache_varlen(q, kv, kv, o, lse, 2, H, H, 20, 30, d, 0.1, 1, cqt, ckt, s) == fa.FA_OK
+        assert fa.fa_get_device_status(s) == fa.FA_ERR_SEQLENS, (cq, ck)
+        assert torch.all(o == 3.0)
+    ok_k = torch.tensor([0, 15, 30], dtype=torch.int32, device="cuda")
+    assert fa.fa_fwd_kvcache_varlen(q, kv, kv, o, lse, 2, H, H, 20, 30, d, 0.1, 1, good_q, ok_k, s) == fa.FA_OK
+    assert fa.fa_get_device_status(s) == fa.FA_OK
+
+
 def test_chunk_argument_errors():
     from exact_tiled_attention_32_b200 import binding as fa
     p = 1 << 20
