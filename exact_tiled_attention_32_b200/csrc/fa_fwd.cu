@@ -77,7 +77,7 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only past 2
 // block j ends; the tensor core runs the other tile's work meanwhile.
 enum TmemLayout : int { kAlias = 0, kSepP = 1, kSharedS = 2 };
 #ifndef FA_LAYOUT_D64
-#define FA_LAYOUT_D64 0
+#define FA_LAYOUT_D64 2
 #endif
 #ifndef FA_LAYOUT_D128
 #define FA_LAYOUT_D128 2
@@ -95,6 +95,9 @@ __host__ __device__ constexpr int tmem_layout() {
 // MUFU busy.
 #ifndef FA_TOKEN
 #define FA_TOKEN 0
+#endif
+#ifndef FA_OFFSET_NS
+#define FA_OFFSET_NS 0
 #endif
 template <int D, bool F8>
 __host__ __device__ constexpr bool sep_p() {
@@ -214,7 +217,6 @@ struct Item {
     int klen;      // keys of the sequence
     int qoff;      // position of query row 0 among the keys
     int tok0;      // packed: first token of the sequence
-    int ktok0;     // packed: first key token of the sequence
     int split;     // split of the key blocks this item covers (0 without splits)
     int j0;        // first key block of the item
     int n[2];      // key blocks each tile visits from j0 on (0: none)
@@ -272,7 +274,6 @@ __device__ __forceinline__ Item decode_item(int idx, const Params& p, const Misc
         it.klen = p.Nk;
         it.qoff = p.q_off;
         it.tok0 = 0;
-        it.ktok0 = 0;
     } else {
         int lo = 0, hi = ms.pmax - 1;      // smallest level whose start <= idx
         while (lo < hi) {
@@ -286,8 +287,7 @@ __device__ __forceinline__ Item decode_item(int idx, const Params& p, const Misc
         it.seq = tab.order[k];
         it.tok0 = tab.seq_off[it.seq];
         it.len = tab.seq_off[it.seq + 1] - it.tok0;
-        it.ktok0 = tab.kseq_off[it.seq];
-        it.klen = tab.kseq_off[it.seq + 1] - it.ktok0;
+        it.klen = tab.kseq_off[it.seq + 1] - tab.kseq_off[it.seq];
         it.qoff = p.causal ? it.klen - it.len : 0;     // a chunk's rows are the last positions
         it.split = 0;
     }
@@ -395,6 +395,7 @@ __device__ void load_role(const Params& p, Misc& ms, const SeqTables& tab, uint3
         }
         ++item_n;
         const int kvh = it.h / p.group;
+        const int ktok0 = PK ? tab.kseq_off[it.seq] : 0;      // packed: the sequence's first key token
         const int nmax = max(it.n[0], it.n[1]);
         for (int j = 0; j < nmax && ok; ++j) {
             for (int kind = 0; kind < 2; ++kind) {       // K_j then V_j
@@ -408,7 +409,7 @@ __device__ void load_role(const Params& p, Misc& ms, const SeqTables& tab, uint3
                     if constexpr (!PK)
                         tma_load_4d(dst, map, bar, b * C::kBoxCols, key0, kvh, it.seq, pol_kv);
                     else
-                        tma_load_4d(dst, map, bar, b * C::kBoxCols, kvh, it.ktok0 + key0, 0, pol_kv);
+                        tma_load_4d(dst, map, bar, b * C::kBoxCols, kvh, ktok0 + key0, 0, pol_kv);
                 }
                 ++kv_it;
                 if (++st == (uint32_t)C::kStages) {
@@ -733,15 +734,18 @@ __device__ void mma_role_split(const Params& p, Misc& ms, const SeqTables& tab, 
                         }
                         if (elect_one()) {
                             constexpr uint32_t idesc = idesc_bf16_f32(kBlockM, kBlockN, false);
+                            FA_TRACE_EV(2, 512 + tj, 3 * t);
                             if constexpr (D == 128)
                                 umma_ss_x8_pre(tmem + tmem_s_col<D, F8>(t), ad, bd, idesc);
                             else
                                 umma_ss_x4_pre(tmem + tmem_s_col<D, F8>(t), ad, bd, idesc);
+                            FA_TRACE_EV(2, 512 + tj, 3 * t + 1);
                             umma_commit(smem_u32(&ms.bar_s_full[t]));
                             if (t == 1 || j >= it.n[1]) {
                                 umma_commit(smem_u32(&ms.bar_kv_empty[kst]));
                                 if (j == nmax - 1) umma_commit(smem_u32(&ms.bar_q_empty));
                             }
+                            FA_TRACE_EV(2, 512 + tj, 3 * t + 2);
                         }
                     } else if (elect_one()) {
                         issue_qk<D, F8>(tmem + tmem_s_col<D, F8>(t), dq0 + t * kTileStep, dk0 + kst * kTileStep);
@@ -829,8 +833,16 @@ __device__ void mma_role_split(const Params& p, Misc& ms, const SeqTables& tab, 
 // column pairs (of every 8) on the polynomial, per path: FP8 (tensor work per
 // block half as long as bf16's, as many exponentials), bf16 d = 64 (the
 // exponentials cost twice the block's MMAs), bf16 d = 128 (equal costs)
+// exponentials on the MUFU in pairs (ex2.approx.f16x2): the argument rounded
+// to half precision (relative 2^-11) and the result too; off by default
+#ifndef FA_EXP_F16
+#define FA_EXP_F16 0
+#endif
+#ifndef FA_EXP_F16_F8
+#define FA_EXP_F16_F8 0
+#endif
 #ifndef FA_POLY_PAIRS_PER8_D64
-#define FA_POLY_PAIRS_PER8_D64 0
+#define FA_POLY_PAIRS_PER8_D64 2
 #endif
 template <int D, bool F8>
 __host__ __device__ constexpr int poly_pairs_per8() {
@@ -893,6 +905,11 @@ __device__ __forceinline__ void exp_half(const uint32_t (&s)[128], uint64_t sl2x
         uint64_t e;
         if ((gi % 8) < NPOLY) {
             e = exp2_poly2(x);
+        } else if (F8 ? FA_EXP_F16_F8 : FA_EXP_F16) {
+            float x0, x1, y0, y1;
+            f2_unpack(x, x0, x1);
+            ex2_f16x2(x0, x1, y0, y1);
+            e = f2_pack(y0, y1);
         } else {
             float x0, x1;
             f2_unpack(x, x0, x1);
@@ -930,8 +947,10 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
     const float sl2 = p.scale_log2;
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
     uint32_t sc = 0, oc = 0, pw = 0;     // S blocks, O finals, P V completions waited for
-    constexpr bool kTok = FA_TOKEN && tmem_layout<D, F8>() == kSepP;
+#if FA_TOKEN
+    constexpr bool kTok = tmem_layout<D, F8>() == kSepP;
     uint32_t tw = 0;                     // turns waited for (phase parity of bar_tok[t])
+#endif
     bool ok = true;
     for (int rr = 0; ok; ++rr) {
         const int idx = item_of_round(rr);
@@ -948,9 +967,18 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
         }
         // keys [0, limit) are allowed for this row (causal: up to its own position)
         const int limit = p.causal ? min(row_pos(row, it.qoff, PK ? 0 : p.qmod) + 1, it.klen) : it.klen;
+#if FA_OFFSET_NS > 0
+        // separate S buffers: start tile 1 a fraction of a block behind tile 0, so
+        // that one tile's loads and maxima overlap the other's exponentials
+        if constexpr (tmem_layout<D, F8>() == kSepP) {
+            if (t == 1) __nanosleep(FA_OFFSET_NS);
+        }
+#endif
         float m_used = -INFINITY;    // max the exponentials are taken against (log2 units)
         float l = 0.f;               // running sum of exp2(x - m_used)
+#if FA_TOKEN
         const int n_common = min(it.n[0], it.n[1]);      // blocks both tiles visit: they take turns
+#endif
         for (int j = 0; j < n; ++j) {
             if (lane == 0 && wq == 0) FA_TRACE_EV(t, sc, 0);
             ok = wait_bar(smem_u32(&ms.bar_s_full[t]), sc & 1, p, ms, kSiteSFull);
@@ -1041,11 +1069,13 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
             }
             const float msub = ((m_used == -INFINITY) ? 0.f : m_used) - kPShift;
             const uint64_t nm2 = f2_pack(-msub, -msub);
+#if FA_TOKEN
             if (kTok && j < n_common && !(t == 0 && j == 0)) {
                 ok = wait_bar(smem_u32(&ms.bar_tok[t]), tw & 1, p, ms, kSitePFull);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 ++tw;
             }
+#endif
             if (!spec || any_need) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i) acc[i] = 0;
@@ -1083,8 +1113,10 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
             __syncwarp();
             if (lane == 0) FA_TRACE_EV(t, sc - 1, wq == 0 ? 4 : 4 + wq);
             if (lane == 0) mbar_arrive(smem_u32(&ms.bar_p_half[t][1]));
+#if FA_TOKEN
             if (kTok && j < n_common && !(t == 1 && j == n_common - 1) && lane == 0)
                 mbar_arrive(smem_u32(&ms.bar_tok[1 - t]));            // the other tile's turn
+#endif
         }
         if (!ok) break;
         // epilogue: O / l -> bf16 -> HBM, and the logsumexp

@@ -539,6 +539,17 @@ __device__ __forceinline__ float ex2_approx(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+// 2^x of a pair of floats through the half-precision MUFU form: the pair is
+// rounded to f16x2 (round to nearest), ex2.approx.f16x2 gives two f16
+// results, widened back to fp32 (lo in the first output)
+__device__ __forceinline__ void ex2_f16x2(float x0, float x1, float& y0, float& y1) {
+    uint32_t h, r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(x1), "f"(x0));
+    asm("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(h));
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "cvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
+        : "=f"(y0), "=f"(y1) : "r"(r));
+}
 // pack four fp32 into four E4M3 bytes (round to nearest even, finite values
 // beyond 448 saturate); a0 lands in bits 0-7
 __device__ __forceinline__ uint32_t pack_e4m3x4(float a0, float a1, float a2, float a3) {
