@@ -10,23 +10,24 @@
 // B200 mapping (one persistent CTA per SM, 384 threads, warp-specialised):
 //   warps 0-3   query tile 0, warps 4-7 query tile 1 (one warpgroup each):
 //               one thread per query row; tcgen05.ld of S, masking, running
-//               max in the log2 domain, exp2 via one FFMA + ex2, lazy rescale of
-//               O in TMEM (only when the max grows by more than 2^8), bf16 P
-//               written back to TMEM over S, and the epilogue O / l -> bf16 ->
-//               HBM plus the logsumexp.
-//   warp 10     MMA issuer (one thread): S_t = Q_t K_j^T and O_t += P_t V_j as
-//               tcgen05.mma kind::f16 (bf16 in, fp32 accumulate in TMEM); the A
-//               operand of P_t V_j is read straight from TMEM.  A single issuer
-//               keeps the two tiles' MMA batches alternating, which keeps the two
-//               softmax warpgroups out of phase (ping-pong).
+//               max in the log2 domain, exp2 via one FFMA + ex2 (some column
+//               pairs on an FMA-pipe polynomial at d = 64), lazy rescale of O
+//               in TMEM (only when the max grows by more than 2^8), bf16 P
+//               written to TMEM, and the epilogue O / l -> bf16 -> HBM plus
+//               the logsumexp.
+//   warp 10     MMA issuer: S_t = Q_t K_j^T as tcgen05.mma kind::f16 (bf16 in,
+//               fp32 accumulate in TMEM); with the shared-S layout (bf16) it
+//               issues only these, as soon as the shared S buffer is free.
+//   warp 9      TMEM allocation; with the shared-S layout, the second MMA
+//               issuer: O_t += P_t V_j with P read from TMEM, as soon as P_t
+//               is written.  (FP8: warp 10 issues both kinds, in an order
+//               that keeps the two softmax warpgroups out of phase.)
 //   warp 11     TMA producer: Q (two 128-row tiles per work item) and a ring of
 //               K_j / V_j tiles in 128-byte-swizzled shared memory.
-//   warps 8-9   idle apart from TMEM allocation (warp 9); they complete the
-//               third warpgroup, which gives registers to the softmax
-//               warpgroups through setmaxnreg.
+//   warp 8      idle; it completes the third warpgroup, which gives registers
+//               to the softmax warpgroups through setmaxnreg.
 //
-// TMEM columns (512 allocated): S0/P0 [0,128), S1/P1 [128,256),
-// O0 [256, 256+D), O1 [384, 384+D).
+// TMEM (512 columns): see TmemLayout below.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -59,6 +60,15 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxStages = 10;
 constexpr int kBoxBytes = kBlockM * 64 * 2;   // one 128-row x 64-column bf16 TMA box
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only past 2^8
+// FP8: P is computed as 2^kF8Shift * exp2(x - m_used) and must stay within
+// E4M3's largest value (448 = 2^8.807): with the reference m_used at most
+// kF8Threshold below the row's true maximum, P <= 2^(kF8Shift + kF8Threshold).
+#ifndef FA_F8_THRESHOLD
+#define FA_F8_THRESHOLD 0.0f
+#endif
+constexpr float kF8Threshold = FA_F8_THRESHOLD;
+constexpr float kF8Shift = FA_F8_THRESHOLD > 0.f ? 8.75f - FA_F8_THRESHOLD : 8.0f;
+static_assert(kF8Shift + kF8Threshold <= 8.8f, "FP8 P must stay below 448");
 
 // TMEM layouts (512 columns), per path:
 //  kAlias   S0/P0 [0,128), S1/P1 [128,256), O0 [256,384), O1 [384,512):
@@ -89,16 +99,7 @@ template <int D, bool F8>
 __host__ __device__ constexpr int tmem_layout() {
     return F8 ? FA_LAYOUT_F8 : (D == 64 ? FA_LAYOUT_D64 : FA_LAYOUT_D128);
 }
-// kSepP only: the two tiles' exponential phases take turns (tile 0, tile 1,
-// tile 0, ... over the key blocks both tiles of an item visit), so that one
-// tile loads its scores and forms its row maxima while the other keeps the
-// MUFU busy.
-#ifndef FA_TOKEN
-#define FA_TOKEN 0
-#endif
-#ifndef FA_OFFSET_NS
-#define FA_OFFSET_NS 0
-#endif
+
 template <int D, bool F8>
 __host__ __device__ constexpr bool sep_p() {
     return tmem_layout<D, F8>() != kAlias;
@@ -172,7 +173,6 @@ struct Misc {
     uint64_t bar_p_half[2][2];     // P_t keys 0-63 / 64-127 are in TMEM
     uint64_t bar_s_free[2];        // separate-P layout: the softmax warps have read S_t
     uint64_t bar_pv_done[2];       // separate-P layout: O_t += P_t V_j has completed
-    uint64_t bar_tok[2];           // kSepP with FA_TOKEN: the exponentials may start (tile t's turn)
     uint32_t tmem_base;
     int abort_flag;
     int bad;
@@ -327,17 +327,9 @@ constexpr uint32_t kSuspendNs = FA_SUSPEND_NS;
 
 // Bounded wait: gives up after timeout_ns (recording the site in the status
 // word and raising the CTA's abort flag) or as soon as another role aborted.
-#ifndef FA_SPIN
-#define FA_SPIN 0
-#endif
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Params& p, Misc& ms,
                                       int site) {
     if (mbar_try_wait(bar, parity)) return true;
-#if FA_SPIN > 0
-    // a short busy poll first: a phase that completes within it is seen at once
-    for (int i = 0; i < FA_SPIN; ++i)
-        if (mbar_test_wait(bar, parity)) return true;
-#endif
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
@@ -833,14 +825,6 @@ __device__ void mma_role_split(const Params& p, Misc& ms, const SeqTables& tab, 
 // column pairs (of every 8) on the polynomial, per path: FP8 (tensor work per
 // block half as long as bf16's, as many exponentials), bf16 d = 64 (the
 // exponentials cost twice the block's MMAs), bf16 d = 128 (equal costs)
-// exponentials on the MUFU in pairs (ex2.approx.f16x2): the argument rounded
-// to half precision (relative 2^-11) and the result too; off by default
-#ifndef FA_EXP_F16
-#define FA_EXP_F16 0
-#endif
-#ifndef FA_EXP_F16_F8
-#define FA_EXP_F16_F8 0
-#endif
 #ifndef FA_POLY_PAIRS_PER8_D64
 #define FA_POLY_PAIRS_PER8_D64 2
 #endif
@@ -848,13 +832,6 @@ template <int D, bool F8>
 __host__ __device__ constexpr int poly_pairs_per8() {
     return F8 ? FA_POLY_PAIRS_PER8_F8 : (D == 64 ? FA_POLY_PAIRS_PER8_D64 : FA_POLY_PAIRS_PER8);
 }
-// The row maximum may be formed alongside the first half's exponentials,
-// taken against the current reference m_used (set after key block 0); the
-// half is redone only when the block's maximum exceeds m_used by more than
-// the rescale threshold (bf16 paths; FP8 keeps the exact running maximum).
-#ifndef FA_SPEC_MAX
-#define FA_SPEC_MAX 0
-#endif
 __device__ __forceinline__ uint64_t f2_const(uint32_t bits) {
     return (static_cast<uint64_t>(bits) << 32) | bits;
 }
@@ -905,11 +882,6 @@ __device__ __forceinline__ void exp_half(const uint32_t (&s)[128], uint64_t sl2x
         uint64_t e;
         if ((gi % 8) < NPOLY) {
             e = exp2_poly2(x);
-        } else if (F8 ? FA_EXP_F16_F8 : FA_EXP_F16) {
-            float x0, x1, y0, y1;
-            f2_unpack(x, x0, x1);
-            ex2_f16x2(x0, x1, y0, y1);
-            e = f2_pack(y0, y1);
         } else {
             float x0, x1;
             f2_unpack(x, x0, x1);
@@ -947,10 +919,7 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
     const float sl2 = p.scale_log2;
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
     uint32_t sc = 0, oc = 0, pw = 0;     // S blocks, O finals, P V completions waited for
-#if FA_TOKEN
-    constexpr bool kTok = tmem_layout<D, F8>() == kSepP;
-    uint32_t tw = 0;                     // turns waited for (phase parity of bar_tok[t])
-#endif
+
     bool ok = true;
     for (int rr = 0; ok; ++rr) {
         const int idx = item_of_round(rr);
@@ -967,18 +936,8 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
         }
         // keys [0, limit) are allowed for this row (causal: up to its own position)
         const int limit = p.causal ? min(row_pos(row, it.qoff, PK ? 0 : p.qmod) + 1, it.klen) : it.klen;
-#if FA_OFFSET_NS > 0
-        // separate S buffers: start tile 1 a fraction of a block behind tile 0, so
-        // that one tile's loads and maxima overlap the other's exponentials
-        if constexpr (tmem_layout<D, F8>() == kSepP) {
-            if (t == 1) __nanosleep(FA_OFFSET_NS);
-        }
-#endif
         float m_used = -INFINITY;    // max the exponentials are taken against (log2 units)
         float l = 0.f;               // running sum of exp2(x - m_used)
-#if FA_TOKEN
-        const int n_common = min(it.n[0], it.n[1]);      // blocks both tiles visit: they take turns
-#endif
         for (int j = 0; j < n; ++j) {
             if (lane == 0 && wq == 0) FA_TRACE_EV(t, sc, 0);
             ok = wait_bar(smem_u32(&ms.bar_s_full[t]), sc & 1, p, ms, kSiteSFull);
@@ -1006,30 +965,14 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
             constexpr int kPoly = poly_pairs_per8<D, F8>();
             // FP8: exact running maximum (threshold 0), so that P <= 1 before the
             // 2^8 shift below; bf16: lazy rescale
-            constexpr float kThr = F8 ? 0.f : kRescaleThreshold;
+            constexpr float kThr = F8 ? kF8Threshold : kRescaleThreshold;
             // FP8: P is computed as 2^8 * exp2(x - m) in (0, 256], so that E4M3
             // holds every entry above 2^-14 of the row maximum as a normal
             // number (relative rounding error <= 2^-4); l carries the same
             // factor, and lse takes it back out
-            constexpr float kPShift = F8 ? 8.f : 0.f;
+            constexpr float kPShift = F8 ? kF8Shift : 0.f;
             uint64_t acc[4] = {0, 0, 0, 0};      // packed row sums (+0.0f pairs)
             uint32_t pk[32];
-            // speculative half 0 against the current reference (every row of
-            // the warp has one after its first key block)
-            const bool spec = FA_SPEC_MAX && !F8 && j > 0 && __all_sync(0xffffffffu, m_used != -INFINITY);
-            if (spec) {
-                // stored at once (over scores already in registers), so that
-                // pk is free while the maximum is formed; not yet signalled
-                exp_half<F8, 0, kPoly>(s, sl2x2, f2_pack(-m_used, -m_used), pk, acc);
-                if (!pv_free) {
-                    ok = wait_bar(smem_u32(&ms.bar_pv_done[t]), pw & 1, p, ms, kSitePvDone);
-                    if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-                    ++pw;
-                    pv_free = true;
-                    tc_fence_after();
-                }
-                tmem_st32(taddr_p, pk);
-            }
             const float mx = row_max128(s);
             const float m_new = fmaxf(m_used, mx * sl2);
             if (lane == 0 && wq == 0) FA_TRACE_EV(t, sc - 1, 3);
@@ -1069,29 +1012,18 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
             }
             const float msub = ((m_used == -INFINITY) ? 0.f : m_used) - kPShift;
             const uint64_t nm2 = f2_pack(-msub, -msub);
-#if FA_TOKEN
-            if (kTok && j < n_common && !(t == 0 && j == 0)) {
-                ok = wait_bar(smem_u32(&ms.bar_tok[t]), tw & 1, p, ms, kSitePFull);
+            exp_half<F8, 0, kPoly>(s, sl2x2, nm2, pk, acc);
+            if (!pv_free) {
+                ok = wait_bar(smem_u32(&ms.bar_pv_done[t]), pw & 1, p, ms, kSitePvDone);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-                ++tw;
+                ++pw;
+                pv_free = true;
+                tc_fence_after();
             }
-#endif
-            if (!spec || any_need) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) acc[i] = 0;
-                exp_half<F8, 0, kPoly>(s, sl2x2, nm2, pk, acc);
-                if (!pv_free) {
-                    ok = wait_bar(smem_u32(&ms.bar_pv_done[t]), pw & 1, p, ms, kSitePvDone);
-                    if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-                    ++pw;
-                    pv_free = true;
-                    tc_fence_after();
-                }
-                if constexpr (F8)
-                    tmem_st16(taddr_p, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
-                else
-                    tmem_st32(taddr_p, pk);
-            }
+            if constexpr (F8)
+                tmem_st16(taddr_p, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
+            else
+                tmem_st32(taddr_p, pk);
             // keys 0-63 of P are ready: the tensor core can start on them
             tmem_wait_st();
             tc_fence_before();
@@ -1113,10 +1045,7 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
             __syncwarp();
             if (lane == 0) FA_TRACE_EV(t, sc - 1, wq == 0 ? 4 : 4 + wq);
             if (lane == 0) mbar_arrive(smem_u32(&ms.bar_p_half[t][1]));
-#if FA_TOKEN
-            if (kTok && j < n_common && !(t == 1 && j == n_common - 1) && lane == 0)
-                mbar_arrive(smem_u32(&ms.bar_tok[1 - t]));            // the other tile's turn
-#endif
+
         }
         if (!ok) break;
         // epilogue: O / l -> bf16 -> HBM, and the logsumexp
@@ -1158,7 +1087,7 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
                 if (valid) {
                     float lg;
                     asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg) : "f"(l));
-                    p.lse_part[prid] = (l > 0.f) ? (m_used + lg - (F8 ? 8.f : 0.f)) * 0.69314718055994531f : -INFINITY;
+                    p.lse_part[prid] = (l > 0.f) ? (m_used + lg - (F8 ? kF8Shift : 0.f)) * 0.69314718055994531f : -INFINITY;
                 }
                 tc_fence_before();
                 continue;
@@ -1188,7 +1117,7 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
         if (valid) {
             float lg;
             asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg) : "f"(l));
-            *lrow = (l > 0.f) ? (m_used + lg - (F8 ? 8.f : 0.f)) * 0.69314718055994531f : -INFINITY;
+            *lrow = (l > 0.f) ? (m_used + lg - (F8 ? kF8Shift : 0.f)) * 0.69314718055994531f : -INFINITY;
         }
         tc_fence_before();
     }
@@ -1222,7 +1151,6 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             mbar_init(smem_u32(&ms.bar_o_final[t]), 1);
             mbar_init(smem_u32(&ms.bar_s_free[t]), 4);     // one arrival per warp
             mbar_init(smem_u32(&ms.bar_pv_done[t]), 1);
-            mbar_init(smem_u32(&ms.bar_tok[t]), 4);        // one arrival per warp of the other tile
         }
         ms.abort_flag = 0;
         ms.bad = 0;

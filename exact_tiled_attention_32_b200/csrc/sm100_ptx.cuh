@@ -61,19 +61,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// true once the phase with the given parity has completed; never suspends
-__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 // --------------------------------------------------------------------- TMA
 // 4-D tiled bulk-tensor load into this CTA's shared memory; completion is
 // signalled on `bar` as transaction bytes.  No multicast.
@@ -538,17 +525,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
-}
-// 2^x of a pair of floats through the half-precision MUFU form: the pair is
-// rounded to f16x2 (round to nearest), ex2.approx.f16x2 gives two f16
-// results, widened back to fp32 (lo in the first output)
-__device__ __forceinline__ void ex2_f16x2(float x0, float x1, float& y0, float& y1) {
-    uint32_t h, r;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(x1), "f"(x0));
-    asm("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(h));
-    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
-        "cvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
-        : "=f"(y0), "=f"(y1) : "r"(r));
 }
 // pack four fp32 into four E4M3 bytes (round to nearest even, finite values
 // beyond 448 saturate); a0 lands in bits 0-7
