@@ -64,7 +64,7 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only past 2
 // E4M3's largest value (448 = 2^8.807): with the reference m_used at most
 // kF8Threshold below the row's true maximum, P <= 2^(kF8Shift + kF8Threshold).
 #ifndef FA_F8_THRESHOLD
-#define FA_F8_THRESHOLD 0.0f
+#define FA_F8_THRESHOLD 3.0f
 #endif
 constexpr float kF8Threshold = FA_F8_THRESHOLD;
 constexpr float kF8Shift = FA_F8_THRESHOLD > 0.f ? 8.75f - FA_F8_THRESHOLD : 8.0f;
@@ -963,13 +963,13 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
                     if (c >= lim) s[c] = __float_as_uint(-INFINITY);
             }
             constexpr int kPoly = poly_pairs_per8<D, F8>();
-            // FP8: exact running maximum (threshold 0), so that P <= 1 before the
-            // 2^8 shift below; bf16: lazy rescale
+            // bf16: lazy rescale (the reference may trail the true maximum by
+            // up to 2^8); FP8: threshold kF8Threshold with P computed as
+            // 2^kF8Shift * exp2(x - m) <= 2^8.75 < 448, so that E4M3 holds every
+            // entry above 2^-(6 + kF8Shift) of the row maximum as a normal number
+            // (relative rounding error <= 2^-4); l carries the same factor, and
+            // lse takes it back out
             constexpr float kThr = F8 ? kF8Threshold : kRescaleThreshold;
-            // FP8: P is computed as 2^8 * exp2(x - m) in (0, 256], so that E4M3
-            // holds every entry above 2^-14 of the row maximum as a normal
-            // number (relative rounding error <= 2^-4); l carries the same
-            // factor, and lse takes it back out
             constexpr float kPShift = F8 ? kF8Shift : 0.f;
             uint64_t acc[4] = {0, 0, 0, 0};      // packed row sums (+0.0f pairs)
             uint32_t pk[32];

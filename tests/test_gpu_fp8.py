@@ -3,14 +3,18 @@ fp64 oracle of attention on the dequantised inputs.
 
 Tolerance (per output element, derived from the arithmetic): the forward's
 1e-2, plus one bf16 rounding of O (2^-7 |O|), plus the E4M3 rounding of P for
-the P V product.  The kernel computes P = 2^8 exp(s - m_run) <= 2^8 with the
-exact running maximum m_run, so every entry with exp(s - m) >= 2^-14 of the
-final row maximum m is a normal E4M3 number (relative error <= 2^-4), and an
-entry below that is off by at most 2^-18 (half the subnormal step, in units of
-the row maximum).  After the division by the row sum l = sum_j exp(s_j - m):
-|dO_c| <= 1e-2 + 2^-7 |O_c| + 2^-4 sum_j p_j |v_jc| + 2^-18 sum_{tiny j} |v_jc| / l.
+the P V product.  The kernel computes P = 2^SHIFT exp2(x - m_ref) against a
+reference m_ref that is never above the row's final maximum m and never more
+than THRESHOLD (log2 units) below the scores it is applied to, with
+SHIFT + THRESHOLD = 8.75, so P <= 2^8.75 < 448 (E4M3's largest value).
+Every entry with exp(s - m) >= 2^-(6 + SHIFT) of the final maximum then has
+P >= 2^-6, a normal E4M3 number (relative error <= 2^-4); an entry below that
+is off by at most half the subnormal step, 2^-10 in P units, i.e. at most
+2^-(10 + SHIFT) in units of the final maximum.  After the division by the
+row sum l = sum_j exp(s_j - m):
+|dO_c| <= 1e-2 + 2^-7 |O_c| + 2^-4 sum_j p_j |v_jc| + 2^-(10+SHIFT) sum_{tiny j} |v_jc| / l.
 The weights p, l and the tiny set come from the exact scores of the
-dequantised inputs.
+dequantised inputs.  The kernel's THRESHOLD is 3 (SHIFT 5.75).
 
 Mean bound (over the compared elements): the worst case above adds every
 weight's rounding error with the same sign; the mean error is checked
@@ -33,6 +37,7 @@ from exact_tiled_attention_32_b200 import synthetic as syn
 pytestmark = pytest.mark.gpu
 
 S = syn.FP8_SCALE
+F8_SHIFT = 5.75          # the kernel's P scaling (log2); tiny: below 2^-(6 + F8_SHIFT) of the row maximum
 
 
 def _dev(codes):
@@ -69,8 +74,8 @@ def _bound(w, rows, o_ref):
         s = w.scale * (K @ qf[rid])
         e = np.exp(s - s.max())
         l = e.sum()
-        tiny = e < 2.0 ** -14
-        tiny_t[n] = 2.0 ** -18 * V[tiny].sum(axis=0) / l
+        tiny = e < 2.0 ** -(6 + F8_SHIFT)
+        tiny_t[n] = 2.0 ** -(10 + F8_SHIFT) * V[tiny].sum(axis=0) / l
         out[n] = 2.0 ** -4 * (e / l) @ V + tiny_t[n]
         rms[n] = 2.0 ** -4 / np.sqrt(3.0) * np.sqrt(((e / l) ** 2) @ (V ** 2))
     worst = 1e-2 + 2.0 ** -7 * np.abs(o_ref) + out
