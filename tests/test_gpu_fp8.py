@@ -183,3 +183,34 @@ def test_c3f8_sampled_rows():
     o, lse = _run(w)
     rows = sample_rows(w, early=4, tile_stride=16, n_random=4, seed=8)
     _check(w, o, lse, rows, "c3f8")
+
+
+def test_c5f8_sampled_rows():
+    """The packed FP8 workload the bench times (c5's 16 sequences in E4M3),
+    sequence by sequence: the first rows, the first and last row of every
+    eighth tile and random rows of every head, against the oracle of that
+    sequence's dense problem under the same bounds."""
+    import torch
+    from exact_tiled_attention_32_b200 import binding as fa
+    w = syn.config("c5f8").draw()
+    cu = torch.from_numpy(w.cu_seqlens).cuda()
+    o, lse = fa.attention_forward_fp8(_dev(w.q), _dev(w.k), _dev(w.v), S, S, S, causal=True, scale=w.scale,
+                                      cu_seqlens=cu)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status() == 0
+    o = o.float().cpu().numpy().astype(np.float64)
+    lse = lse.cpu().numpy().astype(np.float64)
+    rng = np.random.default_rng(9)
+    for s_, L in enumerate(w.lengths):
+        a = int(w.cu_seqlens[s_])
+        ws = syn.Workload("fp8seq", 1, w.Hq, w.Hkv, L, 128, True, 0, fp8=True)
+        ws.q = np.ascontiguousarray(w.q[a:a + L].transpose(1, 0, 2)[None])
+        ws.k = np.ascontiguousarray(w.k[a:a + L].transpose(1, 0, 2)[None])
+        ws.v = np.ascontiguousarray(w.v[a:a + L].transpose(1, 0, 2)[None])
+        od = o[a:a + L].transpose(1, 0, 2).reshape(-1, 128)
+        ld = lse[:, a:a + L].reshape(-1)
+        ts = set(range(4)) | {L - 1} | set(rng.integers(0, L, 3).tolist())
+        for m in range(0, (L + 127) // 128, 8):
+            ts.update((128 * m, min(128 * m + 127, L - 1)))
+        rows = np.array(sorted(h * L + t for h in range(w.Hq) for t in ts))
+        _check(ws, od, ld, rows, f"c5f8 seq {s_} (L={L})")
