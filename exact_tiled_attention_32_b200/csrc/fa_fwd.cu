@@ -122,7 +122,7 @@ static_assert(tmem_o_col<64, false>(1) + 64 <= 512 && tmem_o_col<128, false>(1) 
 // where a wait gave up (reported in status[1])
 enum WaitSite : int {
     kSiteQEmpty = 1, kSiteKvEmpty, kSiteQFull, kSiteKvFull, kSitePFull, kSiteSFull, kSiteOFinal, kSiteSFree,
-    kSitePvDone
+    kSitePvDone, kSiteFeed
 };
 
 struct alignas(64) Params {
@@ -132,6 +132,9 @@ struct alignas(64) Params {
     const int32_t* cu_seqlens;
     const int32_t* cu_seqlens_k;   // packed query chunks: key offsets (NULL: the keys are the queries' tokens)
     int* status;
+    unsigned long long* sched;   // work counter: {launch epoch (bits 32-63), items taken (0-31)}
+    unsigned epoch;              // this launch's epoch (nonzero)
+    int dyn;                     // 1: dynamic schedule (sched, epoch); 0: static snake
     int B, Hq, Hkv, N;         // N: query rows per sequence (dense) or total tokens (packed)
     int Nk;                    // dense: keys per sequence (== N except for a query chunk)
     int q_off;                 // dense: position of query row 0 among the keys (Nk - N for a chunk)
@@ -173,6 +176,8 @@ struct Misc {
     uint64_t bar_p_half[2][2];     // P_t keys 0-63 / 64-127 are in TMEM
     uint64_t bar_s_free[2];        // separate-P layout: the softmax warps have read S_t
     uint64_t bar_pv_done[2];       // separate-P layout: O_t += P_t V_j has completed
+    uint64_t bar_feed_full[4], bar_feed_empty[4];   // the item ring (dynamic schedule)
+    int feed[4];
     uint32_t tmem_base;
     int abort_flag;
     int bad;
@@ -356,6 +361,86 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, const P
     }
 }
 
+// ------------------------------------------------------------ work feed
+// Dynamic schedule (FA_DYN_SCHED, the default).  CTA c starts with item c;
+// after that the producer thread takes the next item of the global order
+// from a counter in global memory each time its CTA's loads of the previous
+// item are all issued, and hands the index to the other roles through a ring
+// of kFeedDepth slots in shared memory.  So every CTA takes the next item when
+// it is about to be ready for one (a longest-first order then balances the
+// CTAs), and the items in flight on the GPU at any time are consecutive in
+// the order, i.e. come from the few (batch, head) units whose K/V share L2.
+// The counter word carries the launch's epoch in its upper half.  A CTA that
+// reads an earlier launch's epoch there swaps in {epoch, 0} with a
+// compare-and-swap against the value it read; the word changes only through
+// such a swap until it holds this launch's epoch (counting adds are made only
+// after that has been seen), so exactly one swap succeeds and every failed one
+// means the word has moved on.  The counter needs no reset between launches,
+// even after an aborted one.  Launches with few items per CTA (p.dyn = 0), and
+// every launch of a build with FA_DYN_SCHED=0, follow the static snake of
+// item_of_round instead.
+#ifndef FA_DYN_SCHED
+#define FA_DYN_SCHED 1
+#endif
+constexpr int kFeedDepth = 4;
+// the next dynamic item (0, 1, ... in this launch); 0x3fffffff (no item,
+// error recorded) if the word keeps changing under the swap, which only a
+// launch of long ago still running on the same counter could cause
+__device__ __forceinline__ int sched_take(const Params& p, Misc& ms) {
+    const unsigned long long tag = static_cast<unsigned long long>(p.epoch) << 32;
+    unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(p.sched);
+    for (int tries = 0; static_cast<unsigned>(cur >> 32) != p.epoch; ++tries) {
+        if (tries == 64) {
+            *reinterpret_cast<volatile int*>(&ms.abort_flag) = 1;
+            if (atomicCAS(p.status, 0, FA_ERR_DEVICE_TIMEOUT) == 0) {
+                p.status[1] = kSiteFeed;
+                p.status[2] = blockIdx.x;
+            }
+            return 0x3fffffff;
+        }
+        const unsigned long long seen = atomicCAS(p.sched, cur, tag);
+        // success: the word is now {epoch, 0}; failure: another CTA's swap
+        // (the only other change an old-epoch word can see) moved it on
+        cur = seen == cur ? tag : seen;
+    }
+    return static_cast<int>(atomicAdd(p.sched, 1ull) & 0xffffffffull);
+}
+// item of round r for this CTA's producer (all items past the first are dynamic)
+__device__ __forceinline__ int producer_item(const Params& p, Misc& ms, int r, int total) {
+    if (!FA_DYN_SCHED || !p.dyn) return item_of_round(r);
+    if (r == 0) return blockIdx.x;
+    return min(static_cast<int>(gridDim.x) + sched_take(p, ms), total);
+}
+// a consumer warp takes its r-th item (all lanes; one arrival per warp)
+__device__ __forceinline__ bool feed_take(const Params& p, Misc& ms, int r, int& idx) {
+    if (!FA_DYN_SCHED || !p.dyn) {
+        idx = item_of_round(r);
+        return true;
+    }
+    if (r == 0) {
+        idx = blockIdx.x;
+        return true;
+    }
+    const uint32_t u = static_cast<uint32_t>(r - 1);     // rounds 1, 2, ... pass through the ring
+    const uint32_t s = u % kFeedDepth;
+    if (!wait_all(smem_u32(&ms.bar_feed_full[s]), (u / kFeedDepth) & 1u, p, ms, kSiteFeed)) return false;
+    idx = *reinterpret_cast<volatile int*>(&ms.feed[s]);
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&ms.bar_feed_empty[s]));
+    return true;
+}
+// the producer thread publishes its r-th item (r >= 1; total: no more items)
+__device__ __forceinline__ bool feed_give(const Params& p, Misc& ms, int r, int idx) {
+    if (!FA_DYN_SCHED || !p.dyn) return true;
+    if (r == 0) return true;
+    const uint32_t u = static_cast<uint32_t>(r - 1);
+    const uint32_t s = u % kFeedDepth;
+    if (!wait_bar(smem_u32(&ms.bar_feed_empty[s]), ((u / kFeedDepth) & 1u) ^ 1u, p, ms, kSiteFeed)) return false;
+    *reinterpret_cast<volatile int*>(&ms.feed[s]) = idx;
+    mbar_arrive(smem_u32(&ms.bar_feed_full[s]));
+    return true;
+}
+
 // ---------------------------------------------------------------- producer
 template <int D, bool PK, bool F8 = false>
 __device__ void load_role(const Params& p, Misc& ms, const SeqTables& tab, uint32_t smem_q, uint32_t smem_kv,
@@ -367,7 +452,11 @@ __device__ void load_role(const Params& p, Misc& ms, const SeqTables& tab, uint3
     uint32_t st = 0, ph = 0;      // ring position of tile kv_it: stage and phase parity
     bool ok = true;
     for (int r = 0; ok; ++r) {
-        const int idx = item_of_round(r);
+        // the next item, taken only now that this CTA's loads of its previous
+        // item are all issued (taking it earlier would reserve it for a CTA
+        // that may still be busy for long)
+        const int idx = producer_item(p, ms, r, total);
+        if (!(ok = feed_give(p, ms, r, idx))) break;
         if (idx >= total) break;
         const Item it = decode_item<PK>(idx, p, ms, tab);
         if (max(it.n[0], it.n[1]) == 0) continue;      // a split with no key block
@@ -470,7 +559,8 @@ __device__ void mma_role(const Params& p, Misc& ms, const SeqTables& tab, uint32
     uint32_t pc[2] = {0, 0};
     bool ok = true;
     for (int r = 0; ok; ++r) {
-        const int idx = item_of_round(r);
+        int idx;
+        if (!(ok = feed_take(p, ms, r, idx))) break;
         if (idx >= total) break;
         const Item it = decode_item<PK>(idx, p, ms, tab);
         if (max(it.n[0], it.n[1]) == 0) continue;      // a split with no key block
@@ -568,7 +658,8 @@ __device__ void mma_role_sep_p(const Params& p, Misc& ms, const SeqTables& tab, 
     uint32_t sn[2] = {0, 0};      // S issued into buffer 0 / 1: every S but the first waits for bar_s_free
     bool ok = true;
     for (int r = 0; ok; ++r) {
-        const int idx = item_of_round(r);
+        int idx;
+        if (!(ok = feed_take(p, ms, r, idx))) break;
         if (idx >= total) break;
         const Item it = decode_item<PK>(idx, p, ms, tab);
         if (max(it.n[0], it.n[1]) == 0) continue;      // a split with no key block
@@ -686,7 +777,8 @@ __device__ void mma_role_split(const Params& p, Misc& ms, const SeqTables& tab, 
     uint32_t sn[2] = {0, 0};      // S issued into buffer 0 / 1: every S but the first waits for bar_s_free
     bool ok = true;
     for (int r = 0; ok; ++r) {
-        const int idx = item_of_round(r);
+        int idx;
+        if (!(ok = feed_take(p, ms, r, idx))) break;
         if (idx >= total) break;
         const Item it = decode_item<PK>(idx, p, ms, tab);
         if (max(it.n[0], it.n[1]) == 0) continue;      // a split with no key block
@@ -922,7 +1014,16 @@ __device__ void softmax_role(const Params& p, Misc& ms, const SeqTables& tab, ui
 
     bool ok = true;
     for (int rr = 0; ok; ++rr) {
-        const int idx = item_of_round(rr);
+        // (feed_take's cases spelled out: this form keeps the loop free of spills)
+        int idx = item_of_round(rr);
+        if (FA_DYN_SCHED && p.dyn && rr > 0) {
+            if (!feed_take(p, ms, rr, idx)) {
+                ok = false;
+                break;
+            }
+        } else if (FA_DYN_SCHED && p.dyn) {
+            idx = blockIdx.x;
+        }
         if (idx >= total) break;
         const Item it = decode_item<PK>(idx, p, ms, tab);
         const int n = t ? it.n[1] : it.n[0];
@@ -1140,6 +1241,11 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         mbar_init(smem_u32(&ms.bar_q_full), 1);
         mbar_init(smem_u32(&ms.bar_q_empty), 1);
         mbar_init(smem_u32(&ms.bar_drain), split_issue<D, F8>() ? 2 : 1);
+        for (int s = 0; s < kFeedDepth; ++s) {
+            mbar_init(smem_u32(&ms.bar_feed_full[s]), 1);
+            // consumers: the softmax warps and the MMA issuer warp(s)
+            mbar_init(smem_u32(&ms.bar_feed_empty[s]), kNumSoftmaxWarps + (split_issue<D, F8>() ? 2 : 1));
+        }
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(smem_u32(&ms.bar_kv_full[s]), 1);
             mbar_init(smem_u32(&ms.bar_kv_empty[s]), 1);
@@ -1358,6 +1464,8 @@ int init_device(int dev, DeviceState** out) {
             bool good = g_encode != nullptr;
             good = good && cudaMalloc(&ds.status, 4 * sizeof(int)) == cudaSuccess;
             good = good && cudaMemset(ds.status, 0, 4 * sizeof(int)) == cudaSuccess;
+            good = good && cudaMalloc(&ds.sched, kSchedSlots * sizeof(unsigned long long)) == cudaSuccess;
+            good = good && cudaMemset(ds.sched, 0, kSchedSlots * sizeof(unsigned long long)) == cudaSuccess;
             good = good && cudaFuncSetAttribute(fa_fwd_kernel<64, false>,
                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 Cfg<64, false>::kSmemBytes) == cudaSuccess;
@@ -1415,8 +1523,15 @@ static bool make_maps(Params& P, const void* q, const void* k, const void* v, in
            encode_map(&P.tm_v, v, dk, sk, box, fp8);
 }
 
+// The dynamic schedule runs the items of groups of (batch, head) units whose
+// K/V fit in this many MiB of L2 (126 MB) one group after the other.
 #ifndef FA_L2_GROUP_MIB
-#define FA_L2_GROUP_MIB 1000000ll
+#define FA_L2_GROUP_MIB 32ll
+#endif
+// Launches with fewer items than this many per SM keep the static snake
+// (a CTA's one or two items: nothing to balance, and no counter to wait on).
+#ifndef FA_DYN_MIN_ITEMS_PER_SM
+#define FA_DYN_MIN_ITEMS_PER_SM 4
 #endif
 
 #ifdef FA_TRACE
@@ -1425,6 +1540,18 @@ static unsigned long long* g_trace = nullptr;
 
 static bool aligned(const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) == 0; }
 
+// the work counter and epoch of this device's next forward launch: launch n
+// takes counter n % kSchedSlots with epoch n / kSchedSlots + 1
+struct Sched {
+    unsigned long long* word;
+    unsigned epoch;
+};
+static Sched next_sched(std::atomic<unsigned>& seq, unsigned long long* words, unsigned slots) {
+    const unsigned n = seq.fetch_add(1, std::memory_order_relaxed);
+    return Sched{words + n % slots, n / slots + 1u};
+}
+static Sched next_sched(DeviceState* ds) { return next_sched(ds->sched_seq, ds->sched, kSchedSlots); }
+
 
 // Fills the launch parameters and launches the kernel variant for (d, packed)
 // on `stream`.  Nk / q_off describe a dense query chunk (Nk keys per sequence,
@@ -1432,7 +1559,7 @@ static bool aligned(const void* ptr, uintptr_t a) { return (reinterpret_cast<uin
 // qmod, splits, o_part, lse_part: see Params (a plain forward has 0, 1, NULL, NULL).
 static int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                       int N, int Nk, int q_off, int d, float scale, int causal, const int32_t* cu_seqlens,
-                      cudaStream_t s, int* status, int num_sms, int qmod = 0, int splits = 1,
+                      cudaStream_t s, int* status, int num_sms, Sched sched, int qmod = 0, int splits = 1,
                       float* o_part = nullptr, float* lse_part = nullptr, bool fp8 = false,
                       float qk_scale = 1.f, float v_scale = 1.f, const int32_t* cu_seqlens_k = nullptr) {
     const bool packed = cu_seqlens != nullptr;
@@ -1451,12 +1578,19 @@ static int launch_fwd(const void* q, const void* k, const void* v, void* o, floa
     P.Nk = Nk;
     P.q_off = q_off;
     P.group = Hq / Hkv;
+    // work items: dense, known here; packed, counted on the device (at least
+    // one per sequence and head per 256 tokens)
+    const long long items = packed ? std::max<long long>(1, (long long)N / kRowsPerItem) * Hq
+                                   : (long long)((N + kRowsPerItem - 1) / kRowsPerItem) * B * Hq * splits;
+    P.dyn = (FA_DYN_SCHED && items >= (long long)FA_DYN_MIN_ITEMS_PER_SM * num_sms) ? 1 : 0;
+    P.sched = sched.word;
+    P.epoch = sched.epoch;
     {
-        // K/V of one group of units should stay resident in L2 (126 MB) while
-        // the group's items run
+        // dynamic schedule: K/V of one group of units stay resident in L2
+        // while the group's items run; static: one group
         const long long kv_bytes = 4ll * Nk * d;                   // K and V of one kv head
         long long g_kv = std::max(1ll, (FA_L2_GROUP_MIB << 20) / std::max(1ll, kv_bytes));
-        long long G = std::min<long long>(g_kv * P.group, (long long)B * Hq);
+        long long G = P.dyn ? std::min<long long>(g_kv * P.group, (long long)B * Hq) : (long long)B * Hq;
         P.group_units = (int)std::max(1ll, G);
     }
     P.causal = causal ? 1 : 0;
@@ -1471,13 +1605,9 @@ static int launch_fwd(const void* q, const void* k, const void* v, void* o, floa
 #ifdef FA_TRACE
     P.trace = g_trace;
 #endif
-    long long items;
-    if (!packed) {
-        items = (long long)((N + kRowsPerItem - 1) / kRowsPerItem) * B * Hq * splits;
-    } else {
-        items = (long long)num_sms;    // exact count is known only on the device
-    }
-    const int grid = (int)std::min<long long>(items, num_sms);
+    // dense: one CTA per item up to one per SM; packed: one per SM (the CTAs
+    // with no item of the device's count return at once)
+    const int grid = packed ? num_sms : (int)std::min<long long>(items, num_sms);
     if (fp8 && packed)
         fa_fwd_kernel<128, true, true><<<grid, kThreads, Cfg<128, true, true>::kSmemBytes, s>>>(P);
     else if (fp8)
@@ -1526,7 +1656,7 @@ extern "C" int fa_fwd(const void* q, const void* k, const void* v, void* o, floa
     if (st != FA_OK) return st;
 
     return launch_fwd(q, k, v, o, lse, B, Hq, Hkv, N, N, 0, d, scale, causal, cu_seqlens,
-                      static_cast<cudaStream_t>(stream), ds->status, ds->num_sms);
+                      static_cast<cudaStream_t>(stream), ds->status, ds->num_sms, next_sched(ds));
 }
 
 extern "C" int fa_fwd_kvcache(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
@@ -1548,7 +1678,7 @@ extern "C" int fa_fwd_kvcache(const void* q, const void* k, const void* v, void*
     if (st != FA_OK) return st;
     // the chunk's rows are the last Nq positions of the key sequence
     return launch_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, causal ? Nk - Nq : 0, d, scale, causal, nullptr,
-                      static_cast<cudaStream_t>(stream), ds->status, ds->num_sms);
+                      static_cast<cudaStream_t>(stream), ds->status, ds->num_sms, next_sched(ds));
 }
 
 extern "C" int fa_fwd_kvcache_varlen(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
@@ -1571,8 +1701,8 @@ extern "C" int fa_fwd_kvcache_varlen(const void* q, const void* k, const void* v
     const int st = init_device(dev, &ds);
     if (st != FA_OK) return st;
     return launch_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, 0, d, scale, causal, cu_seqlens_q,
-                      static_cast<cudaStream_t>(stream), ds->status, ds->num_sms, 0, 1, nullptr, nullptr, false, 1.f,
-                      1.f, cu_seqlens_k);
+                      static_cast<cudaStream_t>(stream), ds->status, ds->num_sms, next_sched(ds), 0, 1, nullptr,
+                      nullptr, false, 1.f, 1.f, cu_seqlens_k);
 }
 
 // ------------------------------------------------------------ split keys
@@ -1674,12 +1804,12 @@ extern "C" int fa_fwd_splitkv(const void* q, const void* k, const void* v, void*
     const int q_off = causal ? Nk - Nq : 0;
     if (num_splits == 1)
         return launch_fwd(q, k, v, o, lse, B, sh.Hq, sh.Hkv, sh.N, Nk, q_off, d, scale, causal, nullptr, s,
-                          ds->status, ds->num_sms, sh.qmod);
+                          ds->status, ds->num_sms, next_sched(ds), sh.qmod);
     const long long rows = (long long)B * Hq * Nq;
     float* o_part = static_cast<float*>(workspace);
     float* lse_part = o_part + static_cast<size_t>(num_splits) * rows * d;
     const int rc = launch_fwd(q, k, v, o, lse, B, sh.Hq, sh.Hkv, sh.N, Nk, q_off, d, scale, causal, nullptr, s,
-                              ds->status, ds->num_sms, sh.qmod, num_splits, o_part, lse_part);
+                              ds->status, ds->num_sms, next_sched(ds), sh.qmod, num_splits, o_part, lse_part);
     if (rc != FA_OK) return rc;
     const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
     if (d == 64)
@@ -1711,8 +1841,8 @@ static int fwd_fp8(const void* q, const void* k, const void* v, void* o, float* 
     const int st = init_device(dev, &ds);
     if (st != FA_OK) return st;
     return launch_fwd(q, k, v, o, lse, B, Hq, Hkv, N, N, 0, d, scale, causal, cu_seqlens,
-                      static_cast<cudaStream_t>(stream), ds->status, ds->num_sms, 0, 1, nullptr, nullptr, true,
-                      q_scale * k_scale, v_scale);
+                      static_cast<cudaStream_t>(stream), ds->status, ds->num_sms, next_sched(ds), 0, 1, nullptr,
+                      nullptr, true, q_scale * k_scale, v_scale);
 }
 
 extern "C" int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
@@ -1745,7 +1875,8 @@ extern "C" int fa_fwd_partial(const void* q, const void* k, const void* v, float
     const int st = init_device(dev, &ds);
     if (st != FA_OK) return st;
     return launch_fwd(q, k, v, nullptr, nullptr, B, Hq, Hkv, Nq, Nk, causal ? Nk - Nq : 0, d, scale, causal, nullptr,
-                      static_cast<cudaStream_t>(stream), ds->status, ds->num_sms, 0, 1, o_part, lse_part);
+                      static_cast<cudaStream_t>(stream), ds->status, ds->num_sms, next_sched(ds), 0, 1, o_part,
+                      lse_part);
 }
 
 extern "C" int fa_merge_partials(const float* o_parts, const float* lse_parts, int nparts, long long rows, int d,
@@ -1826,8 +1957,10 @@ extern "C" const char* fa_status_string(int status) {
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = 256;       // the array's size: the stated maximum
-constexpr size_t kStatusBytes = 4 * sizeof(int);   // what the kernel needs (status words)
-static_assert(kStatusBytes <= kNoAllocScratchBytes, "no-alloc scratch too small");
+constexpr size_t kStatusBytes = 4 * sizeof(int);   // the status words, at the start of the array
+constexpr int kNoAllocSchedSlots = 16;             // work counters after them (64-bit words)
+static_assert(kStatusBytes + kNoAllocSchedSlots * sizeof(unsigned long long) <= kNoAllocScratchBytes,
+              "no-alloc scratch too small");
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
@@ -1836,6 +1969,7 @@ struct NoAllocState {
     int status_code = FA_OK;
     int num_sms = 0;
     int* scratch = nullptr;    // device address of g_noalloc_scratch on this device
+    std::atomic<unsigned> sched_seq{0};
 };
 NoAllocState g_noalloc[fa_sm100::kMaxDevices];
 std::mutex g_noalloc_mu;
@@ -1918,8 +2052,10 @@ extern "C" int fa_fwd_noalloc(const void* q, const void* k, const void* v, void*
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // the status words keep the previous call's contents: start this call at zero
     if (cudaMemsetAsync(st->scratch, 0, kStatusBytes, s) != cudaSuccess) return FA_ERR_LAUNCH;
+    const Sched sched = next_sched(st->sched_seq, reinterpret_cast<unsigned long long*>(st->scratch + 4),
+                                   kNoAllocSchedSlots);
     return launch_fwd(q, k, v, o, lse, B, Hq, Hkv, N, N, 0, d, scale, causal, cu_seqlens, s, st->scratch,
-                      st->num_sms);
+                      st->num_sms, sched);
 }
 
 extern "C" int fa_get_noalloc_status(void* stream) {

@@ -2,6 +2,7 @@
 // libfa.so (not part of the C ABI).
 #pragma once
 #include <cuda.h>
+#include <atomic>
 #include <cstdint>
 
 namespace fa_sm100 {
@@ -12,7 +13,14 @@ struct DeviceState {
     int status_code = FA_OK;
     int num_sms = 0;
     int* status = nullptr;        // device: [0] code, [1] wait site, [2] block
+    unsigned long long* sched = nullptr;   // device: kSchedSlots work counters {epoch, items taken}
+    std::atomic<unsigned> sched_seq{0};   // launches so far (picks the counter)
 };
+
+// Work counters per device: consecutive forward launches take consecutive
+// counters, so launches running at the same time on different streams do not
+// share one; a counter's epoch tells its launches apart.
+constexpr int kSchedSlots = 64;
 
 constexpr int kMaxDevices = 64;
 

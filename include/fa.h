@@ -69,7 +69,12 @@ typedef enum {
  * may be NULL.
  *
  * Ownership: the caller owns every buffer.  The library allocates only a
- * small per-device status word, once, on the first call on that device.
+ * small per-device status word and a ring of 64 work counters (8 bytes each),
+ * once, on the first call on that device.  A launch with at least 4 work
+ * items (pairs of 128-row query tiles) per SM hands the items to its CTAs
+ * through one of those counters; consecutive calls take consecutive counters,
+ * each tagged with the call's number, so calls in flight together on
+ * different streams do not share one and no counter needs resetting.
  *
  * Errors: argument errors are found on the host before any launch and return
  * the codes above.  Errors found on the device (a pipeline wait that ran past
@@ -340,10 +345,11 @@ const char* fa_status_string(int status);
  * This entry point takes the same arguments, has the same layouts, limits and
  * host-side error codes as fa_fwd, and computes the same result with the same
  * kernel.  It calls no cudaMalloc, cudaFree or other allocating routine: its
- * only scratch, the status words (16 bytes whatever the problem size), lives
- * in a fixed 256-byte array compiled into the library, which every GPU that
- * loads the library holds until the process exits.  Since the need does not
- * grow with B, N, Hq or d, no problem is too large for the array.
+ * only scratch, the status words (16 bytes) and a ring of 16 work counters
+ * (128 bytes) whatever the problem size, lives in a fixed 256-byte array
+ * compiled into the library, which every GPU that loads the library holds
+ * until the process exits.  Since the need does not grow with B, N, Hq or d,
+ * no problem is too large for the array.
  *
  * The first call on each device sets that device up (device properties, the
  * kernels' shared-memory limits and the array's device address); make that
@@ -352,7 +358,8 @@ const char* fa_status_string(int status);
  * All calls share the array, which keeps the last call's contents; each call
  * clears the status words on its stream before its kernel starts.  Calls that
  * overlap on the GPU (different streams, or several host threads) race on the
- * status words.  Device-side errors of this entry point (FA_ERR_DEVICE_TIMEOUT,
+ * status words (the work counters they take are distinct unless 16 or more
+ * calls are in flight at once).  Device-side errors of this entry point (FA_ERR_DEVICE_TIMEOUT,
  * FA_ERR_SEQLENS) are written to that array only: read them with
  * fa_get_noalloc_status, not fa_get_device_status (which reports fa_fwd's
  * word).

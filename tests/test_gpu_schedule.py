@@ -1,0 +1,101 @@
+"""The forward's dynamic work schedule.
+
+Every CTA starts with its own item and then takes the next item of a global
+order from a per-launch counter; consecutive launches take consecutive
+counters out of a small ring, each tagged with the launch's epoch, so a
+counter is reused (with a new epoch) every ring-length launches and never
+reset.  Which CTA computes which item changes from launch to launch, but each
+item is computed whole by one CTA, so the output must be bitwise the same on
+every launch: checked here over more launches than the ring holds, for
+shapes with far more items than CTAs (causal, uneven item sizes), with fewer
+items than CTAs, packed batches (item count known only on the device), the
+no-allocation entry point (its own, smaller ring) and two streams at once.
+One launch per shape is also checked against the oracle.
+"""
+import pytest
+
+import oracle
+from exact_tiled_attention_32_b200 import synthetic as syn
+from fa_util import assert_parity, gather, to_device
+
+pytestmark = pytest.mark.gpu
+
+RING = 64            # work counters per device in the library (fa_fwd and the entry points built on it)
+NOALLOC_RING = 16    # counters of fa_fwd_noalloc
+
+
+def _shape(name):
+    if name == "many-causal":
+        return syn.Workload(name, 2, 16, 4, 4096, 64, True, 1401).draw()
+    if name == "few-items":
+        return syn.Workload(name, 1, 2, 2, 700, 128, False, 1402).draw()
+    return syn.packed_from_lengths(name, [1500, 1, 300, 2049, 77, 640], 8, 128, True, 1403, Hkv=2).draw()
+
+
+def _launch(fa, entry, w, q, k, v, cu, stream):
+    import torch
+    o = torch.empty_like(q)
+    lse = torch.empty((w.Hq, w.N) if w.packed else (w.B, w.Hq, w.N), dtype=torch.float32, device=q.device)
+    rc = entry(q, k, v, o, lse, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal, cu, stream)
+    assert rc == fa.FA_OK
+    return o, lse
+
+
+@pytest.mark.parametrize("name", ["many-causal", "few-items", "packed"])
+def test_repeated_launches_are_bitwise_identical(name):
+    import torch
+    from exact_tiled_attention_32_b200 import binding as fa
+    w = _shape(name)
+    q, k, v = to_device(w.q), to_device(w.k), to_device(w.v)
+    cu = None if w.cu_seqlens is None else torch.from_numpy(w.cu_seqlens).cuda()
+    stream = torch.cuda.current_stream()
+    o0, l0 = _launch(fa, fa.fa_fwd, w, q, k, v, cu, stream)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status(stream) == fa.FA_OK
+    og, lg = gather(w, o0, l0)
+    oo, lo = oracle.attention(w.q, w.k, w.v, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal, w.cu_seqlens)
+    assert_parity(og, lg, oo, lo, f"{name} against the oracle")
+    mismatches = 0
+    for i in range(RING + 9):               # every counter reused at least once, with a new epoch
+        o, lse = _launch(fa, fa.fa_fwd, w, q, k, v, cu, stream)
+        mismatches += int(not (torch.equal(o, o0) and torch.equal(lse, l0)))
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status(stream) == fa.FA_OK
+    assert mismatches == 0
+
+
+def test_noalloc_ring_reuse_is_bitwise_identical():
+    import torch
+    from exact_tiled_attention_32_b200 import binding as fa
+    w = _shape("many-causal")
+    q, k, v = to_device(w.q), to_device(w.k), to_device(w.v)
+    stream = torch.cuda.current_stream()
+    o0, l0 = _launch(fa, fa.fa_fwd, w, q, k, v, None, stream)
+    for i in range(NOALLOC_RING + 5):
+        o, lse = _launch(fa, fa.fa_fwd_noalloc, w, q, k, v, None, stream)
+        assert fa.fa_get_noalloc_status(stream) == fa.FA_OK
+        assert torch.equal(o, o0) and torch.equal(lse, l0), i
+
+
+def test_two_streams_at_once():
+    """Launches in flight together on two streams take different counters."""
+    import torch
+    from exact_tiled_attention_32_b200 import binding as fa
+    wa, wb = _shape("many-causal"), _shape("packed")
+    qa, ka, va = to_device(wa.q), to_device(wa.k), to_device(wa.v)
+    qb, kb, vb = to_device(wb.q), to_device(wb.k), to_device(wb.v)
+    cub = torch.from_numpy(wb.cu_seqlens).cuda()
+    main = torch.cuda.current_stream()
+    ra = _launch(fa, fa.fa_fwd, wa, qa, ka, va, None, main)
+    rb = _launch(fa, fa.fa_fwd, wb, qb, kb, vb, cub, main)
+    torch.cuda.synchronize()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    outs = []
+    for i in range(12):
+        outs.append(_launch(fa, fa.fa_fwd, wa, qa, ka, va, None, s1))
+        outs.append(_launch(fa, fa.fa_fwd, wb, qb, kb, vb, cub, s2))
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status() == fa.FA_OK
+    for i, (o, lse) in enumerate(outs):
+        ref = ra if i % 2 == 0 else rb
+        assert torch.equal(o, ref[0]) and torch.equal(lse, ref[1]), i
