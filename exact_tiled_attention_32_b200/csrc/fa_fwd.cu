@@ -145,6 +145,8 @@ struct alignas(64) Params {
     float* lse_part;           // dense, when set: logsumexp of each split, [splits][B*Hq*N]
     int group;                 // Hq / Hkv
     int group_units;           // dense: (batch, head) units scheduled together
+    long long l2_group_bytes;  // packed, dynamic schedule: K/V bytes of a head block
+    int pk_grouped;            // packed: sequence by sequence in head blocks (else by pair level)
     int causal, packed;
     float scale_log2;          // scale * log2(e) (FP8: times the Q and K scales)
     float o_scale;             // FP8: the V scale, applied to O in the epilogue
@@ -192,6 +194,11 @@ struct SeqTables {
     int order[kMaxSeqs];       // sequences by pair count, descending
     int pcnt[kMaxPairs];       // number of sequences with more than p pairs
     int pstart[kMaxPairs];     // first item index at pair level p
+    // the dynamic schedule's order: sequence order[k]'s items start at item
+    // sstart[k]; its heads run in blocks of gh[k] (K/V of a block fit the
+    // L2 budget), each block's items heaviest pair first
+    int sstart[kMaxSeqs];
+    int gh[kMaxSeqs];
 };
 
 template <int D, bool PK, bool F8 = false>
@@ -279,6 +286,27 @@ __device__ __forceinline__ Item decode_item(int idx, const Params& p, const Misc
         it.klen = p.Nk;
         it.qoff = p.q_off;
         it.tok0 = 0;
+    } else if (p.pk_grouped) {
+        int lo = 0, hi = p.B - 1;          // last sorted sequence whose start <= idx
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (tab.sstart[mid] <= idx) lo = mid; else hi = mid - 1;
+        }
+        it.seq = tab.order[lo];
+        const int pk = (tab.seq_off[it.seq + 1] - tab.seq_off[it.seq] + kRowsPerItem - 1) / kRowsPerItem;
+        const int gh = tab.gh[lo];
+        const int r = idx - tab.sstart[lo];
+        const int hb = min(r / (pk * gh), (p.Hq - 1) / gh);
+        const int r2 = r - hb * pk * gh;
+        const int bsz = min(gh, p.Hq - hb * gh);
+        const int lvl = r2 / bsz;
+        it.h = hb * gh + (r2 - lvl * bsz);
+        pair = pk - 1 - lvl;
+        it.tok0 = tab.seq_off[it.seq];
+        it.len = tab.seq_off[it.seq + 1] - it.tok0;
+        it.klen = tab.kseq_off[it.seq + 1] - tab.kseq_off[it.seq];
+        it.qoff = p.causal ? it.klen - it.len : 0;     // a chunk's rows are the last positions
+        it.split = 0;
     } else {
         int lo = 0, hi = ms.pmax - 1;      // smallest level whose start <= idx
         while (lo < hi) {
@@ -1320,6 +1348,15 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             }
             ms.pmax = pmax;
             ms.total_items = acc;
+            int acc2 = 0;
+            for (int k = 0; k < p.B; ++k) {
+                const int sq = tab.order[k];
+                const long long kv = 2ll * C::kElem * D * max(1, tab.kseq_off[sq + 1] - tab.kseq_off[sq]);
+                const long long g = max(1ll, p.l2_group_bytes / kv) * p.group;   // whole GQA groups
+                tab.gh[k] = static_cast<int>(min(g, static_cast<long long>(p.Hq)));
+                tab.sstart[k] = acc2;
+                acc2 += pairs_of(sq) * p.Hq;
+            }
         }
     }
 
@@ -1592,6 +1629,12 @@ static int launch_fwd(const void* q, const void* k, const void* v, void* o, floa
         long long g_kv = std::max(1ll, (FA_L2_GROUP_MIB << 20) / std::max(1ll, kv_bytes));
         long long G = P.dyn ? std::min<long long>(g_kv * P.group, (long long)B * Hq) : (long long)B * Hq;
         P.group_units = (int)std::max(1ll, G);
+        P.l2_group_bytes = FA_L2_GROUP_MIB << 20;
+        // packed batches in the dynamic schedule: sequence by sequence (longest
+        // first) in blocks of heads whose K/V fit the budget.  Not for FP8,
+        // whose half-size K/V already hit L2 more often and whose packed
+        // batch measured faster in the pair-level order
+        P.pk_grouped = (packed && P.dyn && !fp8) ? 1 : 0;
     }
     P.causal = causal ? 1 : 0;
     P.packed = packed ? 1 : 0;
