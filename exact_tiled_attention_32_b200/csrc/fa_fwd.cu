@@ -204,10 +204,13 @@ struct SeqTables {
 template <int D, bool PK, bool F8 = false>
 struct Cfg {
     static_assert(D == 64 || D == 128, "head dim");
-    static_assert(!F8 || D == 128, "FP8: d = 128");
     static constexpr int kElem = F8 ? 1 : 2;                // bytes per element
-    static constexpr int kTileBytes = kBlockM * D * kElem;  // one 128 x D tile
-    static constexpr int kBoxes = D * kElem / 128;          // 128-byte-wide TMA boxes per tile row
+    // bytes per tile row in shared memory: FP8 rows are always 128 bytes (at
+    // d = 64 the TMA box's columns past d read as zeros, so the 128-byte
+    // swizzled layout and the K = 128 score MMAs of d = 128 serve unchanged)
+    static constexpr int kRowBytes = F8 ? 128 : D * kElem;
+    static constexpr int kTileBytes = kBlockM * kRowBytes;  // one 128-row tile
+    static constexpr int kBoxes = kRowBytes / 128;          // 128-byte-wide TMA boxes per tile row
     static constexpr int kBoxCols = 128 / kElem;            // elements per box row
     // K/V ring depth: what fits next to the two Q tiles (and the packed tables)
     static constexpr int kStages = F8 ? 10 : ((D == 128) ? (PK ? 4 : 5) : 10);
@@ -1521,6 +1524,12 @@ int init_device(int dev, DeviceState** out) {
             good = good && cudaFuncSetAttribute(fa_fwd_kernel<128, true, true>,
                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 Cfg<128, true, true>::kSmemBytes) == cudaSuccess;
+            good = good && cudaFuncSetAttribute(fa_fwd_kernel<64, false, true>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                Cfg<64, false, true>::kSmemBytes) == cudaSuccess;
+            good = good && cudaFuncSetAttribute(fa_fwd_kernel<64, true, true>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                Cfg<64, true, true>::kSmemBytes) == cudaSuccess;
             ds.status_code = good ? FA_OK : FA_ERR_LAUNCH;
         }
     }
@@ -1651,7 +1660,11 @@ static int launch_fwd(const void* q, const void* k, const void* v, void* o, floa
     // dense: one CTA per item up to one per SM; packed: one per SM (the CTAs
     // with no item of the device's count return at once)
     const int grid = packed ? num_sms : (int)std::min<long long>(items, num_sms);
-    if (fp8 && packed)
+    if (fp8 && d == 64 && packed)
+        fa_fwd_kernel<64, true, true><<<grid, kThreads, Cfg<64, true, true>::kSmemBytes, s>>>(P);
+    else if (fp8 && d == 64)
+        fa_fwd_kernel<64, false, true><<<grid, kThreads, Cfg<64, false, true>::kSmemBytes, s>>>(P);
+    else if (fp8 && packed)
         fa_fwd_kernel<128, true, true><<<grid, kThreads, Cfg<128, true, true>::kSmemBytes, s>>>(P);
     else if (fp8)
         fa_fwd_kernel<128, false, true><<<grid, kThreads, Cfg<128, false, true>::kSmemBytes, s>>>(P);
@@ -1867,7 +1880,7 @@ static int fwd_fp8(const void* q, const void* k, const void* v, void* o, float* 
                    const int32_t* cu_seqlens, void* stream) {
     const bool packed = cu_seqlens != nullptr;
     if (B < 0 || N < 0 || Hq < 1) return FA_ERR_SHAPE;
-    if (d != 128) return FA_ERR_HEADDIM;
+    if (d != 64 && d != 128) return FA_ERR_HEADDIM;
     if (Hkv < 1 || Hq % Hkv != 0) return FA_ERR_GQA;
     if (!(q_scale > 0.f) || !(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(q_scale) ||
         !std::isfinite(k_scale) || !std::isfinite(v_scale))

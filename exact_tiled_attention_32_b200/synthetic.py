@@ -34,7 +34,8 @@ one stream; for the packed batch the sequence lengths are drawn first):
 * dec: one decode step -- 1 query row per (batch, head) against a 32768-key
   cache, B=8, Hq=32, Hkv=8, d=128 (with one row, causal allows every key)
 * c3f8: c3's shape with Q, K, V drawn as N(0,1) times 32 and rounded to
-  nearest-even FP8 E4M3 (per-tensor scale 1/32)
+  nearest-even FP8 E4M3 (per-tensor scale 1/32); c5f8: c5's batch, c2f8:
+  c2's non-causal shape (d = 64), drawn the same way
 * E4M3: 1 sign, 4 exponent bits (bias 7), 3 mantissa bits, subnormals in
   steps of 2^-9; the encoder rounds half to even and saturates at 448
 """
@@ -297,7 +298,7 @@ def packed_from_lengths(name, lens, H, d, causal, seed, Hkv=None) -> Workload:
 
 
 def config(name: str) -> Workload:
-    """The named workloads c1, c2nc, c2c, c3, c4, c5, p3, dec, c3f8, c5f8 (inputs not yet drawn)."""
+    """The named workloads c1, c2nc, c2c, c3, c4, c5, p3, dec, c3f8, c5f8, c2f8 (inputs not yet drawn)."""
     if name == "c1":
         return Workload("c1", 1, 1, 1, 256, 64, False, 1001)
     if name == "c2nc":
@@ -317,6 +318,9 @@ def config(name: str) -> Workload:
     if name == "c3f8":
         # c3 with Q, K, V in E4M3 (per-tensor scale 1/32)
         return Workload("c3f8", 1, 32, 32, 16384, 128, True, 1008, fp8=True)
+    if name == "c2f8":
+        # c2's non-causal shape (d = 64) with E4M3 inputs
+        return Workload("c2f8", 2, 8, 8, 4096, 64, False, 1009, fp8=True)
     if name == "c5f8":
         # c5's packed batch (same lengths) with E4M3 inputs
         w = packed_workload("c5f8", 16, 512, 8192, 16, 128, True, 1005)
@@ -329,4 +333,4 @@ def config(name: str) -> Workload:
     raise KeyError(name)
 
 
-CONFIGS = ("c1", "c2nc", "c2c", "c3", "c4", "c5", "p3", "dec", "c3f8", "c5f8")
+CONFIGS = ("c1", "c2nc", "c2c", "c3", "c4", "c5", "p3", "dec", "c3f8", "c5f8", "c2f8")

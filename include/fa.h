@@ -110,7 +110,7 @@ int fa_fwd_kvcache(const void* q, const void* k, const void* v, void* o, float* 
                    void* stream);
 
 /*
- * fa_fwd_fp8 -- the forward with FP8 inputs (dense batches, d = 128),
+ * fa_fwd_fp8 -- the forward with FP8 inputs (dense batches, d = 64 or 128),
  * asynchronous on `stream`.  "FlashAttention and Chunked Prefill Mechanics"
  * (section 1) names FlashAttention-3's FP8 support; the same tiled algorithm
  * runs on E4M3 operands with fp32 accumulation:
@@ -124,9 +124,12 @@ int fa_fwd_kvcache(const void* q, const void* k, const void* v, void* o, float* 
  * S = Q K^T is computed exactly from the codes (E4M3 products are exact in
  * fp32) and scaled by scale * q_scale * k_scale; the exponentials are rounded
  * to E4M3 for the P V product (relative error <= 2^-4 for P >= 2^-6), O is
- * divided by the fp32 row sum and multiplied by v_scale.  Errors: as fa_fwd;
- * FA_ERR_HEADDIM for d != 128, FA_ERR_SHAPE for a scale that is not finite
- * and positive.
+ * divided by the fp32 row sum and multiplied by v_scale.  At d = 64 each
+ * 64-byte row is read into a 128-byte shared-memory row whose other half the
+ * copy fills with zeros, so the score MMAs run over 128 columns (half of
+ * them zero; the FP8 forward is bound by its exponentials, not its MMAs).
+ * Errors: as fa_fwd; FA_ERR_HEADDIM for d other than 64 or 128, FA_ERR_SHAPE
+ * for a scale that is not finite and positive.
  */
 int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
                int B, int Hq, int Hkv, int N, int d, float scale, int causal,
@@ -137,7 +140,7 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
  * sequences ("Flash Attention" page, "Flash Attention 2 Improvements":
  * variable sequence lengths; "FlashAttention and Chunked Prefill Mechanics",
  * section 1: FP8).  Layouts, masks and errors are those of fa_fwd with
- * cu_seqlens != NULL (q, o [N_total, Hq, 128]; k, v [N_total, Hkv, 128];
+ * cu_seqlens != NULL (q, o [N_total, Hq, d]; k, v [N_total, Hkv, d], d = 64 or 128;
  * lse [Hq, N_total]; cu_seqlens int32 [B + 1] on the device with
  * cu_seqlens[B] == N, checked on the device: FA_ERR_SEQLENS through
  * fa_get_device_status), with E4M3 q, k, v codes and per-tensor scales as

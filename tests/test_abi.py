@@ -180,7 +180,7 @@ def test_fp8_argument_errors_found_on_the_host():
     from exact_tiled_attention_32_b200 import binding as fa
     p = 1 << 20
     call = lambda d=128, qs=1.0, Hkv=2, ptrs=(p,) * 5, B=1: fa.fa_fwd_fp8(*ptrs, B, 4, Hkv, 256, d, 0.1, 1, qs, 1.0, 1.0)
-    assert call(d=64) == fa.FA_ERR_HEADDIM
+    assert call(d=96) == fa.FA_ERR_HEADDIM      # d = 64 and 128 are supported
     assert call(qs=0.0) == fa.FA_ERR_SHAPE
     assert call(qs=float("nan")) == fa.FA_ERR_SHAPE
     assert call(Hkv=3) == fa.FA_ERR_GQA
@@ -195,7 +195,7 @@ def test_fp8_varlen_argument_errors_found_on_the_host():
 
     def call(B=2, d=128, cu=p, ptrs=(p, p, p, p, p)):
         return fa.fa_fwd_fp8_varlen(*ptrs, B, 2, 2, 128, d, 0.1, 1, 1, 1, 1, cu)
-    assert call(d=64) == fa.FA_ERR_HEADDIM
+    assert call(d=96) == fa.FA_ERR_HEADDIM
     assert call(cu=0) == fa.FA_ERR_NULL
     assert call(cu=p + 2) == fa.FA_ERR_ALIGN
     assert call(B=1025) == fa.FA_ERR_SHAPE

@@ -99,38 +99,45 @@ def _check(w, o, lse, rows, what):
 
 
 CASES = [
-    # B, Hq, Hkv, N, causal
-    (1, 2, 2, 256, False),
-    (1, 2, 2, 256, True),
-    (1, 4, 2, 300, True),      # GQA, ragged last tile
-    (2, 2, 1, 1000, True),
-    (1, 3, 3, 129, False),
+    # B, Hq, Hkv, N, causal, d
+    (1, 2, 2, 256, False, 128),
+    (1, 2, 2, 256, True, 128),
+    (1, 4, 2, 300, True, 128),      # GQA, ragged last tile
+    (2, 2, 1, 1000, True, 128),
+    (1, 3, 3, 129, False, 128),
+    # d = 64: 64-byte rows, read into the 128-byte tiles with zero columns
+    (1, 2, 2, 256, False, 64),
+    (1, 4, 2, 300, True, 64),
+    (2, 2, 1, 1000, True, 64),
+    (1, 3, 3, 129, False, 64),
 ]
 
 
-@pytest.mark.parametrize("B,Hq,Hkv,N,causal", CASES)
-def test_fp8_all_rows(B, Hq, Hkv, N, causal):
-    w = syn.Workload("fp8", B, Hq, Hkv, N, 128, causal, 1100 + N, fp8=True).draw()
+@pytest.mark.parametrize("B,Hq,Hkv,N,causal,d", CASES)
+def test_fp8_all_rows(B, Hq, Hkv, N, causal, d):
+    w = syn.Workload("fp8", B, Hq, Hkv, N, d, causal, 1100 + N + d, fp8=True).draw()
     o, lse = _run(w)
-    _check(w, o, lse, np.arange(B * Hq * N), f"fp8 {B},{Hq},{Hkv},{N},{causal}")
+    _check(w, o, lse, np.arange(B * Hq * N), f"fp8 {B},{Hq},{Hkv},{N},{causal},d={d}")
 
 
 PACKED = [
-    # lengths, Hq, Hkv, causal
-    ([300, 1, 129, 0, 513], 4, 2, True),
-    ([300, 1, 129, 0, 513], 4, 2, False),
-    ([128, 256, 77], 2, 1, True),
+    # lengths, Hq, Hkv, causal, d
+    ([300, 1, 129, 0, 513], 4, 2, True, 128),
+    ([300, 1, 129, 0, 513], 4, 2, False, 128),
+    ([128, 256, 77], 2, 1, True, 128),
+    ([300, 1, 129, 0, 513], 4, 2, True, 64),
+    ([128, 256, 77], 2, 1, False, 64),
 ]
 
 
-@pytest.mark.parametrize("lens,Hq,Hkv,causal", PACKED)
-def test_fp8_packed_every_sequence(lens, Hq, Hkv, causal):
+@pytest.mark.parametrize("lens,Hq,Hkv,causal,d", PACKED)
+def test_fp8_packed_every_sequence(lens, Hq, Hkv, causal, d):
     """fa_fwd_fp8_varlen against the oracle, sequence by sequence: each
     sequence's rows are compared with those of the dense problem of that
     sequence alone, under the same per-element and mean bounds."""
     import torch
     from exact_tiled_attention_32_b200 import binding as fa
-    w = syn.packed_from_lengths("fp8p", lens, Hq, 128, causal, 1200 + sum(lens), Hkv=Hkv)
+    w = syn.packed_from_lengths("fp8p", lens, Hq, d, causal, 1200 + sum(lens) + d, Hkv=Hkv)
     w.fp8 = True
     w.draw()
     cu = torch.from_numpy(w.cu_seqlens).cuda()
@@ -144,13 +151,13 @@ def test_fp8_packed_every_sequence(lens, Hq, Hkv, causal):
         if L == 0:
             continue
         a = int(w.cu_seqlens[s_])
-        ws = syn.Workload("fp8seq", 1, Hq, Hkv, L, 128, causal, 0, fp8=True)
+        ws = syn.Workload("fp8seq", 1, Hq, Hkv, L, d, causal, 0, fp8=True)
         ws.q = np.ascontiguousarray(w.q[a:a + L].transpose(1, 0, 2)[None])
         ws.k = np.ascontiguousarray(w.k[a:a + L].transpose(1, 0, 2)[None])
         ws.v = np.ascontiguousarray(w.v[a:a + L].transpose(1, 0, 2)[None])
-        od = o[a:a + L].transpose(1, 0, 2).reshape(-1, 128)
+        od = o[a:a + L].transpose(1, 0, 2).reshape(-1, d)
         ld = lse[:, a:a + L].reshape(-1)
-        _check(ws, od, ld, np.arange(Hq * L), f"fp8 packed {lens} seq {s_}")
+        _check(ws, od, ld, np.arange(Hq * L), f"fp8 packed {lens} seq {s_} d={d}")
 
 
 def test_fp8_varlen_argument_errors():
@@ -158,7 +165,7 @@ def test_fp8_varlen_argument_errors():
     p = 1 << 20
     call = lambda B=2, d=128, cu=p, ptrs=(p, p, p, p, p): fa.fa_fwd_fp8_varlen(*ptrs, B, 2, 2, 128, d, 0.1, 1,
                                                                                1, 1, 1, cu)
-    assert call(d=64) == fa.FA_ERR_HEADDIM
+    assert call(d=96) == fa.FA_ERR_HEADDIM
     assert call(cu=0) == fa.FA_ERR_NULL
     assert call(cu=p + 2) == fa.FA_ERR_ALIGN
     assert call(B=1025) == fa.FA_ERR_SHAPE
@@ -168,7 +175,7 @@ def test_fp8_varlen_argument_errors():
 def test_fp8_argument_errors():
     from exact_tiled_attention_32_b200 import binding as fa
     p = 1 << 20
-    assert fa.fa_fwd_fp8(p, p, p, p, p, 1, 2, 2, 128, 64, 0.1, 1, 1, 1, 1) == fa.FA_ERR_HEADDIM
+    assert fa.fa_fwd_fp8(p, p, p, p, p, 1, 2, 2, 128, 96, 0.1, 1, 1, 1, 1) == fa.FA_ERR_HEADDIM
     assert fa.fa_fwd_fp8(p, p, p, p, p, 1, 2, 2, 128, 128, 0.1, 1, 0, 1, 1) == fa.FA_ERR_SHAPE
     assert fa.fa_fwd_fp8(p, p, p, p, p, 1, 2, 2, 128, 128, 0.1, 1, 1, float("inf"), 1) == fa.FA_ERR_SHAPE
     assert fa.fa_fwd_fp8(p, p, p, p, p, 1, 4, 3, 128, 128, 0.1, 1, 1, 1, 1) == fa.FA_ERR_GQA
@@ -183,6 +190,16 @@ def test_c3f8_sampled_rows():
     o, lse = _run(w)
     rows = sample_rows(w, early=4, tile_stride=16, n_random=4, seed=8)
     _check(w, o, lse, rows, "c3f8")
+
+
+def test_c2f8_sampled_rows():
+    """FP8 at d = 64 on c2's non-causal shape (the bench's c2f8): sampled rows
+    of every head, tile boundaries included."""
+    from fa_util import sample_rows
+    w = syn.config("c2f8").draw()
+    o, lse = _run(w)
+    rows = sample_rows(w, early=4, tile_stride=4, n_random=8, seed=10)
+    _check(w, o, lse, rows, "c2f8")
 
 
 def test_c5f8_sampled_rows():
