@@ -99,3 +99,22 @@ def test_two_streams_at_once():
     for i, (o, lse) in enumerate(outs):
         ref = ra if i % 2 == 0 else rb
         assert torch.equal(o, ref[0]) and torch.equal(lse, ref[1]), i
+
+
+def test_packed_long_sequences_in_head_blocks():
+    """A packed bf16 batch big enough for the dynamic schedule whose long
+    sequences run in blocks of fewer heads than Hq: Hq = 10 on 5 KV heads
+    (GQA groups of 2), sequences of 70,000 and 40,000 tokens (K and V of one
+    KV head above 16 MiB: blocks of one group, 2 heads, so five blocks),
+    shorter ones (all heads in one block), a one-token sequence and an empty
+    one.  Sampled rows of every sequence and head (tile boundaries included)
+    against the oracle."""
+    from fa_util import run_gpu, sample_rows
+    w = syn.packed_from_lengths("headblocks", [70000, 3000, 0, 40000, 512, 1], 10, 128, True, 1404,
+                                Hkv=5).draw()
+    o, lse, st = run_gpu(w)
+    assert st == 0
+    rows = sample_rows(w, early=2, tile_stride=64, n_random=3, seed=11)
+    oo, lo = oracle.attention(w.q, w.k, w.v, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal, w.cu_seqlens,
+                              rows=rows)
+    assert_parity(o[rows], lse[rows], oo, lo, "packed head blocks")
