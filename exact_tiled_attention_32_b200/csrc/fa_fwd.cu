@@ -406,8 +406,10 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, const P
 // compare-and-swap against the value it read; the word changes only through
 // such a swap until it holds this launch's epoch (counting adds are made only
 // after that has been seen), so exactly one swap succeeds and every failed one
-// means the word has moved on.  The counter needs no reset between launches,
-// even after an aborted one.  Launches with few items per CTA (p.dyn = 0), and
+// means the word has moved on.  So a launch needs no reset from the one
+// before it, even an aborted one; a launch that ends normally also returns its
+// word to {epoch, 0} (sched_take), for a replay with the same epoch (a CUDA
+// graph).  Launches with few items per CTA (p.dyn = 0), and
 // every launch of a build with FA_DYN_SCHED=0, follow the static snake of
 // item_of_round instead.
 #ifndef FA_DYN_SCHED
@@ -416,8 +418,13 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, const P
 constexpr int kFeedDepth = 4;
 // the next dynamic item (0, 1, ... in this launch); 0x3fffffff (no item,
 // error recorded) if the word keeps changing under the swap, which only a
-// launch of long ago still running on the same counter could cause
-__device__ __forceinline__ int sched_take(const Params& p, Misc& ms) {
+// launch of long ago still running on the same counter could cause.  Each
+// CTA that takes at all stops after its first take past the last item, so a
+// launch makes exactly `total` takes (`total` - G that succeed and one that
+// fails per CTA, G = min(grid, total) CTAs); the take numbered total - 1 is
+// the last and puts the word back to {epoch, 0}, so that a replay of the
+// same launch (a CUDA graph, same epoch) starts from a clean count.
+__device__ __forceinline__ int sched_take(const Params& p, Misc& ms, int total) {
     const unsigned long long tag = static_cast<unsigned long long>(p.epoch) << 32;
     unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(p.sched);
     for (int tries = 0; static_cast<unsigned>(cur >> 32) != p.epoch; ++tries) {
@@ -434,13 +441,15 @@ __device__ __forceinline__ int sched_take(const Params& p, Misc& ms) {
         // (the only other change an old-epoch word can see) moved it on
         cur = seen == cur ? tag : seen;
     }
-    return static_cast<int>(atomicAdd(p.sched, 1ull) & 0xffffffffull);
+    const int c = static_cast<int>(atomicAdd(p.sched, 1ull) & 0xffffffffull);
+    if (c == total - 1) atomicExch(p.sched, tag);
+    return c;
 }
 // item of round r for this CTA's producer (all items past the first are dynamic)
 __device__ __forceinline__ int producer_item(const Params& p, Misc& ms, int r, int total) {
     if (!FA_DYN_SCHED || !p.dyn) return item_of_round(r);
     if (r == 0) return blockIdx.x;
-    return min(static_cast<int>(gridDim.x) + sched_take(p, ms), total);
+    return min(static_cast<int>(gridDim.x) + sched_take(p, ms, total), total);
 }
 // a consumer warp takes its r-th item (all lanes; one arrival per warp)
 __device__ __forceinline__ bool feed_take(const Params& p, Misc& ms, int r, int& idx) {

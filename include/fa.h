@@ -74,7 +74,10 @@ typedef enum {
  * items (pairs of 128-row query tiles) per SM hands the items to its CTAs
  * through one of those counters; consecutive calls take consecutive counters,
  * each tagged with the call's number, so calls in flight together on
- * different streams do not share one and no counter needs resetting.
+ * different streams do not share one; a launch that completes leaves its
+ * counter at zero, so a captured call (a CUDA graph) can be replayed.  (A
+ * replay of a launch that reported FA_ERR_DEVICE_TIMEOUT may find its counter
+ * not at zero; make a new call instead.)
  *
  * Errors: argument errors are found on the host before any launch and return
  * the codes above.  Errors found on the device (a pipeline wait that ran past

@@ -118,3 +118,35 @@ def test_packed_long_sequences_in_head_blocks():
     oo, lo = oracle.attention(w.q, w.k, w.v, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal, w.cu_seqlens,
                               rows=rows)
     assert_parity(o[rows], lse[rows], oo, lo, "packed head blocks")
+
+
+def test_cuda_graph_replays():
+    """A forward captured in a CUDA graph keeps its counter and epoch on every
+    replay; the launch's last take puts the counter back to zero, so each
+    replay computes every item: five replays give the eager call's output
+    bitwise, on a dense shape (dynamic schedule: 1024 items) and a packed
+    one."""
+    import torch
+    from exact_tiled_attention_32_b200 import binding as fa
+    cases = [syn.Workload("graph-dense", 1, 32, 8, 16384, 64, True, 1405).draw(),
+             syn.packed_from_lengths("graph-packed", [40000, 3000, 20000, 512], 8, 128, True, 1406, Hkv=4).draw()]
+    for w in cases:
+        q, k, v = to_device(w.q), to_device(w.k), to_device(w.v)
+        cu = None if w.cu_seqlens is None else torch.from_numpy(w.cu_seqlens).cuda()
+        ref_o, ref_lse = fa.attention_forward(q, k, v, causal=w.causal, scale=w.scale, cu_seqlens=cu)
+        torch.cuda.synchronize()
+        assert fa.fa_get_device_status() == fa.FA_OK
+        o = torch.empty_like(ref_o)
+        lse = torch.empty_like(ref_lse)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            s = torch.cuda.current_stream()
+            rc = fa.fa_fwd(q, k, v, o, lse, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, w.causal, cu, s)
+        assert rc == fa.FA_OK
+        for i in range(5):
+            o.fill_(7.0)
+            g.replay()
+            torch.cuda.synchronize()
+            assert fa.fa_get_device_status() == fa.FA_OK, (w.name, i)
+            assert torch.equal(o, ref_o) and torch.equal(lse, ref_lse), (w.name, i)
+        del g
