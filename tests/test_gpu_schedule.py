@@ -150,3 +150,57 @@ def test_cuda_graph_replays():
             assert fa.fa_get_device_status() == fa.FA_OK, (w.name, i)
             assert torch.equal(o, ref_o) and torch.equal(lse, ref_lse), (w.name, i)
         del g
+
+
+def test_partials_and_merge_under_the_dynamic_schedule():
+    """fa_fwd_partial on a launch big enough for the dynamic schedule (2048
+    items), over two key halves of a causal problem, merged with
+    fa_merge_partials: O and lse equal fa_fwd's within the forward's
+    tolerances, and sampled rows match the oracle."""
+    import torch
+    from exact_tiled_attention_32_b200 import binding as fa
+    from fa_util import compare, gather, sample_rows
+    w = syn.Workload("partials", 1, 32, 8, 16384, 128, True, 1407).draw()
+    q, k, v = to_device(w.q), to_device(w.k), to_device(w.v)
+    o_ref, lse_ref = fa.attention_forward(q, k, v, causal=True, scale=w.scale)
+    s = torch.cuda.current_stream()
+    half = w.N // 2
+    rows = w.B * w.Hq * w.N
+    o_parts = torch.empty((2, rows, w.d), dtype=torch.float32, device="cuda")
+    lse_parts = torch.empty((2, rows), dtype=torch.float32, device="cuda")
+    # share 0, keys [0, half): row t sees keys 0 .. min(t, half - 1): a causal
+    # call for the rows below half, a non-causal one for the rows from half on
+    kk, vv = k[:, :, :half].contiguous(), v[:, :, :half].contiguous()
+    o0 = o_parts[0].view(w.B, w.Hq, w.N, w.d)
+    l0 = lse_parts[0].view(w.B, w.Hq, w.N)
+    qa, qb = q[:, :, :half].contiguous(), q[:, :, half:].contiguous()
+    oa = torch.empty((w.B, w.Hq, half, w.d), dtype=torch.float32, device="cuda")
+    la = torch.empty((w.B, w.Hq, half), dtype=torch.float32, device="cuda")
+    ob, lb = torch.empty_like(oa), torch.empty_like(la)
+    assert fa.fa_fwd_partial(qa, kk, vv, oa, la, w.B, w.Hq, w.Hkv, half, half, w.d, w.scale, 1, s) == fa.FA_OK
+    assert fa.fa_fwd_partial(qb, kk, vv, ob, lb, w.B, w.Hq, w.Hkv, half, half, w.d, w.scale, 0, s) == fa.FA_OK
+    o0[:, :, :half] = oa
+    o0[:, :, half:] = ob
+    l0[:, :, :half] = la
+    l0[:, :, half:] = lb
+    # share 1: keys [half, N): rows below half see none of them (-inf), rows t >= half see
+    # keys half .. t: a causal chunk of half rows against half keys
+    o1 = o_parts[1].view(w.B, w.Hq, w.N, w.d)
+    l1 = lse_parts[1].view(w.B, w.Hq, w.N)
+    o1[:, :, :half] = 0
+    l1[:, :, :half] = float("-inf")
+    kc, vc = k[:, :, half:].contiguous(), v[:, :, half:].contiguous()
+    assert fa.fa_fwd_partial(qb, kc, vc, ob, lb, w.B, w.Hq, w.Hkv, half, half, w.d, w.scale, 1, s) == fa.FA_OK
+    o1[:, :, half:] = ob
+    l1[:, :, half:] = lb
+    o = torch.empty_like(o_ref)
+    lse = torch.empty_like(lse_ref)
+    assert fa.fa_merge_partials(o_parts, lse_parts, 2, rows, w.d, o, lse, s) == fa.FA_OK
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status() == fa.FA_OK
+    mx, mean, lmx = compare(*gather(w, o, lse), *gather(w, o_ref, lse_ref))
+    assert mx <= 1e-2 and mean <= 1e-3 and lmx <= 1e-3, (mx, mean, lmx)
+    sel = sample_rows(w, early=4, tile_stride=16, n_random=4, seed=12)
+    oo, lo = oracle.attention(w.q, w.k, w.v, w.B, w.Hq, w.Hkv, w.N, w.d, w.scale, True, rows=sel)
+    og, lg = gather(w, o, lse)
+    assert_parity(og[sel], lg[sel], oo, lo, "merged partials")
