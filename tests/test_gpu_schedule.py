@@ -7,9 +7,10 @@ counter is reused (with a new epoch) every ring-length launches and never
 reset.  Which CTA computes which item changes from launch to launch, but each
 item is computed whole by one CTA, so the output must be bitwise the same on
 every launch: checked here over more launches than the ring holds, for
-shapes with far more items than CTAs (causal, uneven item sizes), with fewer
-items than CTAs, packed batches (item count known only on the device), the
-no-allocation entry point (its own, smaller ring) and two streams at once.
+a shape with far more items than CTAs (1,024: the dynamic schedule; causal,
+uneven item sizes), one with fewer items than CTAs (the static schedule), a
+packed batch (item count known only on the device), the no-allocation entry
+point (its own, smaller ring) and two streams at once.
 One launch per shape is also checked against the oracle.
 """
 import pytest
@@ -26,7 +27,8 @@ NOALLOC_RING = 16    # counters of fa_fwd_noalloc
 
 def _shape(name):
     if name == "many-causal":
-        return syn.Workload(name, 2, 16, 4, 4096, 64, True, 1401).draw()
+        # 1,024 items (pairs of query tiles) on 148 SMs: the dynamic schedule
+        return syn.Workload(name, 2, 16, 4, 8192, 64, True, 1401).draw()
     if name == "few-items":
         return syn.Workload(name, 1, 2, 2, 700, 128, False, 1402).draw()
     return syn.packed_from_lengths(name, [1500, 1, 300, 2049, 77, 640], 8, 128, True, 1403, Hkv=2).draw()
